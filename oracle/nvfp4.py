@@ -25,7 +25,9 @@ with them):
   R2 block scale: unsigned E4M3 (bias 7, max 448, subnormals down to 2^-9),
      s = E4M3_RNE_satfinite(fp32(amax_block / fp32(6 * gs))).
   R3 global scale: gs = fp32(amax) / fp32(448 * 6), one per tensor (per module
-     for weights), computed once from a calibration batch for activations.
+     for weights), computed once from a calibration batch for activations;
+     a tensor whose amax is 0 gets gs = 1 (any positive gs quantises it to
+     all-zero codes and scales, and 0 would divide by zero).
   R4 element code: q = E2M1(fp32(x * r)) with r = fp32(1 / fp32(s_dec * gs)),
      using the DECODED (rounded) block scale; an all-zero scale gives code 0.
   R5 dequantised value: e2m1(q) * s_dec * gs, exact in float64.
@@ -117,7 +119,9 @@ def e4m3_encode(t) -> np.ndarray:
 
 # ------------------------------------------------------------ global scale (R3)
 def global_scale(amax) -> np.float32:
-    """gs = fp32(amax) / fp32(2688)."""
+    """gs = fp32(amax) / fp32(2688); 1 for an all-zero tensor (reading R3)."""
+    if F32(amax) == 0:
+        return F32(1.0)
     return F32(F32(amax) / GS_DIVISOR)
 
 
