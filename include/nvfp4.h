@@ -1,0 +1,219 @@
+/*
+ * nvfp4.h -- C ABI of the NVFP4 W4A4 linear layer for B200 (sm_100a).
+ *
+ * The layer is the one every linear layer of the hybrid Gated DeltaNet /
+ * attention model becomes in the paper "Why Gated DeltaNet Survives 4-Bit
+ * Quantization: NVFP4 W4A4 for the Recurrent Half of a Hybrid 27B LLM":
+ * 4-bit weights and 4-bit activations in NVFP4 (nefut abstract, "Minima:
+ * NVFP4 W4A4, quantizing all 496 linear layers"), 16-element block scaling
+ * (bayesiansapien wiki, "The four-part mechanism study", part 1), fused
+ * multi-module projections whose per-module global scales are applied
+ * separately (wiki, "Two practical repairs"; aimodeling, "What engineers
+ * should actually take away"), optionally followed by the GDN gate
+ * nonlinearities (wiki, mechanism study part 2).
+ *
+ * Number format (the pages give none; these are the readings the library
+ * implements):
+ *   codes   E2M1, 4 bits, magnitudes {0,.5,1,1.5,2,3,4,6}, bit 3 = sign.
+ *           Packed two per byte along K: element 2i in the LOW nibble.
+ *   scales  unsigned E4M3 (bias 7, max 448), one per 16 consecutive K elements.
+ *   gs      FP32 global scale per tensor (per module for fused weights),
+ *           gs = fp32(amax) / fp32(2688).
+ *   quantize: s = E4M3_RNE_satfinite(fp32(amax16 / fp32(6 gs)));
+ *             q = E2M1_RNE_satfinite(fp32(x * fp32(1 / fp32(s_dec gs)))),
+ *             all codes 0 when s_dec == 0.
+ *
+ * Memory layouts (all buffers are owned by the caller; the library never
+ * allocates memory and never frees it):
+ *   bf16 inputs   row-major [rows, ld], ld >= K elements, ld % 8 == 0,
+ *                 base 16-byte aligned.
+ *   codes         dense row-major uint8 [rows, K/2] (row stride K/2 bytes),
+ *                 nvfp4_codes_bytes(rows, K) bytes, base 16-byte aligned.
+ *   scales        "128x4 atom" layout consumed by tcgen05 block-scaled MMA:
+ *                 the byte of logical scale S[r, j] (row r, block j = k/16)
+ *                 sits at
+ *                   ((r/128) * (K/64) + j/4) * 512 + (r%32) * 16
+ *                     + ((r/32)%4) * 4 + j%4
+ *                 Rows are padded to a multiple of 128; padding bytes are
+ *                 written as 0 by the quantisers.  nvfp4_scale_bytes(rows, K)
+ *                 bytes, base 16-byte aligned.
+ *   outputs y     row-major [M, ldy], ldy >= N, bf16 (ldy % 8 == 0) or fp32
+ *                 (ldy % 4 == 0), base 16-byte aligned.
+ *
+ * Shapes: K % 64 == 0 and K >= 64; N % 16 == 0; M >= 0 (M == 0 is a no-op).
+ *
+ * Errors: every call returns an nvfp4_status and never throws.  Arguments
+ * are validated on the host before anything is launched; validation
+ * failures return INVALID_ARG / ALIGNMENT / UNSUPPORTED_SHAPE without
+ * touching the GPU.  Launch failures return NVFP4_ERR_CUDA.  Kernels never
+ * trap: every wait inside a kernel is bounded in time, and a wait that runs
+ * out records a device error word and makes the kernel return;
+ * nvfp4_last_device_error() reads (and clears) it.  NaN/Inf inputs are
+ * outside the contract (results undefined, no fault).
+ *
+ * Streams: `stream` is a cudaStream_t (NULL = legacy default stream).  All
+ * calls are asynchronous on that stream except nvfp4_quantize_weight() and
+ * nvfp4_last_device_error(), which synchronise it.
+ */
+#ifndef NVFP4_H_
+#define NVFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#pragma GCC visibility push(default)
+#endif
+
+typedef struct CUstream_st* nvfp4_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = -1,        /* null pointer, bad enum, bad segment table, bad scale */
+  NVFP4_ERR_ALIGNMENT = -2,          /* pointer or leading dimension not 16-byte aligned */
+  NVFP4_ERR_UNSUPPORTED_SHAPE = -3,  /* K % 64, N % 16, ld < K, ... */
+  NVFP4_ERR_CUDA = -4,               /* a CUDA runtime/driver call failed */
+  NVFP4_ERR_TIMEOUT = -5,            /* a bounded in-kernel wait ran out */
+  NVFP4_ERR_UNSUPPORTED_DEVICE = -6  /* current device is not compute capability 10.0 */
+} nvfp4_status;
+
+typedef enum {
+  NVFP4_OP_NONE = 0,      /* y = alpha * acc */
+  NVFP4_OP_SIGMOID = 1,   /* beta = 1 / (1 + exp(-alpha * acc)) */
+  NVFP4_OP_GDN_DECAY = 2  /* g = -exp(A_log[h]) * softplus(alpha * acc + dt_bias[h]) */
+} nvfp4_op;
+
+typedef enum {
+  NVFP4_OUT_BF16 = 0,     /* round to nearest even */
+  NVFP4_OUT_FP32 = 1      /* the fp32 epilogue value before bf16 rounding (test mode) */
+} nvfp4_out_dtype;
+
+/* One module of a fused projection: columns [n_offset, next n_offset) of y.
+ * alpha = fp32(a_gs * w_gs) is applied to that module's columns only -- the
+ * global-scale mismatch repair.  For NVFP4_OP_GDN_DECAY, a_log and dt_bias
+ * are DEVICE pointers to `width` floats each (h = column - n_offset);
+ * otherwise they are ignored. */
+typedef struct {
+  int64_t n_offset;
+  float w_gs;
+  float a_gs;
+  int32_t op;
+  const float* a_log;
+  const float* dt_bias;
+} nvfp4_segment;
+
+#define NVFP4_MAX_SEGMENTS 32
+
+/* Byte sizes of the code and scale buffers for `rows` x K elements. */
+size_t nvfp4_codes_bytes(int64_t rows, int64_t K);
+size_t nvfp4_scale_bytes(int64_t rows, int64_t K);   /* ceil(rows/128)*128 * K/16 */
+
+/* gs = fp32(amax) / fp32(2688) (reading of the calibrated FP32 per-tensor
+ * global scale; host arithmetic, IEEE division).  amax == 0 gives 1: an
+ * all-zero tensor quantises to zero codes and scales under any positive gs. */
+float nvfp4_global_scale(float amax);
+
+/* amax_dev[0] = max |x| over x[0:R, 0:K] (bf16, row stride ldx elements).
+ * amax_dev: caller-owned DEVICE float (the result, overwritten).  Used for
+ * static activation calibration (calibration-only PTQ: aimodeling "Where the
+ * taboo came from") and for weight global scales. */
+nvfp4_status nvfp4_amax(const void* x_bf16, int64_t R, int64_t K, int64_t ldx,
+                        float* amax_dev, nvfp4_stream_t stream);
+
+/* Activation quantisation (step a1): bf16 x [M, K] -> codes [M, K/2] and
+ * scales (atom layout, padding rows zeroed) under the static global scale
+ * a_gs > 0.  All pointers are device pointers. */
+nvfp4_status nvfp4_quantize_act(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
+                                float a_gs, void* codes, void* scales,
+                                nvfp4_stream_t stream);
+
+/* Weight quantisation (step a2, offline).  W [N, K] bf16 is split into
+ * modules at seg_offsets (HOST array of nseg ascending row offsets, first 0,
+ * each a multiple of 16; NULL with nseg == 1 means one module).  Each module
+ * gets its own w_gs = amax(module)/2688, written to w_gs_out (HOST array of
+ * nseg floats), and is quantised with it into the shared codes / scales
+ * buffers (padding rows zeroed).  `workspace` is caller-owned DEVICE scratch
+ * of nvfp4_quantize_weight_workspace_bytes(nseg) bytes (the per-module amax
+ * reduction); its contents on entry do not matter.  Synchronises `stream`. */
+size_t nvfp4_quantize_weight_workspace_bytes(int32_t nseg);
+nvfp4_status nvfp4_quantize_weight(const void* w_bf16, int64_t N, int64_t K, int64_t ldw,
+                                   const int64_t* seg_offsets, int32_t nseg,
+                                   float* w_gs_out, void* codes, void* scales,
+                                   void* workspace, nvfp4_stream_t stream);
+
+/* Block-scaled FP4 x FP4 GEMM (step a3) with a single module (step a4 with
+ * op NONE): y[m, n] = fp32(a_gs * w_gs) * sum_k xhat[m,k] * what[n,k] / (a_gs w_gs),
+ * i.e. the product of the dequantised operands, accumulated in fp32.
+ * a_* describe the quantised activations [M, K], w_* the quantised weights
+ * [N, K] (both K-major, y = x W^T).  Device pointers. */
+nvfp4_status nvfp4_linear(const void* a_codes, const void* a_scales, float a_gs,
+                          const void* w_codes, const void* w_scales, float w_gs,
+                          int64_t M, int64_t N, int64_t K,
+                          void* y, int64_t ldy, nvfp4_out_dtype out_dtype,
+                          nvfp4_stream_t stream);
+
+/* Fused multi-module projection (steps a3 + a4): one GEMM over the
+ * concatenated weight [N, K]; the epilogue applies each module's own alpha
+ * and op (the pages' global-scale mismatch repair, plus the optional GDN
+ * gates).  segs: HOST array of nseg (1..NVFP4_MAX_SEGMENTS) entries, n_offset
+ * strictly ascending, first 0, each a multiple of 16 and < N; copied during
+ * the call.  For M <= 64 the small-M weight-streaming kernel is used (step
+ * a5), otherwise the persistent tensor-core kernel. */
+nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales,
+                                const void* w_codes, const void* w_scales,
+                                int64_t M, int64_t N, int64_t K,
+                                const nvfp4_segment* segs, int32_t nseg,
+                                void* y, int64_t ldy, nvfp4_out_dtype out_dtype,
+                                nvfp4_stream_t stream);
+
+/* MLP glue between the two projections of the MLP pair (not an NVFP4 step):
+ * h[m, j] = bf16(silu(gu[m, j]) * gu[m, H + j]) for j < H, computed in fp32.
+ * gu: bf16 [M, ld_in] with ld_in >= 2H; h: bf16 [M, ld_out], ld_out >= H.
+ * H % 8 == 0. */
+nvfp4_status nvfp4_silu_mul(const void* gu_bf16, int64_t M, int64_t H, int64_t ld_in,
+                            void* h_bf16, int64_t ld_out, nvfp4_stream_t stream);
+
+/* Human-readable status. */
+const char* nvfp4_status_string(nvfp4_status status);
+
+/* Synchronises `stream`, then reads and clears the device error word that
+ * bounded in-kernel waits set when they run out.  Returns NVFP4_OK or
+ * NVFP4_ERR_TIMEOUT (info, if non-NULL, receives the raw word: bits 63..48
+ * site code, 47..32 role, 31..0 block index), or NVFP4_ERR_CUDA. */
+nvfp4_status nvfp4_last_device_error(nvfp4_stream_t stream, uint64_t* info);
+
+/* Kernel-path selection for tests: 0 = automatic (M <= 64 -> small-M
+ * kernel), 1 = always the persistent tensor-core kernel, 2 = always the
+ * small-M kernel (requires M <= 64).  Process-wide. */
+nvfp4_status nvfp4_set_gemm_path(int32_t path);
+
+/* Time limit of every bounded in-kernel wait, in nanoseconds (default 2e9;
+ * also read once from the environment variable NVFP4_SPIN_LIMIT_NS). */
+nvfp4_status nvfp4_set_wait_limit_ns(uint64_t limit_ns);
+
+/* ---- test entry points (conversion checks; not part of the layer) ------ */
+
+/* out[i] = E2M1 code of in[i] (fp32 -> E2M1, RNE, satfinite), with the same
+ * device conversion the activation quantiser uses.  Device pointers. */
+nvfp4_status nvfp4_test_e2m1(const float* in, uint8_t* out, int64_t n, nvfp4_stream_t stream);
+/* out[i] = unsigned E4M3 code of in[i] >= 0 (RNE, satfinite), the quantiser's
+ * block-scale conversion.  Device pointers. */
+nvfp4_status nvfp4_test_e4m3(const float* in, uint8_t* out, int64_t n, nvfp4_stream_t stream);
+/* Launches one CTA that waits on an mbarrier nobody arrives on, with the
+ * wait limit set to limit_ns; returns what nvfp4_last_device_error reports
+ * (NVFP4_ERR_TIMEOUT when the bound works).  Synchronises `stream`. */
+nvfp4_status nvfp4_test_wait_timeout(uint64_t limit_ns, nvfp4_stream_t stream);
+
+#if defined(__GNUC__)
+#pragma GCC visibility pop
+#endif
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H_ */

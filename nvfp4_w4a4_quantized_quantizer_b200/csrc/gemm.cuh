@@ -1,0 +1,514 @@
+// gemm.cuh -- block-scaled FP4 x FP4 GEMM with the segment epilogue.
+//
+// y[m, n] = op_s( alpha_s * sum_k e2m1(A[m,k]) sa[m,k/16] e2m1(W[n,k]) sw[n,k/16] )
+// for column n in module s.  This is the NVFP4 W4A4 linear layer of the
+// paper "Why Gated DeltaNet Survives 4-Bit Quantization" (nefut abstract:
+// all linear layers W4A4), with the per-module global-scale repair of fused
+// projections (bayesiansapien wiki, "Two practical repairs") and the GDN
+// gates (wiki, mechanism study part 2) in the epilogue.
+//
+// Two kernels:
+//   k_gemm_tc     persistent, warp-specialised, one 128 x 256 output tile at
+//                 a time per CTA (1 CTA per SM).  Warp 0 streams A/B codes
+//                 with TMA (128-byte swizzle) and the scale atoms with bulk
+//                 copies into a 4-stage shared-memory ring; warp 1 copies the
+//                 scale atoms into TMEM (tcgen05.cp) and issues
+//                 tcgen05.mma.kind::mxf4nvf4 (K = 64 per instruction) into a
+//                 128 x 256 fp32 TMEM accumulator; warps 2-9 drain the
+//                 accumulator (each lane = one row, 128 columns), release it
+//                 to the MMA warp, then apply alpha / op and store.
+//   k_gemm_small  M <= 64 (decode shapes): operands swapped so the weight
+//                 rows fill the 128-row MMA side and the tokens are the MMA N
+//                 dimension (16/32/64); one CTA per 128 weight rows streams
+//                 the whole K range through a 6-stage ring.
+// Every wait is bounded (mbar_wait); a wait that runs out records the
+// device error word, raises a CTA-wide abort flag and the kernel returns
+// after draining its own copies and MMAs and freeing TMEM.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace nvfp4 {
+
+constexpr int MAX_SEG = 32;
+
+struct SegTable {
+  int nseg;
+  int n_off[MAX_SEG + 1];  // n_off[nseg] = N
+  float alpha[MAX_SEG];
+  int op[MAX_SEG];
+  const float* a_log[MAX_SEG];
+  const float* dt_bias[MAX_SEG];
+};
+
+struct GemmArgs {
+  const uint8_t* sfa;  // activation (or, swapped, token) scale atoms
+  const uint8_t* sfb;  // weight scale atoms
+  int M, N, K;
+  void* y;
+  int64_t ldy;
+  int out_fp32;
+  uint64_t wait_ns;
+};
+
+// ------------------------------------------------------------- epilogue op
+__device__ __forceinline__ float apply_op(float v, int op, const float* a_log,
+                                          const float* dt_bias, int h) {
+  if (op == 1) return 1.0f / (1.0f + expf(-v));
+  if (op == 2) {
+    const float z = v + __ldg(dt_bias + h);
+    const float sp = fmaxf(z, 0.0f) + log1pf(expf(-fabsf(z)));
+    return -expf(__ldg(a_log + h)) * sp;
+  }
+  return v;
+}
+
+// Advance `seg` so that n lies in [n_off[seg], n_off[seg+1]).
+__device__ __forceinline__ int seg_advance(const SegTable& t, int seg, int n) {
+  while (seg + 1 < t.nseg && n >= t.n_off[seg + 1]) ++seg;
+  return seg;
+}
+
+// ============================================================ k_gemm_tc
+namespace tc {
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 256;                 // fp4 elements per stage (128 bytes per row)
+constexpr int BKB = BK / 2;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BKB;       // 16 KB
+constexpr int B_BYTES = BN * BKB;       // 32 KB
+constexpr int SFA_BYTES = 4 * 512;      // 4 atoms (K = 64 each) x 128 rows
+constexpr int SFB_BYTES = 2 * 4 * 512;  // 2 row blocks of 128
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 54 KB
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 32 * (2 + EPI_WARPS);
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC_COL = 0;
+constexpr uint32_t SFA_COL = 256;       // 4 MMAs x 4 columns
+constexpr uint32_t SFB_COL = 272;       // 4 MMAs x 8 columns
+constexpr int BAR_BYTES = 256;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
+}  // namespace tc
+
+__global__ void __launch_bounds__(tc::THREADS, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const GemmArgs g, const __grid_constant__ SegTable seg) {
+  using namespace tc;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  // bars: full[STAGES], empty[STAGES], tmem_full, tmem_empty, drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 3);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int num_m = (g.M + BM - 1) / BM;
+  const int num_n = (g.N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  const int num_kt = (g.K + BK - 1) / BK;
+  const int64_t kb4 = g.K / 64;            // scale atoms per 128-row block
+  const int sfb_blocks = (g.N + 127) / 128;
+
+  auto full_bar = [&](int s) { return smem_addr(bars + s); };
+  auto empty_bar = [&](int s) { return smem_addr(bars + STAGES + s); };
+  const uint32_t tmem_full = smem_addr(bars + 2 * STAGES);
+  const uint32_t tmem_empty = smem_addr(bars + 2 * STAGES + 1);
+  const uint32_t drain_bar = smem_addr(bars + 2 * STAGES + 2);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(tmem_full, 1);
+    mbar_init(tmem_empty, EPI_WARPS);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_a = policy_evict_last();
+      const uint64_t pol_b = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      int64_t issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int mb = tile % num_m;
+        const int nb = tile / num_m;
+        for (int kt = 0; kt < num_kt; ++kt) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, g.wait_ns, abort_flag)) {
+            if (!*abort_flag) record_error(SITE_PRODUCER_EMPTY, 0);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          const int nk = min(4, (g.K - kt * BK) / 64);
+          const int nb0 = nb * 2;
+          const int nsfb = min(2, sfb_blocks - nb0);
+          const uint32_t bytes = A_BYTES + B_BYTES + nk * 512 * (1 + nsfb);
+          uint8_t* st = smem + stage * STAGE_BYTES;
+          mbar_arrive_expect_tx(full_bar(stage), bytes);
+          tma_load_2d(smem_addr(st), &tmA, kt * BKB, mb * BM, full_bar(stage), pol_a);
+          tma_load_2d(smem_addr(st + A_BYTES), &tmB, kt * BKB, nb * BN, full_bar(stage), pol_b);
+          bulk_load(smem_addr(st + A_BYTES + B_BYTES), g.sfa + (mb * kb4 + kt * 4) * 512,
+                    nk * 512, full_bar(stage), pol_a);
+          for (int j = 0; j < nsfb; ++j)
+            bulk_load(smem_addr(st + A_BYTES + B_BYTES + SFA_BYTES + j * 2048),
+                      g.sfb + ((nb0 + j) * kb4 + kt * 4) * 512, nk * 512, full_bar(stage), pol_b);
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // every copy issued must land before the CTA may exit
+      for (int s = 0; s < STAGES && s < issued; ++s) {
+        const int64_t uses = (issued - 1 - s) / STAGES + 1;
+        if (!mbar_wait(full_bar(s), static_cast<uint32_t>((uses - 1) & 1), g.wait_ns, nullptr))
+          record_error(SITE_DRAIN, 0);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // -------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_mxf4nvf4(BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+        if (!mbar_wait(tmem_empty, static_cast<uint32_t>((local & 1) ^ 1), g.wait_ns, abort_flag)) {
+          if (!*abort_flag) record_error(SITE_MMA_TMEM_EMPTY, 1);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        for (int kt = 0; kt < num_kt; ++kt) {
+          if (!mbar_wait(full_bar(stage), phase, g.wait_ns, abort_flag)) {
+            if (!*abort_flag) record_error(SITE_MMA_FULL, 1);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nk = min(4, (g.K - kt * BK) / 64);
+          const uint8_t* st = smem + stage * STAGE_BYTES;
+          const uint32_t a_s = smem_addr(st);
+          const uint32_t b_s = smem_addr(st + A_BYTES);
+          const uint32_t sfa_s = smem_addr(st + A_BYTES + B_BYTES);
+          const uint32_t sfb_s = sfa_s + SFA_BYTES;
+          for (int kk = 0; kk < nk; ++kk) {
+            tmem_cp_32x128b_x4(tmem_base + SFA_COL + 4 * kk, desc_sf_atom(sfa_s + kk * 512));
+            tmem_cp_32x128b_x4(tmem_base + SFB_COL + 8 * kk, desc_sf_atom(sfb_s + kk * 512));
+            tmem_cp_32x128b_x4(tmem_base + SFB_COL + 8 * kk + 4,
+                               desc_sf_atom(sfb_s + 2048 + kk * 512));
+          }
+          const uint64_t adesc = desc_kmajor_sw128(a_s);
+          const uint64_t bdesc = desc_kmajor_sw128(b_s);
+          for (int kk = 0; kk < nk; ++kk) {
+            // K = 64 fp4 = 32 bytes: advance the start address inside the swizzle atom
+            mma_mxf4nvf4(tmem_base + ACC_COL, adesc + 2 * kk, bdesc + 2 * kk, idesc,
+                         tmem_base + SFA_COL + 4 * kk, tmem_base + SFB_COL + 8 * kk,
+                         (kt | kk) != 0);
+          }
+          tc_commit(empty_bar(stage));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(tmem_full);
+      }
+      // all issued tensor-core work must finish before TMEM is freed
+      tc_commit(drain_bar);
+      if (!mbar_wait(drain_bar, 0, g.wait_ns, nullptr)) record_error(SITE_DRAIN, 1);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------- epilogue
+    const int q = warp & 3;               // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;     // columns [128*half, 128*half + 128)
+    const int row_in_tile = q * 32 + lane;
+    int local = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+      const int mb = tile % num_m;
+      const int nb = tile / num_m;
+      if (!mbar_wait(tmem_full, static_cast<uint32_t>(local & 1), g.wait_ns, abort_flag)) {
+        if (!*abort_flag) record_error(SITE_EPI_TMEM_FULL, 2 + (warp - 2));
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      uint32_t v[128];
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ACC_COL + half * 128;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_x32(taddr + c * 32, v + c * 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tmem_empty);
+
+      const int64_t gm = static_cast<int64_t>(mb) * BM + row_in_tile;
+      if (gm < g.M) {
+        const int n0 = nb * BN + half * 128;
+        int s = seg_advance(seg, 0, n0);
+#pragma unroll
+        for (int grp = 0; grp < 8; ++grp) {
+          const int n = n0 + grp * 16;
+          if (n < g.N) {
+            s = seg_advance(seg, s, n);
+            const float alpha = seg.alpha[s];
+            const int op = seg.op[s];
+            const int h0 = n - seg.n_off[s];
+            float o[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float a = __fmul_rn(alpha, __uint_as_float(v[grp * 16 + i]));
+              o[i] = (op == 0) ? a : apply_op(a, op, seg.a_log[s], seg.dt_bias[s], h0 + i);
+            }
+            if (g.out_fp32) {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.y) + gm * g.ldy + n);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+            } else {
+              uint32_t w[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const __nv_bfloat162 p = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);
+                w[i] = *reinterpret_cast<const uint32_t*>(&p);
+              }
+              uint4* dst =
+                  reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.y) + gm * g.ldy + n);
+              dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+              dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+// ========================================================== k_gemm_small
+namespace sm {
+constexpr int BW = 128;                 // weight rows per CTA (MMA M)
+constexpr int BK = 256;
+constexpr int BKB = BK / 2;
+constexpr int STAGES = 6;
+constexpr int W_BYTES = BW * BKB;       // 16 KB
+constexpr int SFW_BYTES = 4 * 512;
+constexpr int SFX_BYTES = 4 * 512;
+constexpr int EPI_WARPS = 4;
+constexpr int THREADS = 32 * (2 + EPI_WARPS);
+constexpr uint32_t TMEM_COLS = 128;
+constexpr uint32_t ACC_COL = 0;         // NT columns
+constexpr uint32_t SFW_COL = 64;        // 4 MMAs x 4 columns
+constexpr uint32_t SFX_COL = 80;        // 4 MMAs x 4 columns
+constexpr int BAR_BYTES = 256;
+template <int NT>
+struct Cfg {
+  static constexpr int X_BYTES = NT * BKB;   // NT rows x 128 bytes
+  static constexpr int STAGE_BYTES = W_BYTES + X_BYTES + SFW_BYTES + SFX_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+  static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
+};
+}  // namespace sm
+
+// tmW: weight codes [N, K/2]; tmX: token codes [M, K/2].  D (TMEM) is
+// [128 weight rows] x [NT tokens]; y[token, n] is written transposed back.
+template <int NT>
+__global__ void __launch_bounds__(sm::THREADS, 1)
+    k_gemm_small(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                 const GemmArgs g, const __grid_constant__ SegTable seg) {
+  using namespace sm;
+  using C = Cfg<NT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
+  // bars: full[STAGES], empty[STAGES], acc_full, drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int wt = blockIdx.x;              // weight tile: rows [128 wt, 128 wt + 128)
+  const int num_kt = (g.K + BK - 1) / BK;
+  const int64_t kb4 = g.K / 64;
+
+  auto full_bar = [&](int s) { return smem_addr(bars + s); };
+  auto empty_bar = [&](int s) { return smem_addr(bars + STAGES + s); };
+  const uint32_t acc_full = smem_addr(bars + 2 * STAGES);
+  const uint32_t drain_bar = smem_addr(bars + 2 * STAGES + 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tensormap(&tmW);
+    prefetch_tensormap(&tmX);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();   // weights stream through once
+      const uint64_t pol_x = policy_evict_last();    // tokens are re-read by every CTA
+      int stage = 0;
+      uint32_t phase = 0;
+      int64_t issued = 0;
+      for (int kt = 0; kt < num_kt; ++kt) {
+        if (!mbar_wait(empty_bar(stage), phase ^ 1u, g.wait_ns, abort_flag)) {
+          if (!*abort_flag) record_error(SITE_PRODUCER_EMPTY, 0);
+          *abort_flag = 1;
+          break;
+        }
+        const int nk = min(4, (g.K - kt * BK) / 64);
+        const uint32_t bytes = W_BYTES + C::X_BYTES + 2 * nk * 512;
+        uint8_t* st = smem + stage * C::STAGE_BYTES;
+        mbar_arrive_expect_tx(full_bar(stage), bytes);
+        tma_load_2d(smem_addr(st), &tmW, kt * BKB, wt * BW, full_bar(stage), pol_w);
+        tma_load_2d(smem_addr(st + W_BYTES), &tmX, kt * BKB, 0, full_bar(stage), pol_x);
+        bulk_load(smem_addr(st + W_BYTES + C::X_BYTES), g.sfb + (wt * kb4 + kt * 4) * 512, nk * 512,
+                  full_bar(stage), pol_w);
+        bulk_load(smem_addr(st + W_BYTES + C::X_BYTES + SFW_BYTES), g.sfa + (kt * 4) * 512,
+                  nk * 512, full_bar(stage), pol_x);
+        ++issued;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      for (int s = 0; s < STAGES && s < issued; ++s) {
+        const int64_t uses = (issued - 1 - s) / STAGES + 1;
+        if (!mbar_wait(full_bar(s), static_cast<uint32_t>((uses - 1) & 1), g.wait_ns, nullptr))
+          record_error(SITE_DRAIN, 0);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_mxf4nvf4(BW, NT);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int kt = 0; kt < num_kt; ++kt) {
+        if (!mbar_wait(full_bar(stage), phase, g.wait_ns, abort_flag)) {
+          if (!*abort_flag) record_error(SITE_MMA_FULL, 1);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int nk = min(4, (g.K - kt * BK) / 64);
+        const uint8_t* st = smem + stage * C::STAGE_BYTES;
+        const uint32_t w_s = smem_addr(st);
+        const uint32_t x_s = smem_addr(st + W_BYTES);
+        const uint32_t sfw_s = smem_addr(st + W_BYTES + C::X_BYTES);
+        const uint32_t sfx_s = sfw_s + SFW_BYTES;
+        for (int kk = 0; kk < nk; ++kk) {
+          tmem_cp_32x128b_x4(tmem_base + SFW_COL + 4 * kk, desc_sf_atom(sfw_s + kk * 512));
+          tmem_cp_32x128b_x4(tmem_base + SFX_COL + 4 * kk, desc_sf_atom(sfx_s + kk * 512));
+        }
+        const uint64_t wdesc = desc_kmajor_sw128(w_s);
+        const uint64_t xdesc = desc_kmajor_sw128(x_s);
+        for (int kk = 0; kk < nk; ++kk)
+          mma_mxf4nvf4(tmem_base + ACC_COL, wdesc + 2 * kk, xdesc + 2 * kk, idesc,
+                       tmem_base + SFW_COL + 4 * kk, tmem_base + SFX_COL + 4 * kk, (kt | kk) != 0);
+        tc_commit(empty_bar(stage));
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (ok) tc_commit(acc_full);
+      tc_commit(drain_bar);
+      if (!mbar_wait(drain_bar, 0, g.wait_ns, nullptr)) record_error(SITE_DRAIN, 1);
+    }
+    __syncwarp();
+  } else {
+    const int q = warp & 3;
+    const int n = wt * BW + q * 32 + lane;   // output feature of this lane
+    if (mbar_wait(acc_full, 0, g.wait_ns, abort_flag)) {
+      tc_fence_after();
+      uint32_t v[NT];
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ACC_COL;
+#pragma unroll
+      for (int c = 0; c < NT / 16; ++c) {
+        uint32_t (&r)[16] = *reinterpret_cast<uint32_t(*)[16]>(v + 16 * c);
+        tmem_ld_x16(taddr + 16 * c, r);
+      }
+      tmem_wait_ld();
+      if (n < g.N) {
+        const int s = seg_advance(seg, 0, n);
+        const float alpha = seg.alpha[s];
+        const int op = seg.op[s];
+        const int h = n - seg.n_off[s];
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          if (j < g.M) {
+            const float a = __fmul_rn(alpha, __uint_as_float(v[j]));
+            const float o = (op == 0) ? a : apply_op(a, op, seg.a_log[s], seg.dt_bias[s], h);
+            if (g.out_fp32)
+              static_cast<float*>(g.y)[static_cast<int64_t>(j) * g.ldy + n] = o;
+            else
+              static_cast<__nv_bfloat16*>(g.y)[static_cast<int64_t>(j) * g.ldy + n] =
+                  __float2bfloat16_rn(o);
+          }
+        }
+      }
+    } else {
+      if (!*abort_flag) record_error(SITE_EPI_TMEM_FULL, warp);
+      *abort_flag = 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+}  // namespace nvfp4

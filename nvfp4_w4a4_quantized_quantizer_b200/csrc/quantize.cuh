@@ -1,0 +1,266 @@
+// quantize.cuh -- NVFP4 quantisation kernels (HBM-bound).
+//
+// k_quantize: bf16 rows -> packed E2M1 codes + UE4M3 block scales written
+// directly in the 128x4 atom layout that tcgen05 block-scaled MMA consumes.
+// The arithmetic is the NVFP4 16-element block scaling of the paper "Why
+// Gated DeltaNet Survives 4-Bit Quantization" (bayesiansapien wiki, "The
+// four-part mechanism study", part 1), with these steps per block:
+//   c     = fp32(6 * gs)
+//   s     = E4M3_RNE_satfinite(fp32(amax16 / c))
+//   r     = fp32(1 / fp32(s_dec * gs))       (0 when s_dec == 0)
+//   q_k   = E2M1_RNE_satfinite(fp32(x_k * r))
+// Every rounding is an explicit _rn intrinsic or a .rn conversion, so the
+// compiler cannot contract or reorder it.
+//
+// Work mapping: one warp handles one (row, 256-element chunk) unit per step:
+// lane t loads elements 8t..8t+7 (one 16-byte load; the warp reads 512
+// contiguous bytes), lanes 2b and 2b+1 form 16-element block b and exchange
+// their partial amax with one shuffle, each lane writes 4 code bytes (the
+// warp writes 128 contiguous bytes), and every 8th lane gathers the four
+// scale bytes of blocks j..j+3 (contiguous in the atom layout) into one
+// 32-bit store.  Each warp keeps UNROLL units in flight.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace nvfp4 {
+
+// ------------------------------------------------------------ conversions
+// Eight fp32 values -> eight E2M1 codes packed in 32 bits, element e in
+// bits 4e..4e+3 (even elements in the low nibble of each byte).  The PTX
+// conversion puts its first source in the high nibble.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&v)[8]) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  return out;
+}
+
+// fp32 (>= 0) -> unsigned E4M3 code, round to nearest even, saturating at 448.
+__device__ __forceinline__ uint32_t cvt_e4m3(float v) {
+  uint16_t out;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(0.0f), "f"(v));
+  return static_cast<uint32_t>(out) & 0xFFu;
+}
+
+// Unsigned E4M3 code -> its exact fp32 value, built from the bit fields.
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+  const uint32_t e = (code >> 3) & 0xFu;
+  const uint32_t m = code & 7u;
+  if (e == 0) return static_cast<float>(m) * 0.001953125f;  // m * 2^-9, exact
+  return __uint_as_float(((e + 120u) << 23) | (m << 20));   // (1 + m/8) * 2^(e-7)
+}
+
+// Byte offset of logical scale S[r, j] inside the 128x4 atom layout.
+__host__ __device__ __forceinline__ uint64_t sf_offset(int64_t r, int64_t j, int64_t K) {
+  const int64_t kb4 = K / 64;  // atoms per 128-row block along K
+  return static_cast<uint64_t>(((r >> 7) * kb4 + (j >> 2)) * 512 + (r & 31) * 16 +
+                               ((r >> 5) & 3) * 4 + (j & 3));
+}
+
+struct QuantArgs {
+  const __nv_bfloat16* x;  // first row of the range
+  int64_t rows;            // rows in the range
+  int64_t K;
+  int64_t ldx;             // elements
+  int64_t row0;            // logical row of x[0] in the code / scale buffers
+  float gs;
+  uint8_t* codes;          // base of the full code buffer [*, K/2]
+  uint8_t* scales;         // base of the full scale buffer (atom layout)
+  int64_t pad_from;        // zero scale rows [pad_from, pad_to)
+  int64_t pad_to;
+};
+
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+constexpr int QUANT_THREADS = 256;
+constexpr int QUANT_UNROLL = 4;
+
+__global__ void __launch_bounds__(QUANT_THREADS) k_quantize(const QuantArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t gwarp = (static_cast<int64_t>(blockIdx.x) * QUANT_THREADS + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * QUANT_THREADS) >> 5;
+  const int64_t chunks = (a.K + 255) / 256;
+  const int64_t units = a.rows * chunks;
+  const float c = __fmul_rn(6.0f, a.gs);
+  const int64_t code_ld = a.K / 2;
+
+  for (int64_t u0 = gwarp; u0 < units; u0 += nwarps * QUANT_UNROLL) {
+    uint4 raw[QUANT_UNROLL];
+    int64_t row[QUANT_UNROLL];
+    int kidx[QUANT_UNROLL];
+    bool valid[QUANT_UNROLL];
+#pragma unroll
+    for (int i = 0; i < QUANT_UNROLL; ++i) {
+      const int64_t u = u0 + i * nwarps;
+      const bool in = u < units;
+      const int64_t r = in ? u / chunks : 0;
+      const int ch = in ? static_cast<int>(u - r * chunks) : 0;
+      row[i] = r;
+      kidx[i] = ch * 256 + lane * 8;
+      valid[i] = in && kidx[i] < a.K;
+      raw[i] = valid[i] ? ld_stream_v4(a.x + r * a.ldx + kidx[i]) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < QUANT_UNROLL; ++i) {
+      float f[8];
+      bf16x8_to_f32(raw[i], f);
+      float amax = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      const uint32_t s = cvt_e4m3(__fdiv_rn(amax, c));
+      const float sdec = e4m3_value(s);
+      const float r = (sdec == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(sdec, a.gs));
+      float y[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[e] = __fmul_rn(f[e], r);
+      uint32_t packed = cvt_e2m1x8(y);
+      if (sdec == 0.0f) packed = 0;
+      // scale bytes of blocks 4g..4g+3 (lanes 8g, 8g+2, 8g+4, 8g+6) -> lane 8g
+      const uint32_t s1 = __shfl_down_sync(0xffffffffu, s, 2);
+      const uint32_t s2 = __shfl_down_sync(0xffffffffu, s, 4);
+      const uint32_t s3 = __shfl_down_sync(0xffffffffu, s, 6);
+      if (valid[i]) {
+        const int64_t grow = a.row0 + row[i];
+        *reinterpret_cast<uint32_t*>(a.codes + grow * code_ld + kidx[i] / 2) = packed;
+        if ((lane & 7) == 0) {
+          const uint32_t word = s | (s1 << 8) | (s2 << 16) | (s3 << 24);
+          *reinterpret_cast<uint32_t*>(a.scales + sf_offset(grow, kidx[i] / 16, a.K)) = word;
+        }
+      }
+    }
+  }
+
+  // zero the scale bytes of the padding rows (rows past the last real row
+  // inside the last 128-row block)
+  const int64_t kb = a.K / 16;
+  const int64_t pad_words = (a.pad_to - a.pad_from) * (kb / 4);
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * QUANT_THREADS + threadIdx.x; t < pad_words;
+       t += static_cast<int64_t>(gridDim.x) * QUANT_THREADS) {
+    const int64_t r = a.pad_from + t / (kb / 4);
+    const int64_t j = (t % (kb / 4)) * 4;
+    *reinterpret_cast<uint32_t*>(a.scales + sf_offset(r, j, a.K)) = 0u;
+  }
+}
+
+// ------------------------------------------------------------------- amax
+// out[0] = max |x| over rows x K.  `out` must hold 0.0f on entry (the host
+// clears it on the same stream); non-negative floats order like their bit
+// patterns, so an integer atomicMax on the bits is an exact float max.
+constexpr int AMAX_THREADS = 256;
+
+__global__ void __launch_bounds__(AMAX_THREADS) k_amax(const __nv_bfloat16* __restrict__ x,
+                                                       int64_t rows, int64_t K, int64_t ldx,
+                                                       float* out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t gwarp = (static_cast<int64_t>(blockIdx.x) * AMAX_THREADS + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * AMAX_THREADS) >> 5;
+  float m = 0.0f;
+  for (int64_t r = gwarp; r < rows; r += nwarps) {
+    const __nv_bfloat16* p = x + r * ldx;
+    for (int64_t k = lane * 8; k < K; k += 256) {
+      float f[8];
+      bf16x8_to_f32(ld_stream_v4(p + k), f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ float red[AMAX_THREADS / 32];
+  if (lane == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float b = 0.0f;
+    for (int i = 0; i < AMAX_THREADS / 32; ++i) b = fmaxf(b, red[i]);
+    atomicMax(reinterpret_cast<unsigned int*>(out), __float_as_uint(b));
+  }
+}
+
+// ------------------------------------------------------- MLP glue (SiLU*up)
+constexpr int SILU_THREADS = 256;
+
+__global__ void __launch_bounds__(SILU_THREADS) k_silu_mul(const __nv_bfloat16* __restrict__ gu,
+                                                           int64_t M, int64_t H, int64_t ld_in,
+                                                           __nv_bfloat16* __restrict__ h,
+                                                           int64_t ld_out) {
+  const int64_t vec_per_row = H / 8;
+  const int64_t total = M * vec_per_row;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * SILU_THREADS + threadIdx.x; t < total;
+       t += static_cast<int64_t>(gridDim.x) * SILU_THREADS) {
+    const int64_t m = t / vec_per_row;
+    const int64_t j = (t - m * vec_per_row) * 8;
+    float g[8], u[8];
+    bf16x8_to_f32(ld_stream_v4(gu + m * ld_in + j), g);
+    bf16x8_to_f32(ld_stream_v4(gu + m * ld_in + H + j), u);
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float a0 = __fmul_rn(__fdiv_rn(g[2 * e], 1.0f + expf(-g[2 * e])), u[2 * e]);
+      const float a1 = __fmul_rn(__fdiv_rn(g[2 * e + 1], 1.0f + expf(-g[2 * e + 1])), u[2 * e + 1]);
+      const __nv_bfloat162 p = __floats2bfloat162_rn(a0, a1);
+      w[e] = *reinterpret_cast<const uint32_t*>(&p);
+    }
+    *reinterpret_cast<uint4*>(h + m * ld_out + j) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// ------------------------------------------------------------ test kernels
+__global__ void k_test_e2m1(const float* in, uint8_t* out, int64_t n) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+  {
+    const float v[8] = {in[i], 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    out[i] = static_cast<uint8_t>(cvt_e2m1x8(v) & 0xFu);
+  }
+}
+
+__global__ void k_test_e4m3(const float* in, uint8_t* out, int64_t n) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    out[i] = static_cast<uint8_t>(cvt_e4m3(in[i]));
+}
+
+// One CTA waits on an mbarrier that nothing arrives on; the bounded wait
+// must give up after limit_ns and record the error word.
+__global__ void k_test_wait_timeout(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_addr(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (!mbar_wait(smem_addr(&bar), 0, limit_ns, &abort_flag)) record_error(SITE_TEST, 0);
+  }
+  __syncthreads();
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,176 @@
+"""GPU parity: block-scaled FP4 GEMM (both kernels) vs the float64 oracle.
+
+Operands are either built directly in the device layout from random codes
+and scales (so the GEMM is checked independently of the quantiser) or come
+from the quantisers.  Bar: fp32 output within max |err| <= 1e-3 rms and
+relative Frobenius <= 1e-5 of the float64 product of the dequantised
+operands; bf16 output = bf16_RNE(fp32 output) exactly.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+import nvfp4_w4a4_quantized_quantizer_b200 as nv
+from tests import _helpers as H
+
+pytestmark = pytest.mark.gpu
+
+LARGE, SMALL, AUTO = 1, 2, 0
+
+
+@pytest.fixture(autouse=True)
+def _reset_path():
+    yield
+    nv.nvfp4_set_gemm_path(AUTO)
+
+
+def sf_pack(logical: np.ndarray, rows: int, K: int) -> np.ndarray:
+    """Logical [rows, K/16] scale codes -> atom-layout bytes (padding rows 0)."""
+    padded = (rows + 127) // 128 * 128
+    buf = np.zeros(padded * K // 16, np.uint8)
+    kb = K // 16
+    r = np.arange(rows)[:, None]
+    j = np.arange(kb)[None, :]
+    off = ((r // 128) * (kb // 4) + j // 4) * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + j % 4
+    buf[off] = logical
+    return buf
+
+
+def pack(codes: np.ndarray) -> np.ndarray:
+    return ((codes[:, 0::2] & 0xF) | ((codes[:, 1::2] & 0xF) << 4)).astype(np.uint8)
+
+
+def dev_operands(codes, scales, rows, K):
+    c = torch.from_numpy(pack(codes)).cuda()
+    s = torch.from_numpy(sf_pack(scales, rows, K)).cuda()
+    return c, s
+
+
+def run(path, ac, as_, a_gs, wc, ws, w_gs, M, N, K):
+    nv.nvfp4_set_gemm_path(path)
+    y32 = nv.nvfp4_linear(ac, as_, a_gs, wc, ws, w_gs, M, N, K, out_dtype=nv.OUT_FP32)
+    yb = nv.nvfp4_linear(ac, as_, a_gs, wc, ws, w_gs, M, N, K, out_dtype=nv.OUT_BF16)
+    st, info = nv.nvfp4_last_device_error()
+    assert st == 0, f"device error word {info:#x}"
+    return y32.cpu().numpy(), yb.float().cpu().numpy()
+
+
+@pytest.mark.parametrize("path,M", [(LARGE, 16), (SMALL, 16)])
+@pytest.mark.parametrize("p", [0, 1, 14, 15, 16, 31, 63, 64, 127, 128, 200, 255])
+def test_all_code_pairs_single_k(path, M, p):
+    """Row m holds code m, column n holds code n, both at k = p only; random scales."""
+    K, N = 256, 16
+    rng = np.random.default_rng(p)
+    ac = np.zeros((M, K), np.uint8)
+    wc = np.zeros((N, K), np.uint8)
+    ac[:, p] = np.arange(16)
+    wc[:, p] = np.arange(16)
+    as_ = rng.integers(1, 127, size=(M, K // 16)).astype(np.uint8)
+    ws = rng.integers(1, 127, size=(N, K // 16)).astype(np.uint8)
+    a_gs, w_gs = np.float32(0.5), np.float32(0.25)
+    y32, yb = run(path, *dev_operands(ac, as_, M, K), float(a_gs), *dev_operands(wc, ws, N, K),
+                  float(w_gs), M, N, K)
+    ref = oracle.linear64(oracle.dequantize(ac, as_, a_gs), oracle.dequantize(wc, ws, w_gs))
+    # every product is exact; only the final alpha multiply rounds (half an fp32 ulp)
+    assert np.all(np.abs(y32 - ref) <= np.abs(ref) * 2.0 ** -23)
+    H.check_bf16_out(yb, y32, ref, "pairs")
+
+
+@pytest.mark.parametrize("path,M,N,K", [
+    (LARGE, 128, 256, 256), (LARGE, 256, 512, 512), (LARGE, 200, 272, 320),
+    (LARGE, 129, 16, 64), (LARGE, 2048, 2560, 256), (LARGE, 300, 608, 1280),
+    (SMALL, 1, 16, 64), (SMALL, 7, 128, 320), (SMALL, 16, 400, 1024), (SMALL, 17, 144, 256),
+    (SMALL, 33, 272, 512), (SMALL, 64, 1040, 768)])
+def test_random_codes_and_scales(path, M, N, K):
+    rng = np.random.default_rng(M * 131 + N * 7 + K)
+    ac = rng.integers(0, 16, size=(M, K)).astype(np.uint8)
+    wc = rng.integers(0, 16, size=(N, K)).astype(np.uint8)
+    as_ = rng.integers(0x28, 0x58, size=(M, K // 16)).astype(np.uint8)   # 2^-2 .. 2^4
+    ws = rng.integers(0x28, 0x58, size=(N, K // 16)).astype(np.uint8)
+    a_gs, w_gs = np.float32(0.0173), np.float32(0.00291)
+    y32, yb = run(path, *dev_operands(ac, as_, M, K), float(a_gs), *dev_operands(wc, ws, N, K),
+                  float(w_gs), M, N, K)
+    ref = oracle.linear64(oracle.dequantize(ac, as_, a_gs), oracle.dequantize(wc, ws, w_gs))
+    H.check_gemm_fp32(y32, ref, f"random {M}x{N}x{K}")
+    H.check_bf16_out(yb, y32, ref, f"random {M}x{N}x{K}")
+
+
+def test_cancellation_heavy_accumulation():
+    """Alternating large +-6 * 448 products with small ones: fp32 accumulation must hold 1e-5."""
+    M, N, K = 128, 256, 5120
+    rng = np.random.default_rng(77)
+    ac = rng.integers(0, 16, size=(M, K)).astype(np.uint8)
+    wc = rng.integers(0, 16, size=(N, K)).astype(np.uint8)
+    ac[:, 0::64] = 7
+    wc[:, 0::128] = 7
+    wc[:, 64::128] = 15
+    as_ = rng.integers(0x08, 0x7F, size=(M, K // 16)).astype(np.uint8)
+    ws = rng.integers(0x08, 0x7F, size=(N, K // 16)).astype(np.uint8)
+    for path in (LARGE,):
+        y32, yb = run(path, *dev_operands(ac, as_, M, K), 1e-3, *dev_operands(wc, ws, N, K), 2e-3,
+                      M, N, K)
+        ref = oracle.linear64(oracle.dequantize(ac, as_, np.float32(1e-3)),
+                              oracle.dequantize(wc, ws, np.float32(2e-3)))
+        H.check_gemm_fp32(y32, ref, "cancellation")
+
+
+@pytest.mark.parametrize("path,M,N,K", [(LARGE, 200, 272, 320), (LARGE, 512, 768, 1024),
+                                        (SMALL, 5, 144, 320), (SMALL, 64, 256, 5120),
+                                        (AUTO, 64, 128, 256)])
+def test_quantize_then_gemm(path, M, N, K):
+    xb = workloads.random_bf16((M, K), seed=M + K, std=2.0)
+    wb = workloads.random_bf16((N, K), seed=N + K + 1, std=1 / np.sqrt(K))
+    xf, wf = H.f32(xb), H.f32(wb)
+    a_gs = oracle.global_scale(np.abs(xf).max())
+    ac, as_ = nv.nvfp4_quantize_act(H.bf16_dev(xb), float(a_gs))
+    wc, ws, (w_gs,) = nv.nvfp4_quantize_weight(H.bf16_dev(wb))
+    qx, sx = oracle.quantize(xf, a_gs)
+    w_gs_ref = oracle.global_scale(np.abs(wf).max())
+    assert np.float32(w_gs) == w_gs_ref
+    qw, sw = oracle.quantize(wf, w_gs_ref)
+    np.testing.assert_array_equal(H.unpack_codes(ac.cpu().numpy()), qx)
+    np.testing.assert_array_equal(H.unpack_codes(wc.cpu().numpy()), qw)
+    y32, yb = run(path, ac, as_, float(a_gs), wc, ws, float(w_gs), M, N, K)
+    ref = oracle.linear64(oracle.dequantize(qx, sx, a_gs), oracle.dequantize(qw, sw, w_gs_ref))
+    H.check_gemm_fp32(y32, ref, "quantize+gemm")
+    H.check_bf16_out(yb, y32, ref, "quantize+gemm")
+
+
+def test_tiny_workload_end_to_end():
+    """The tiny configuration: calibrate, quantise, GEMM, bf16 output."""
+    w = workloads.WORKLOADS[1]
+    calib, live, wbits = workloads.activations(w, calib=True), workloads.activations(w), workloads.weights(w)
+    a_gs = nv.nvfp4_global_scale(nv.nvfp4_amax(H.bf16_dev(calib)).item())
+    assert np.float32(a_gs) == oracle.global_scale(np.abs(H.f32(calib)).max())
+    ac, as_ = nv.nvfp4_quantize_act(H.bf16_dev(live), a_gs)
+    wc, ws, (w_gs,) = nv.nvfp4_quantize_weight(H.bf16_dev(wbits))
+    y = nv.nvfp4_linear(ac, as_, a_gs, wc, ws, w_gs, w.M, w.N, w.K)
+    y32 = nv.nvfp4_linear(ac, as_, a_gs, wc, ws, w_gs, w.M, w.N, w.K, out_dtype=nv.OUT_FP32)
+    qx, sx = oracle.quantize(H.f32(live), np.float32(a_gs))
+    qw, sw = oracle.quantize(H.f32(wbits), np.float32(w_gs))
+    ref = oracle.linear64(oracle.dequantize(qx, sx, a_gs), oracle.dequantize(qw, sw, w_gs))
+    H.check_gemm_fp32(y32.cpu().numpy(), ref, "tiny")
+    H.check_bf16_out(y.float().cpu().numpy(), y32.cpu().numpy(), ref, "tiny")
+
+
+def test_output_row_stride_and_no_overwrite():
+    """ldy > N: columns past N are never written (large and small kernels)."""
+    M, N, K, ldy = 150, 144, 256, 160
+    rng = np.random.default_rng(9)
+    ac = rng.integers(0, 16, size=(M, K)).astype(np.uint8)
+    wc = rng.integers(0, 16, size=(N, K)).astype(np.uint8)
+    as_ = rng.integers(0x30, 0x40, size=(M, K // 16)).astype(np.uint8)
+    ws = rng.integers(0x30, 0x40, size=(N, K // 16)).astype(np.uint8)
+    A, W = dev_operands(ac, as_, M, K), dev_operands(wc, ws, N, K)
+    ref = oracle.linear64(oracle.dequantize(ac, as_, np.float32(0.01)),
+                          oracle.dequantize(wc, ws, np.float32(0.02)))
+    for path, m in ((LARGE, M), (SMALL, 40)):
+        nv.nvfp4_set_gemm_path(path)
+        y = torch.full((m, ldy), -7.0, dtype=torch.float32, device="cuda")
+        nv.nvfp4_linear(A[0], A[1], 0.01, W[0], W[1], 0.02, m, N, K, y=y[:, :N],
+                        out_dtype=nv.OUT_FP32)
+        out = y.cpu().numpy()
+        assert np.all(out[:, N:] == -7.0)
+        H.check_gemm_fp32(out[:, :N], ref[:m], f"ldy path {path}")
