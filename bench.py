@@ -1,0 +1,464 @@
+"""Benchmark of the NVFP4 W4A4 linear layer on B200.
+
+One step = one pass of the layer's hot path over one batch: quantise the bf16
+activations (E2M1 codes + E4M3 block scales under the static global scale)
+and run the block-scaled FP4 GEMM with the segment epilogue, bf16 output.
+Default workload: the single prefill projection M=4096, K=5120, N=5120
+(activations Student-t(3)/sqrt(3) with 8 outlier channels x100, weights
+N(0, 1/sqrt(K)), static activation scale calibrated on a 512-row batch).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload prefill|gdn_inproj|decode]
+
+Prints one JSON line on rank 0.  Multi-GPU runs (torchrun, one rank per GPU)
+are weak-scaled replicas: every rank runs the same layer on its own batch, no
+collective touches the data path; the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "NVFP4 W4A4 linear TFLOPS & % of B200 FP4 peak; small-M weight GB/s"
+FP4_PER_BF16 = 4.0          # nominal dense FP4 / BF16 tensor throughput ratio (9 / 2.25 PFLOP/s)
+ROTATE_ACT = 6              # distinct activation buffers (each step uses the next one)
+ROTATE_W = 4                # distinct weight copies
+
+
+# --------------------------------------------------------------- plumbing
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sus=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples taken while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "20"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.path is None:
+            return None
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) >= 9:
+                try:
+                    rows.append((float(f[1]), float(f[2]), float(f[3]), f[5], f[6], f[7], f[8]))
+                except ValueError:
+                    pass
+        os.unlink(self.path)
+        if not rows:
+            return None
+        loaded = [r for r in rows if r[2] > 300.0] or rows
+        reasons = set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in loaded:
+            for name, v in zip(names, r[3:]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": rows[0][1],
+                "power_w_max": max(r[2] for r in rows), "samples": len(loaded),
+                "reasons": sorted(reasons)}
+
+
+def source_digest():
+    h = hashlib.sha256()
+    for f in ("ptx.cuh", "gemm.cuh", "quantize.cuh", "api.cu"):
+        h.update(open(os.path.join(ROOT, "nvfp4_w4a4_quantized_quantizer_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(name: str):
+    """dram bytes per launch from the committed ncu summary, if it matches the current source."""
+    p = os.path.join(ROOT, "profiles", name)
+    if not os.path.exists(p):
+        return None
+    text = open(p).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    d = re.search(r"source_digest:\s*([0-9a-f]+)", text)
+    if m and d and d.group(1) == source_digest():
+        return float(m.group(1))
+    return None
+
+
+# ------------------------------------------------------------- workloads
+def _dev_bf16(bits, device):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+class Layer:
+    """Device-resident operands of one workload, with rotated copies."""
+
+    def __init__(self, wl: workloads.Workload, M: int, device, rotate_act=ROTATE_ACT,
+                 rotate_w=ROTATE_W):
+        import nvfp4_w4a4_quantized_quantizer_b200 as nv
+        self.nv, self.wl, self.M, self.N, self.K = nv, wl, M, wl.N, wl.K
+        calib = _dev_bf16(workloads.activations(wl, calib=True), device)
+        self.a_gs = nv.nvfp4_global_scale(nv.nvfp4_amax(calib).item())
+        self.x_host = workloads.activations(wl, M=M)
+        x = _dev_bf16(self.x_host, device)
+        self.xs = [x] + [x.clone() for _ in range(rotate_act - 1)]
+        wbits = _dev_bf16(workloads.weights(wl), device)
+        wc, ws, self.w_gs = nv.nvfp4_quantize_weight(wbits, seg_offsets=wl.seg_offsets)
+        del wbits
+        self.ws = [(wc, ws)] + [(wc.clone(), ws.clone()) for _ in range(rotate_w - 1)]
+        self.codes = [torch.empty((M, self.K // 2), dtype=torch.uint8, device=device) for _ in range(2)]
+        self.scales = [torch.empty(nv.nvfp4_scale_bytes(M, self.K), dtype=torch.uint8, device=device)
+                       for _ in range(2)]
+        self.ys = [torch.empty((M, self.N), dtype=torch.bfloat16, device=device) for _ in range(2)]
+        self.segs = []
+        gate_dev = {}
+        if any(s.op == "gdn_decay" for s in wl.segments):
+            a_log, dt = workloads.gate_params(wl)
+            gate_dev = dict(a_log=torch.from_numpy(a_log).to(device), dt=torch.from_numpy(dt).to(device))
+        for s, off, g in zip(wl.segments, wl.seg_offsets, self.w_gs):
+            op = {"none": nv.OP_NONE, "sigmoid": nv.OP_SIGMOID, "gdn_decay": nv.OP_GDN_DECAY}[s.op]
+            self.segs.append(nv.SegmentSpec(off, g, self.a_gs, op,
+                                            gate_dev.get("a_log") if op == nv.OP_GDN_DECAY else None,
+                                            gate_dev.get("dt") if op == nv.OP_GDN_DECAY else None))
+
+    def quantize(self, i, stream, x=None):
+        xx = self.xs[i % len(self.xs)] if x is None else x
+        self.nv.nvfp4_quantize_act(xx, self.a_gs, codes=self.codes[i % 2], scales=self.scales[i % 2],
+                                   stream=stream)
+
+    def gemm(self, i, stream):
+        wc, ws = self.ws[i % len(self.ws)]
+        self.nv.nvfp4_fused_linear(self.codes[i % 2], self.scales[i % 2], wc, ws, self.M, self.N,
+                                   self.K, self.segs, y=self.ys[i % 2], stream=stream)
+
+    @property
+    def flops(self):
+        return 2.0 * self.M * self.N * self.K
+
+    @property
+    def weight_bytes(self):
+        return self.N * self.K // 2 + self.nv.nvfp4_scale_bytes(self.N, self.K)
+
+
+def time_steps(layer: Layer, steps: int, warmup: int, stream, per_kernel: bool):
+    """Device time of `steps` back-to-back steps (events on `stream`), plus per-kernel means."""
+    for i in range(warmup):
+        layer.quantize(i, stream)
+        layer.gemm(i, stream)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3 * steps + 1)] if per_kernel else None
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(steps):
+        if per_kernel:
+            ev[3 * i].record(stream)
+        layer.quantize(i, stream)
+        if per_kernel:
+            ev[3 * i + 1].record(stream)
+        layer.gemm(i, stream)
+        if per_kernel:
+            ev[3 * i + 2].record(stream)
+    end.record(stream)
+    end.synchronize()
+    total_ms = start.elapsed_time(end)
+    q_ms = g_ms = None
+    if per_kernel:
+        q_ms = sum(ev[3 * i].elapsed_time(ev[3 * i + 1]) for i in range(steps)) / steps
+        g_ms = sum(ev[3 * i + 1].elapsed_time(ev[3 * i + 2]) for i in range(steps)) / steps
+    return total_ms, q_ms, g_ms
+
+
+def e2e(layer: Layer, steps: int, warmup: int, stream):
+    """Same metric through the public API from pinned host buffers: H2D of the
+    step's activations, quantise, GEMM, D2H of the bf16 output, every step."""
+    xh = torch.from_numpy(layer.x_host.view(np.int16)).view(torch.bfloat16).pin_memory()
+    yh = torch.empty((layer.M, layer.N), dtype=torch.bfloat16).pin_memory()
+    xd = torch.empty_like(layer.xs[0])
+
+    def one(i):
+        with torch.cuda.stream(stream):
+            xd.copy_(xh, non_blocking=True)
+            layer.quantize(i, stream, x=xd)
+            layer.gemm(i, stream)
+            yh.copy_(layer.ys[i % 2], non_blocking=True)
+
+    for i in range(warmup):
+        one(i)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(steps):
+        one(i)
+    b.record(stream)
+    b.synchronize()
+    ms = a.elapsed_time(b) / steps
+    return ms, xh.numel() * 2, yh.numel() * 2
+
+
+def small_m_sweep(device, stream, iters=200, warmup=10):
+    """Decode-shaped sweep on the fused GDN in-projection weights: weight-stream GB/s."""
+    import nvfp4_w4a4_quantized_quantizer_b200 as nv
+    wl = workloads.WORKLOADS[5]
+    out = {}
+    base = Layer(wl, 64, device, rotate_act=1, rotate_w=ROTATE_W)
+    for M in wl.m_sweep:
+        x = base.xs[0][:M]
+        c, s = nv.nvfp4_quantize_act(x, base.a_gs, stream=stream)
+        y = torch.empty((M, base.N), dtype=torch.bfloat16, device=device)
+
+        def run(i):
+            wc, ws = base.ws[i % len(base.ws)]
+            nv.nvfp4_quantize_act(x, base.a_gs, codes=c, scales=s, stream=stream)
+            nv.nvfp4_fused_linear(c, s, wc, ws, M, base.N, base.K, base.segs, y=y, stream=stream)
+
+        for i in range(warmup):
+            run(i)
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * iters)]
+        for i in range(iters):
+            wc, ws = base.ws[i % len(base.ws)]
+            nv.nvfp4_quantize_act(x, base.a_gs, codes=c, scales=s, stream=stream)
+            ev[2 * i].record(stream)
+            nv.nvfp4_fused_linear(c, s, wc, ws, M, base.N, base.K, base.segs, y=y, stream=stream)
+            ev[2 * i + 1].record(stream)
+        torch.cuda.synchronize()
+        g_ms = statistics.median(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(iters))
+        out[f"M={M}"] = {"gemm_us": round(g_ms * 1e3, 2),
+                         "weight_GBps": round(base.weight_bytes / (g_ms * 1e-3) / 1e9, 1),
+                         "tokens_per_s": round(M / (g_ms * 1e-3), 1)}
+    return out
+
+
+# ------------------------------------------------------------ CPU oracle
+class OracleSample:
+    """The oracle, as it stands, on bounded samples of the workload: quantise a
+    few activation rows, dequantise, float64 GEMM against the dequantised
+    weights (static: quantised and dequantised once, outside the timing)."""
+
+    def __init__(self, wl: workloads.Workload):
+        import oracle
+        self.oracle, self.wl = oracle, wl
+        f32 = workloads.bf16_bits_to_f32
+        calib = f32(workloads.activations(wl, calib=True))
+        self.a_gs = oracle.global_scale(np.abs(calib).max())
+        wf = f32(workloads.weights(wl))
+        self.what = np.empty(wf.shape, np.float64)
+        for s, off in zip(wl.segments, wl.seg_offsets):
+            sl = slice(off, off + s.width)
+            gs = oracle.global_scale(np.abs(wf[sl]).max())
+            q, sc = oracle.quantize(wf[sl], gs)
+            self.what[sl] = oracle.dequantize(q, sc, gs)
+        self.x = f32(workloads.activations(wl, rows=(0, min(256, wl.M))))
+        try:
+            from threadpoolctl import threadpool_info
+            self.threads = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
+        except Exception:  # pragma: no cover
+            self.threads = os.cpu_count()
+
+    def run(self, rows: int):
+        q, sc = self.oracle.quantize(self.x[:rows], self.a_gs)
+        return self.oracle.linear64(self.oracle.dequantize(q, sc, self.a_gs), self.what)
+
+    def flops(self, rows: int) -> float:
+        return 2.0 * rows * self.wl.N * self.wl.K
+
+    def describe(self, rows: int, reps: int, el: float) -> str:
+        return (f"{rows} activation rows x K={self.wl.K} x N={self.wl.N} per step: oracle quantise + "
+                f"dequantise + float64 GEMM vs pre-dequantised weights; {reps} steps in {el:.1f} s")
+
+    def timed(self, rows: int, steps: int, warmup: int):
+        for _ in range(warmup):
+            self.run(rows)
+        t0 = time.perf_counter()
+        for _ in range(steps):
+            self.run(rows)
+        el = time.perf_counter() - t0
+        return self.flops(rows) * steps / el / 1e12, el
+
+
+def cpu_baseline(wl: workloads.Workload, target_s: float = 12.0, rows: int = 32):
+    s = OracleSample(wl)
+    t0 = time.perf_counter()
+    s.run(rows)
+    t1 = time.perf_counter() - t0
+    steps = max(1, int(target_s / max(t1, 1e-3)))
+    tflops, el = s.timed(rows, steps, 0)
+    return {"value": round(tflops, 6), "unit": "TFLOPS", "cores": s.threads, "kind": "oracle",
+            "sample": s.describe(rows, steps, el)}
+
+
+# ------------------------------------------------------------------ main
+WORKLOAD_BY_NAME = {"prefill": 2, "gdn_inproj": 3, "decode": 5}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="prefill", choices=sorted(WORKLOAD_BY_NAME))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-small-m", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    ws, rank, local = dist_env()
+    wl = workloads.WORKLOADS[WORKLOAD_BY_NAME[args.workload]]
+    M = wl.M
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        samp = OracleSample(wl)
+        t0 = time.perf_counter()
+        samp.run(1)
+        t1 = time.perf_counter() - t0
+        budget = 120.0 / (args.steps + args.warmup)          # whole run within a few minutes
+        rows = int(np.clip(budget / max(t1, 1e-4), 1, 256))
+        tflops, el = samp.timed(rows, args.steps, args.warmup)
+        line = {"metric": METRIC, "value": round(tflops, 6), "unit": "TFLOPS", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(el / args.steps * 1e3, 3),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "impl": "reference",
+                "config": {"workload": wl.name, "M": M, "N": wl.N, "K": wl.K,
+                           "sample_rows_per_step": rows},
+                "cpu_baseline": {"value": round(tflops, 6), "unit": "TFLOPS", "cores": samp.threads,
+                                 "kind": "oracle", "sample": samp.describe(rows, args.steps, el)},
+                "e2e": {"value": round(tflops, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import nvfp4_w4a4_quantized_quantizer_b200 as nv
+    nv.load()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    pg = None
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+        pg = dist
+    stream = torch.cuda.Stream(device)
+    layer = Layer(wl, M, device)
+    torch.cuda.synchronize()
+
+    # main timed region: barrier + sync on both sides, max over ranks
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        total_ms, _, _ = time_steps(layer, args.steps, args.warmup, stream, per_kernel=False)
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    clocks = clk.summary()
+    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+    if pg:
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_step = total_ms / args.steps
+    value = ws * layer.flops / (ms_step * 1e-3) / 1e12
+
+    # per-kernel device times (separate pass, events around each launch)
+    _, q_ms, g_ms = time_steps(layer, min(args.steps, 500), 5, stream, per_kernel=True)
+    pk = peaks()
+    fp4_peak = pk["bf16"] * FP4_PER_BF16
+    g_tflops = layer.flops / (g_ms * 1e-3) / 1e12
+    q_bytes = layer.M * layer.K * 2 + layer.M * layer.K // 2 + nv.nvfp4_scale_bytes(layer.M, layer.K)
+    q_gbs = q_bytes / (q_ms * 1e-3) / 1e9
+    traffic = ncu_traffic(f"gemm_tc_{wl.name}.md")
+
+    e_ms, h2d, d2h = e2e(layer, max(20, min(200, args.steps // 20)), 3, stream)
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "M": M, "N": wl.N, "K": wl.K,
+                   "step": "quantize_act + fused NVFP4 GEMM (bf16 out)",
+                   "l2": f"inputs rotated over {ROTATE_ACT} activation / {ROTATE_W} weight copies "
+                         "(working set > L2)", "parallelism": f"replicas x{ws}"},
+        "roofline": {"bound": "tensor", "achieved": round(g_tflops, 1), "peak": round(fp4_peak, 1),
+                     "unit": "TFLOP/s", "frac": round(g_tflops / fp4_peak, 4),
+                     "traffic": traffic,
+                     "peak_note": f"{pk['source']} bf16 burst {pk['bf16']} x {FP4_PER_BF16} nominal FP4/BF16"},
+        "kernels": {"gemm_us": round(g_ms * 1e3, 2), "gemm_tflops": round(g_tflops, 1),
+                    "quantize_us": round(q_ms * 1e3, 2), "quantize_GBps": round(q_gbs, 1),
+                    "quantize_hbm_frac": round(q_gbs / pk["hbm"], 4)},
+        "e2e": {"value": round(layer.flops / (e_ms * 1e-3) / 1e12, 2), "unit": "TFLOPS",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and not args.no_small_m and ws == 1:
+        sm = small_m_sweep(device, stream)
+        for v in sm.values():
+            v["hbm_frac"] = round(v["weight_GBps"] / pk["hbm"], 4)
+        line["small_m"] = sm
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -27,7 +27,9 @@ round-to-nearest-even):
   stream 5 and shared by the live and calibration batches; those columns are
   multiplied by 100 after the t/sqrt(3) scaling;
 * the tiny configuration puts one outlier per row at a uniformly drawn column,
-  multiplied by 50, in both its live and calibration batches.
+  multiplied by 50, in both its live and calibration batches;
+* the decode sweep reuses the GDN in-projection's weights, per-module weight
+  stds and gate parameters (same streams of configuration 3).
 """
 from __future__ import annotations
 
@@ -61,6 +63,11 @@ class Workload:
     calib_rows: int
     w_std_kind: str           # "unit" | "loguniform" | "gate_up_x3"
     m_sweep: Tuple[int, ...] = ()
+    weights_of: int = 0       # draw weights / gate params as configuration `weights_of` does
+
+    @property
+    def weight_cfg(self) -> int:
+        return self.weights_of or self.index
 
     @property
     def N(self) -> int:
@@ -90,7 +97,7 @@ WORKLOADS = {
                 (Segment("gate", 17408), Segment("up", 17408)),
                 "t3_channels", 512, "gate_up_x3"),
     5: Workload(5, "decode_sweep_Mx5120x16480", 64, 5120, GDN_SEGMENTS,
-                "normal_channels", 512, "loguniform", m_sweep=(1, 8, 32, 64)),
+                "normal_channels", 512, "loguniform", m_sweep=(1, 8, 32, 64), weights_of=3),
 }
 
 # Second layer of the MLP pair: down projection [16384 x 17408] -> 5120.
@@ -167,7 +174,7 @@ def segment_stds(w: Workload) -> np.ndarray:
     if w.w_std_kind == "unit":
         return np.full(n, base)
     if w.w_std_kind == "loguniform":
-        rng = _rng(w.index, ST_SEGSTD)
+        rng = _rng(w.weight_cfg, ST_SEGSTD)
         return base * np.exp(rng.uniform(np.log(0.25), np.log(4.0), size=n))
     if w.w_std_kind == "gate_up_x3":
         return np.array([base, 3.0 * base])
@@ -180,7 +187,7 @@ def weights(w: Workload, rows: Optional[Tuple[int, int]] = None) -> np.ndarray:
     offs = np.array(w.seg_offsets + [w.N])
 
     def block(b):
-        rng = _rng(w.index, ST_W, b)
+        rng = _rng(w.weight_cfg, ST_W, b)
         z = rng.standard_normal((ROW_BLOCK, w.K))
         r = b * ROW_BLOCK + np.arange(ROW_BLOCK)
         seg = np.clip(np.searchsorted(offs, r, side="right") - 1, 0, len(stds) - 1)
@@ -204,7 +211,7 @@ def down_weights(rows: Optional[Tuple[int, int]] = None) -> np.ndarray:
 
 def gate_params(w: Workload, heads: int = 48) -> Tuple[np.ndarray, np.ndarray]:
     """(A_log, dt_bias) float32 [heads]: A_log ~ U(-1, 1.5), dt_bias ~ N(0, 0.5)."""
-    rng = _rng(w.index, ST_GATE)
+    rng = _rng(w.weight_cfg, ST_GATE)
     a_log = rng.uniform(-1.0, 1.5, size=heads).astype(np.float32)
     dt_bias = (rng.standard_normal(heads) * 0.5).astype(np.float32)
     return a_log, dt_bias
