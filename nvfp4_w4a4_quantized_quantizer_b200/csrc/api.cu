@@ -193,9 +193,10 @@ nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t K, int64_t ld,
   a.scales = static_cast<uint8_t*>(scales);
   a.pad_from = pad_from;
   a.pad_to = pad_to;
-  const int64_t units = rows * ((K + 255) / 256);
+  const int64_t units = rows * ((K + 256 * nvfp4::QUANT_UNROLL - 1) / (256 * nvfp4::QUANT_UNROLL));
+  if (units >= (1ll << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   const int warps_per_block = nvfp4::QUANT_THREADS / 32;
-  const int grid = grid_for(units, warps_per_block * nvfp4::QUANT_UNROLL, sms * 8);
+  const int grid = grid_for(units, warps_per_block, sms * 8);
   nvfp4::k_quantize<<<grid, nvfp4::QUANT_THREADS, 0, st>>>(a);
   return check_launch();
 }

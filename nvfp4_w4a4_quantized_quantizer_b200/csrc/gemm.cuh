@@ -9,12 +9,14 @@
 //
 // Two kernels:
 //   k_gemm_tc     persistent, warp-specialised, one 128 x 256 output tile at
-//                 a time per CTA (1 CTA per SM).  Warp 0 streams A/B codes
-//                 with TMA (128-byte swizzle) and the scale atoms with bulk
-//                 copies into a 4-stage shared-memory ring; warp 1 copies the
-//                 scale atoms into TMEM (tcgen05.cp) and issues
-//                 tcgen05.mma.kind::mxf4nvf4 (K = 64 per instruction) into a
-//                 128 x 256 fp32 TMEM accumulator; warps 2-9 drain the
+//                 a time per CTA (1 CTA per SM).  Two producer warps stream
+//                 the activation and weight codes with TMA (128-byte swizzle)
+//                 and their scale atoms with bulk copies into a 4-stage
+//                 shared-memory ring; a copier warp moves each stage's scale
+//                 atoms into a per-stage TMEM region (tcgen05.cp) while the
+//                 MMA warp issues tcgen05.mma.kind::mxf4nvf4 (K = 64 per
+//                 instruction) on the previous stage into a 128 x 256 fp32
+//                 TMEM accumulator; eight epilogue warps drain the
 //                 accumulator (each lane = one row, 128 columns), release it
 //                 to the MMA warp, then apply alpha / op and store.
 //   k_gemm_small  M <= 64 (decode shapes): operands swapped so the weight
@@ -66,6 +68,20 @@ __device__ __forceinline__ float apply_op(float v, int op, const float* a_log,
   return v;
 }
 
+// Gate epilogue for 16 consecutive columns, kept out of line: only the few
+// gate columns take it, and inlining it into the unrolled store loops would
+// multiply the kernels' code size.
+__device__ __noinline__ void apply_op_16(float* o, int op, const float* a_log,
+                                         const float* dt_bias, int h0) {
+#pragma unroll 1
+  for (int i = 0; i < 16; ++i) o[i] = apply_op(o[i], op, a_log, dt_bias, h0 + i);
+}
+
+__device__ __noinline__ float apply_op_1(float v, int op, const float* a_log,
+                                         const float* dt_bias, int h) {
+  return apply_op(v, op, a_log, dt_bias, h);
+}
+
 // Advance `seg` so that n lies in [n_off[seg], n_off[seg+1]).
 __device__ __forceinline__ int seg_advance(const SegTable& t, int seg, int n) {
   while (seg + 1 < t.nseg && n >= t.n_off[seg + 1]) ++seg;
@@ -73,6 +89,16 @@ __device__ __forceinline__ int seg_advance(const SegTable& t, int seg, int n) {
 }
 
 // ============================================================ k_gemm_tc
+// Warp roles (12 warps):
+//   0  producer A: TMA of the activation codes + bulk copy of their scale atoms
+//   1  MMA issuer: tcgen05.mma only (one elected lane), TMEM allocation
+//   2  scale copier: tcgen05.cp of the stage's scale atoms into that stage's
+//      TMEM scale region, so the copies overlap the MMAs of the previous stage
+//   3  producer B: TMA of the weight codes + bulk copies of their scale atoms
+//   4-11 epilogue: warp w drains TMEM lane quarter w % 4, column half (w-4)/4
+// Per stage s the scale region is TMEM columns [256 + 48 s, 256 + 48 s + 48):
+// 16 columns of activation scales (4 MMAs x 4) then 32 of weight scales
+// (4 MMAs x 8).  The accumulator is columns [0, 256).
 namespace tc {
 constexpr int BM = 128;
 constexpr int BN = 256;
@@ -85,14 +111,16 @@ constexpr int SFA_BYTES = 4 * 512;      // 4 atoms (K = 64 each) x 128 rows
 constexpr int SFB_BYTES = 2 * 4 * 512;  // 2 row blocks of 128
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 54 KB
 constexpr int EPI_WARPS = 8;
-constexpr int THREADS = 32 * (2 + EPI_WARPS);
+constexpr int EPI_WARP0 = 4;
+constexpr int THREADS = 32 * (EPI_WARP0 + EPI_WARPS);
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
-constexpr uint32_t SFA_COL = 256;       // 4 MMAs x 4 columns
-constexpr uint32_t SFB_COL = 272;       // 4 MMAs x 8 columns
+constexpr uint32_t SF_COL = 256;        // + 48 * stage
+constexpr uint32_t SF_STRIDE = 48;
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
 static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
+static_assert(SF_COL + STAGES * SF_STRIDE <= TMEM_COLS, "TMEM budget");
 }  // namespace tc
 
 __global__ void __launch_bounds__(tc::THREADS, 1)
@@ -103,8 +131,8 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-  // bars: full[STAGES], empty[STAGES], tmem_full, tmem_empty, drain
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 3);
+  // bars: full[S], empty[S], sf_ready[S], tmem_full, tmem_empty, drain_mma, drain_sf
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -118,18 +146,22 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
 
   auto full_bar = [&](int s) { return smem_addr(bars + s); };
   auto empty_bar = [&](int s) { return smem_addr(bars + STAGES + s); };
-  const uint32_t tmem_full = smem_addr(bars + 2 * STAGES);
-  const uint32_t tmem_empty = smem_addr(bars + 2 * STAGES + 1);
-  const uint32_t drain_bar = smem_addr(bars + 2 * STAGES + 2);
+  auto sf_bar = [&](int s) { return smem_addr(bars + 2 * STAGES + s); };
+  const uint32_t tmem_full = smem_addr(bars + 3 * STAGES);
+  const uint32_t tmem_empty = smem_addr(bars + 3 * STAGES + 1);
+  const uint32_t drain_mma = smem_addr(bars + 3 * STAGES + 2);
+  const uint32_t drain_sf = smem_addr(bars + 3 * STAGES + 3);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full_bar(s), 1);
+      mbar_init(full_bar(s), 2);            // both producers arrive (with their bytes)
       mbar_init(empty_bar(s), 1);
+      mbar_init(sf_bar(s), 1);
     }
     mbar_init(tmem_full, 1);
     mbar_init(tmem_empty, EPI_WARPS);
-    mbar_init(drain_bar, 1);
+    mbar_init(drain_mma, 1);
+    mbar_init(drain_sf, 1);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&tmA);
@@ -144,11 +176,11 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------ TMA producer
+  if (warp == 0 || warp == 3) {
+    // ---------------------------------------------------- TMA producers
     if (lane == 0) {
-      const uint64_t pol_a = policy_evict_last();
-      const uint64_t pol_b = policy_evict_last();
+      const bool is_a = (warp == 0);
+      const uint64_t pol = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
       int64_t issued = 0;
@@ -156,26 +188,29 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int mb = tile % num_m;
         const int nb = tile / num_m;
+        const int nb0 = nb * 2;
+        const int nsfb = min(2, sfb_blocks - nb0);
         for (int kt = 0; kt < num_kt; ++kt) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, g.wait_ns, abort_flag)) {
-            if (!*abort_flag) record_error(SITE_PRODUCER_EMPTY, 0);
+            if (!*abort_flag) record_error(SITE_PRODUCER_EMPTY, warp);
             *abort_flag = 1;
             ok = false;
             break;
           }
           const int nk = min(4, (g.K - kt * BK) / 64);
-          const int nb0 = nb * 2;
-          const int nsfb = min(2, sfb_blocks - nb0);
-          const uint32_t bytes = A_BYTES + B_BYTES + nk * 512 * (1 + nsfb);
           uint8_t* st = smem + stage * STAGE_BYTES;
-          mbar_arrive_expect_tx(full_bar(stage), bytes);
-          tma_load_2d(smem_addr(st), &tmA, kt * BKB, mb * BM, full_bar(stage), pol_a);
-          tma_load_2d(smem_addr(st + A_BYTES), &tmB, kt * BKB, nb * BN, full_bar(stage), pol_b);
-          bulk_load(smem_addr(st + A_BYTES + B_BYTES), g.sfa + (mb * kb4 + kt * 4) * 512,
-                    nk * 512, full_bar(stage), pol_a);
-          for (int j = 0; j < nsfb; ++j)
-            bulk_load(smem_addr(st + A_BYTES + B_BYTES + SFA_BYTES + j * 2048),
-                      g.sfb + ((nb0 + j) * kb4 + kt * 4) * 512, nk * 512, full_bar(stage), pol_b);
+          if (is_a) {
+            mbar_arrive_expect_tx(full_bar(stage), A_BYTES + nk * 512);
+            tma_load_2d(smem_addr(st), &tmA, kt * BKB, mb * BM, full_bar(stage), pol);
+            bulk_load(smem_addr(st + A_BYTES + B_BYTES), g.sfa + (mb * kb4 + kt * 4) * 512,
+                      nk * 512, full_bar(stage), pol);
+          } else {
+            mbar_arrive_expect_tx(full_bar(stage), B_BYTES + nk * 512 * nsfb);
+            tma_load_2d(smem_addr(st + A_BYTES), &tmB, kt * BKB, nb * BN, full_bar(stage), pol);
+            for (int j = 0; j < nsfb; ++j)
+              bulk_load(smem_addr(st + A_BYTES + B_BYTES + SFA_BYTES + j * 2048),
+                        g.sfb + ((nb0 + j) * kb4 + kt * 4) * 512, nk * 512, full_bar(stage), pol);
+          }
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -183,12 +218,47 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
           }
         }
       }
-      // every copy issued must land before the CTA may exit
+      // every copy this thread issued must land before the CTA may exit
       for (int s = 0; s < STAGES && s < issued; ++s) {
         const int64_t uses = (issued - 1 - s) / STAGES + 1;
         if (!mbar_wait(full_bar(s), static_cast<uint32_t>((uses - 1) & 1), g.wait_ns, nullptr))
-          record_error(SITE_DRAIN, 0);
+          record_error(SITE_DRAIN, warp);
       }
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // ---------------------------------------------------- scale copier
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        for (int kt = 0; kt < num_kt; ++kt) {
+          if (!mbar_wait(full_bar(stage), phase, g.wait_ns, abort_flag)) {
+            if (!*abort_flag) record_error(SITE_MMA_FULL, 2);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nk = min(4, (g.K - kt * BK) / 64);
+          const uint32_t sfa_s = smem_addr(smem + stage * STAGE_BYTES + A_BYTES + B_BYTES);
+          const uint32_t sfb_s = sfa_s + SFA_BYTES;
+          const uint32_t col = tmem_base + SF_COL + SF_STRIDE * stage;
+          for (int kk = 0; kk < nk; ++kk) {
+            tmem_cp_32x128b_x4(col + 4 * kk, desc_sf_atom(sfa_s + kk * 512));
+            tmem_cp_32x128b_x4(col + 16 + 8 * kk, desc_sf_atom(sfb_s + kk * 512));
+            tmem_cp_32x128b_x4(col + 16 + 8 * kk + 4, desc_sf_atom(sfb_s + 2048 + kk * 512));
+          }
+          tc_commit(sf_bar(stage));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      tc_commit(drain_sf);
+      if (!mbar_wait(drain_sf, 0, g.wait_ns, nullptr)) record_error(SITE_DRAIN, 2);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -207,7 +277,10 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         }
         tc_fence_after();
         for (int kt = 0; kt < num_kt; ++kt) {
-          if (!mbar_wait(full_bar(stage), phase, g.wait_ns, abort_flag)) {
+          // the scale copies of this stage imply its operands have landed (the
+          // copier waited on the full barrier); the full wait below is free
+          if (!mbar_wait(sf_bar(stage), phase, g.wait_ns, abort_flag) ||
+              !mbar_wait(full_bar(stage), phase, g.wait_ns, abort_flag)) {
             if (!*abort_flag) record_error(SITE_MMA_FULL, 1);
             *abort_flag = 1;
             ok = false;
@@ -216,23 +289,13 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
           tc_fence_after();
           const int nk = min(4, (g.K - kt * BK) / 64);
           const uint8_t* st = smem + stage * STAGE_BYTES;
-          const uint32_t a_s = smem_addr(st);
-          const uint32_t b_s = smem_addr(st + A_BYTES);
-          const uint32_t sfa_s = smem_addr(st + A_BYTES + B_BYTES);
-          const uint32_t sfb_s = sfa_s + SFA_BYTES;
-          for (int kk = 0; kk < nk; ++kk) {
-            tmem_cp_32x128b_x4(tmem_base + SFA_COL + 4 * kk, desc_sf_atom(sfa_s + kk * 512));
-            tmem_cp_32x128b_x4(tmem_base + SFB_COL + 8 * kk, desc_sf_atom(sfb_s + kk * 512));
-            tmem_cp_32x128b_x4(tmem_base + SFB_COL + 8 * kk + 4,
-                               desc_sf_atom(sfb_s + 2048 + kk * 512));
-          }
-          const uint64_t adesc = desc_kmajor_sw128(a_s);
-          const uint64_t bdesc = desc_kmajor_sw128(b_s);
+          const uint64_t adesc = desc_kmajor_sw128(smem_addr(st));
+          const uint64_t bdesc = desc_kmajor_sw128(smem_addr(st + A_BYTES));
+          const uint32_t col = tmem_base + SF_COL + SF_STRIDE * stage;
           for (int kk = 0; kk < nk; ++kk) {
             // K = 64 fp4 = 32 bytes: advance the start address inside the swizzle atom
-            mma_mxf4nvf4(tmem_base + ACC_COL, adesc + 2 * kk, bdesc + 2 * kk, idesc,
-                         tmem_base + SFA_COL + 4 * kk, tmem_base + SFB_COL + 8 * kk,
-                         (kt | kk) != 0);
+            mma_mxf4nvf4(tmem_base + ACC_COL, adesc + 2 * kk, bdesc + 2 * kk, idesc, col + 4 * kk,
+                         col + 16 + 8 * kk, (kt | kk) != 0);
           }
           tc_commit(empty_bar(stage));
           if (++stage == STAGES) {
@@ -244,21 +307,21 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         tc_commit(tmem_full);
       }
       // all issued tensor-core work must finish before TMEM is freed
-      tc_commit(drain_bar);
-      if (!mbar_wait(drain_bar, 0, g.wait_ns, nullptr)) record_error(SITE_DRAIN, 1);
+      tc_commit(drain_mma);
+      if (!mbar_wait(drain_mma, 0, g.wait_ns, nullptr)) record_error(SITE_DRAIN, 1);
     }
     __syncwarp();
   } else {
     // ---------------------------------------------------------- epilogue
-    const int q = warp & 3;               // TMEM lane quarter this warp may access
-    const int half = (warp - 2) >> 2;     // columns [128*half, 128*half + 128)
+    const int q = warp & 3;                       // TMEM lane quarter this warp may access
+    const int half = (warp - EPI_WARP0) >> 2;     // columns [128*half, 128*half + 128)
     const int row_in_tile = q * 32 + lane;
     int local = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
       const int mb = tile % num_m;
       const int nb = tile / num_m;
       if (!mbar_wait(tmem_full, static_cast<uint32_t>(local & 1), g.wait_ns, abort_flag)) {
-        if (!*abort_flag) record_error(SITE_EPI_TMEM_FULL, 2 + (warp - 2));
+        if (!*abort_flag) record_error(SITE_EPI_TMEM_FULL, warp);
         *abort_flag = 1;
         break;
       }
@@ -286,9 +349,14 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             const int h0 = n - seg.n_off[s];
             float o[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float a = __fmul_rn(alpha, __uint_as_float(v[grp * 16 + i]));
-              o[i] = (op == 0) ? a : apply_op(a, op, seg.a_log[s], seg.dt_bias[s], h0 + i);
+            for (int i = 0; i < 16; ++i) o[i] = __fmul_rn(alpha, __uint_as_float(v[grp * 16 + i]));
+            if (op != 0) {
+              float t[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) t[i] = o[i];
+              apply_op_16(t, op, seg.a_log[s], seg.dt_bias[s], h0);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) o[i] = t[i];
             }
             if (g.out_fp32) {
               float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.y) + gm * g.ldy + n);
@@ -320,6 +388,11 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
 }
 
 // ========================================================== k_gemm_small
+// Warp roles (8 warps): 0 producer W (weight codes + scale atoms), 1 MMA
+// issuer, 2 scale copier, 3 producer X (token codes + scale atoms), 4-7
+// epilogue (warp w reads TMEM lane quarter w % 4).  TMEM: accumulator
+// columns [0, NT); stage s scale region [64 + 32 s, 64 + 32 s + 32): 16
+// columns of weight scales then 16 of token scales (4 MMAs x 4 each).
 namespace sm {
 constexpr int BW = 128;                 // weight rows per CTA (MMA M)
 constexpr int BK = 256;
@@ -329,12 +402,14 @@ constexpr int W_BYTES = BW * BKB;       // 16 KB
 constexpr int SFW_BYTES = 4 * 512;
 constexpr int SFX_BYTES = 4 * 512;
 constexpr int EPI_WARPS = 4;
-constexpr int THREADS = 32 * (2 + EPI_WARPS);
-constexpr uint32_t TMEM_COLS = 128;
+constexpr int EPI_WARP0 = 4;
+constexpr int THREADS = 32 * (EPI_WARP0 + EPI_WARPS);
+constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t ACC_COL = 0;         // NT columns
-constexpr uint32_t SFW_COL = 64;        // 4 MMAs x 4 columns
-constexpr uint32_t SFX_COL = 80;        // 4 MMAs x 4 columns
+constexpr uint32_t SF_COL = 64;         // + 32 * stage
+constexpr uint32_t SF_STRIDE = 32;
 constexpr int BAR_BYTES = 256;
+static_assert(SF_COL + STAGES * SF_STRIDE <= TMEM_COLS, "TMEM budget");
 template <int NT>
 struct Cfg {
   static constexpr int X_BYTES = NT * BKB;   // NT rows x 128 bytes
@@ -356,8 +431,8 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
-  // bars: full[STAGES], empty[STAGES], acc_full, drain
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 2);
+  // bars: full[S], empty[S], sf_ready[S], acc_full, drain_mma, drain_sf
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -368,16 +443,20 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
 
   auto full_bar = [&](int s) { return smem_addr(bars + s); };
   auto empty_bar = [&](int s) { return smem_addr(bars + STAGES + s); };
-  const uint32_t acc_full = smem_addr(bars + 2 * STAGES);
-  const uint32_t drain_bar = smem_addr(bars + 2 * STAGES + 1);
+  auto sf_bar = [&](int s) { return smem_addr(bars + 2 * STAGES + s); };
+  const uint32_t acc_full = smem_addr(bars + 3 * STAGES);
+  const uint32_t drain_mma = smem_addr(bars + 3 * STAGES + 1);
+  const uint32_t drain_sf = smem_addr(bars + 3 * STAGES + 2);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full_bar(s), 1);
+      mbar_init(full_bar(s), 2);
       mbar_init(empty_bar(s), 1);
+      mbar_init(sf_bar(s), 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(drain_bar, 1);
+    mbar_init(drain_mma, 1);
+    mbar_init(drain_sf, 1);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&tmW);
@@ -392,29 +471,33 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp == 0 || warp == 3) {
     if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();   // weights stream through once
-      const uint64_t pol_x = policy_evict_last();    // tokens are re-read by every CTA
+      const bool is_w = (warp == 0);
+      // weights stream through once; tokens are re-read by every CTA
+      const uint64_t pol = is_w ? policy_evict_first() : policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
       int64_t issued = 0;
       for (int kt = 0; kt < num_kt; ++kt) {
         if (!mbar_wait(empty_bar(stage), phase ^ 1u, g.wait_ns, abort_flag)) {
-          if (!*abort_flag) record_error(SITE_PRODUCER_EMPTY, 0);
+          if (!*abort_flag) record_error(SITE_PRODUCER_EMPTY, warp);
           *abort_flag = 1;
           break;
         }
         const int nk = min(4, (g.K - kt * BK) / 64);
-        const uint32_t bytes = W_BYTES + C::X_BYTES + 2 * nk * 512;
         uint8_t* st = smem + stage * C::STAGE_BYTES;
-        mbar_arrive_expect_tx(full_bar(stage), bytes);
-        tma_load_2d(smem_addr(st), &tmW, kt * BKB, wt * BW, full_bar(stage), pol_w);
-        tma_load_2d(smem_addr(st + W_BYTES), &tmX, kt * BKB, 0, full_bar(stage), pol_x);
-        bulk_load(smem_addr(st + W_BYTES + C::X_BYTES), g.sfb + (wt * kb4 + kt * 4) * 512, nk * 512,
-                  full_bar(stage), pol_w);
-        bulk_load(smem_addr(st + W_BYTES + C::X_BYTES + SFW_BYTES), g.sfa + (kt * 4) * 512,
-                  nk * 512, full_bar(stage), pol_x);
+        if (is_w) {
+          mbar_arrive_expect_tx(full_bar(stage), W_BYTES + nk * 512);
+          tma_load_2d(smem_addr(st), &tmW, kt * BKB, wt * BW, full_bar(stage), pol);
+          bulk_load(smem_addr(st + W_BYTES + C::X_BYTES), g.sfb + (wt * kb4 + kt * 4) * 512,
+                    nk * 512, full_bar(stage), pol);
+        } else {
+          mbar_arrive_expect_tx(full_bar(stage), C::X_BYTES + nk * 512);
+          tma_load_2d(smem_addr(st + W_BYTES), &tmX, kt * BKB, 0, full_bar(stage), pol);
+          bulk_load(smem_addr(st + W_BYTES + C::X_BYTES + SFW_BYTES), g.sfa + (kt * 4) * 512,
+                    nk * 512, full_bar(stage), pol);
+        }
         ++issued;
         if (++stage == STAGES) {
           stage = 0;
@@ -424,8 +507,37 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
       for (int s = 0; s < STAGES && s < issued; ++s) {
         const int64_t uses = (issued - 1 - s) / STAGES + 1;
         if (!mbar_wait(full_bar(s), static_cast<uint32_t>((uses - 1) & 1), g.wait_ns, nullptr))
-          record_error(SITE_DRAIN, 0);
+          record_error(SITE_DRAIN, warp);
       }
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int kt = 0; kt < num_kt; ++kt) {
+        if (!mbar_wait(full_bar(stage), phase, g.wait_ns, abort_flag)) {
+          if (!*abort_flag) record_error(SITE_MMA_FULL, 2);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const int nk = min(4, (g.K - kt * BK) / 64);
+        const uint32_t sfw_s = smem_addr(smem + stage * C::STAGE_BYTES + W_BYTES + C::X_BYTES);
+        const uint32_t sfx_s = sfw_s + SFW_BYTES;
+        const uint32_t col = tmem_base + SF_COL + SF_STRIDE * stage;
+        for (int kk = 0; kk < nk; ++kk) {
+          tmem_cp_32x128b_x4(col + 4 * kk, desc_sf_atom(sfw_s + kk * 512));
+          tmem_cp_32x128b_x4(col + 16 + 4 * kk, desc_sf_atom(sfx_s + kk * 512));
+        }
+        tc_commit(sf_bar(stage));
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      tc_commit(drain_sf);
+      if (!mbar_wait(drain_sf, 0, g.wait_ns, nullptr)) record_error(SITE_DRAIN, 2);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -435,7 +547,8 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
       uint32_t phase = 0;
       bool ok = true;
       for (int kt = 0; kt < num_kt; ++kt) {
-        if (!mbar_wait(full_bar(stage), phase, g.wait_ns, abort_flag)) {
+        if (!mbar_wait(sf_bar(stage), phase, g.wait_ns, abort_flag) ||
+            !mbar_wait(full_bar(stage), phase, g.wait_ns, abort_flag)) {
           if (!*abort_flag) record_error(SITE_MMA_FULL, 1);
           *abort_flag = 1;
           ok = false;
@@ -444,19 +557,12 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
         tc_fence_after();
         const int nk = min(4, (g.K - kt * BK) / 64);
         const uint8_t* st = smem + stage * C::STAGE_BYTES;
-        const uint32_t w_s = smem_addr(st);
-        const uint32_t x_s = smem_addr(st + W_BYTES);
-        const uint32_t sfw_s = smem_addr(st + W_BYTES + C::X_BYTES);
-        const uint32_t sfx_s = sfw_s + SFW_BYTES;
-        for (int kk = 0; kk < nk; ++kk) {
-          tmem_cp_32x128b_x4(tmem_base + SFW_COL + 4 * kk, desc_sf_atom(sfw_s + kk * 512));
-          tmem_cp_32x128b_x4(tmem_base + SFX_COL + 4 * kk, desc_sf_atom(sfx_s + kk * 512));
-        }
-        const uint64_t wdesc = desc_kmajor_sw128(w_s);
-        const uint64_t xdesc = desc_kmajor_sw128(x_s);
+        const uint64_t wdesc = desc_kmajor_sw128(smem_addr(st));
+        const uint64_t xdesc = desc_kmajor_sw128(smem_addr(st + W_BYTES));
+        const uint32_t col = tmem_base + SF_COL + SF_STRIDE * stage;
         for (int kk = 0; kk < nk; ++kk)
-          mma_mxf4nvf4(tmem_base + ACC_COL, wdesc + 2 * kk, xdesc + 2 * kk, idesc,
-                       tmem_base + SFW_COL + 4 * kk, tmem_base + SFX_COL + 4 * kk, (kt | kk) != 0);
+          mma_mxf4nvf4(tmem_base + ACC_COL, wdesc + 2 * kk, xdesc + 2 * kk, idesc, col + 4 * kk,
+                       col + 16 + 4 * kk, (kt | kk) != 0);
         tc_commit(empty_bar(stage));
         if (++stage == STAGES) {
           stage = 0;
@@ -464,8 +570,8 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
         }
       }
       if (ok) tc_commit(acc_full);
-      tc_commit(drain_bar);
-      if (!mbar_wait(drain_bar, 0, g.wait_ns, nullptr)) record_error(SITE_DRAIN, 1);
+      tc_commit(drain_mma);
+      if (!mbar_wait(drain_mma, 0, g.wait_ns, nullptr)) record_error(SITE_DRAIN, 1);
     }
     __syncwarp();
   } else {
@@ -489,8 +595,8 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
           if (j < g.M) {
-            const float a = __fmul_rn(alpha, __uint_as_float(v[j]));
-            const float o = (op == 0) ? a : apply_op(a, op, seg.a_log[s], seg.dt_bias[s], h);
+            float o = __fmul_rn(alpha, __uint_as_float(v[j]));
+            if (op != 0) o = apply_op_1(o, op, seg.a_log[s], seg.dt_bias[s], h);
             if (g.out_fp32)
               static_cast<float*>(g.y)[static_cast<int64_t>(j) * g.ldy + n] = o;
             else

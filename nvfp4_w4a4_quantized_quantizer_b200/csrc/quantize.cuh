@@ -98,59 +98,65 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
 }
 
 constexpr int QUANT_THREADS = 256;
-constexpr int QUANT_UNROLL = 4;
+constexpr int QUANT_UNROLL = 4;            // 256-element chunks per warp work unit
 
+// |x| max of eight bf16 values, exact, with packed bf16x2 instructions.
+__device__ __forceinline__ float bf16x8_absmax(const uint4& v) {
+  const __nv_bfloat162 a = __habs2(*reinterpret_cast<const __nv_bfloat162*>(&v.x));
+  const __nv_bfloat162 b = __habs2(*reinterpret_cast<const __nv_bfloat162*>(&v.y));
+  const __nv_bfloat162 c = __habs2(*reinterpret_cast<const __nv_bfloat162*>(&v.z));
+  const __nv_bfloat162 d = __habs2(*reinterpret_cast<const __nv_bfloat162*>(&v.w));
+  const __nv_bfloat162 m = __hmax2(__hmax2(a, b), __hmax2(c, d));
+  return fmaxf(__low2float(m), __high2float(m));
+}
+
+// A warp work unit is (row, 1024-element segment of the row); the host
+// guarantees rows * segments < 2^31 so the unit index stays 32-bit.
 __global__ void __launch_bounds__(QUANT_THREADS) k_quantize(const QuantArgs a) {
   const int lane = threadIdx.x & 31;
-  const int64_t gwarp = (static_cast<int64_t>(blockIdx.x) * QUANT_THREADS + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * QUANT_THREADS) >> 5;
-  const int64_t chunks = (a.K + 255) / 256;
-  const int64_t units = a.rows * chunks;
+  const uint32_t gwarp = (blockIdx.x * QUANT_THREADS + threadIdx.x) >> 5;
+  const uint32_t nwarps = (gridDim.x * QUANT_THREADS) >> 5;
+  const uint32_t segs = static_cast<uint32_t>((a.K + 256 * QUANT_UNROLL - 1) / (256 * QUANT_UNROLL));
+  const uint32_t units = static_cast<uint32_t>(a.rows) * segs;
   const float c = __fmul_rn(6.0f, a.gs);
   const int64_t code_ld = a.K / 2;
+  const int K = static_cast<int>(a.K);
 
-  for (int64_t u0 = gwarp; u0 < units; u0 += nwarps * QUANT_UNROLL) {
+  for (uint32_t u = gwarp; u < units; u += nwarps) {
+    const uint32_t r = u / segs;
+    const int k0 = static_cast<int>(u - r * segs) * (256 * QUANT_UNROLL) + lane * 8;
+    const __nv_bfloat16* src = a.x + static_cast<int64_t>(r) * a.ldx;
     uint4 raw[QUANT_UNROLL];
-    int64_t row[QUANT_UNROLL];
-    int kidx[QUANT_UNROLL];
-    bool valid[QUANT_UNROLL];
 #pragma unroll
     for (int i = 0; i < QUANT_UNROLL; ++i) {
-      const int64_t u = u0 + i * nwarps;
-      const bool in = u < units;
-      const int64_t r = in ? u / chunks : 0;
-      const int ch = in ? static_cast<int>(u - r * chunks) : 0;
-      row[i] = r;
-      kidx[i] = ch * 256 + lane * 8;
-      valid[i] = in && kidx[i] < a.K;
-      raw[i] = valid[i] ? ld_stream_v4(a.x + r * a.ldx + kidx[i]) : make_uint4(0, 0, 0, 0);
+      const int k = k0 + i * 256;
+      raw[i] = (k < K) ? ld_stream_v4(src + k) : make_uint4(0, 0, 0, 0);
     }
+    const int64_t grow = a.row0 + r;
 #pragma unroll
     for (int i = 0; i < QUANT_UNROLL; ++i) {
-      float f[8];
-      bf16x8_to_f32(raw[i], f);
-      float amax = 0.0f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
+      const int k = k0 + i * 256;
+      if (k0 - lane * 8 + i * 256 >= K) break;            // warp-uniform: chunk past the row end
+      float amax = bf16x8_absmax(raw[i]);
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
       const uint32_t s = cvt_e4m3(__fdiv_rn(amax, c));
       const float sdec = e4m3_value(s);
-      const float r = (sdec == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(sdec, a.gs));
-      float y[8];
+      const float rr = (sdec == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(sdec, a.gs));
+      float f[8];
+      bf16x8_to_f32(raw[i], f);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) y[e] = __fmul_rn(f[e], r);
-      uint32_t packed = cvt_e2m1x8(y);
+      for (int e = 0; e < 8; ++e) f[e] = __fmul_rn(f[e], rr);
+      uint32_t packed = cvt_e2m1x8(f);
       if (sdec == 0.0f) packed = 0;
       // scale bytes of blocks 4g..4g+3 (lanes 8g, 8g+2, 8g+4, 8g+6) -> lane 8g
       const uint32_t s1 = __shfl_down_sync(0xffffffffu, s, 2);
       const uint32_t s2 = __shfl_down_sync(0xffffffffu, s, 4);
       const uint32_t s3 = __shfl_down_sync(0xffffffffu, s, 6);
-      if (valid[i]) {
-        const int64_t grow = a.row0 + row[i];
-        *reinterpret_cast<uint32_t*>(a.codes + grow * code_ld + kidx[i] / 2) = packed;
+      if (k < K) {
+        *reinterpret_cast<uint32_t*>(a.codes + grow * code_ld + k / 2) = packed;
         if ((lane & 7) == 0) {
           const uint32_t word = s | (s1 << 8) | (s2 << 16) | (s3 << 24);
-          *reinterpret_cast<uint32_t*>(a.scales + sf_offset(grow, kidx[i] / 16, a.K)) = word;
+          *reinterpret_cast<uint32_t*>(a.scales + sf_offset(grow, k / 16, a.K)) = word;
         }
       }
     }
