@@ -155,6 +155,42 @@ nvfp4_status code_map(const void* ptr, int64_t rows, int64_t row_bytes, int box_
   return NVFP4_OK;
 }
 
+// 3-D uint64 map over a scale buffer in the 128x4 atom layout, viewed as
+// [row blocks of 128][K/64 atoms][64 x 8 bytes]; box = the 4 atoms of one
+// 256-element k-tile for `box_blocks` row blocks.  Atoms past K or past the
+// last row block read as zero.
+nvfp4_status scale_map(const void* ptr, int64_t rows, int64_t K, int box_blocks, int dev,
+                       CUtensorMap* out) {
+  const MapKey key{ptr, rows, K, -box_blocks, dev};
+  {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    auto it = g_maps.find(key);
+    if (it != g_maps.end()) {
+      *out = it->second;
+      return NVFP4_OK;
+    }
+  }
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return NVFP4_ERR_CUDA;
+  CUtensorMap m;
+  const int64_t kb4 = K / 64;
+  const int64_t blocks = (rows + 127) / 128;
+  const cuuint64_t dims[3] = {64u, static_cast<cuuint64_t>(kb4), static_cast<cuuint64_t>(blocks)};
+  const cuuint64_t strides[2] = {512u, static_cast<cuuint64_t>(kb4 * 512)};
+  const cuuint32_t box[3] = {64u, 4u, static_cast<cuuint32_t>(box_blocks)};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, const_cast<void*>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return NVFP4_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_map_mu);
+  if (g_maps.size() > 4096) g_maps.clear();
+  g_maps[key] = m;
+  *out = m;
+  return NVFP4_OK;
+}
+
 // ------------------------------------------------------------- validation
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -408,6 +444,8 @@ nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales, const
   g.y = y;
   g.ldy = ldy;
   g.out_fp32 = (out_dtype == NVFP4_OUT_FP32);
+  g.sector_stores = ((reinterpret_cast<uintptr_t>(y) & 31u) == 0) &&
+                    ((ldy * (g.out_fp32 ? 4 : 2)) % 32 == 0);
   g.wait_ns = g_wait_ns;
 
   const bool small = (g_gemm_path == 2) || (g_gemm_path == 0 && M <= 64);
@@ -433,9 +471,11 @@ nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales, const
     return launch(nvfp4::k_gemm_small<64>, nvfp4::sm::Cfg<64>::SMEM_BYTES);
   }
 
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tsa, tsb;
   if ((st = code_map(a_codes, M, K / 2, nvfp4::tc::BM, dev, &ta)) != NVFP4_OK) return st;
   if ((st = code_map(w_codes, N, K / 2, nvfp4::tc::BN, dev, &tb)) != NVFP4_OK) return st;
+  if ((st = scale_map(a_scales, M, K, 1, dev, &tsa)) != NVFP4_OK) return st;
+  if ((st = scale_map(w_scales, N, K, 2, dev, &tsb)) != NVFP4_OK) return st;
   if (!info->attr_tc) {
     if (cudaFuncSetAttribute(nvfp4::k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              nvfp4::tc::SMEM_BYTES) != cudaSuccess)
@@ -445,7 +485,8 @@ nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales, const
   const int64_t tiles = ((M + nvfp4::tc::BM - 1) / nvfp4::tc::BM) *
                         ((N + nvfp4::tc::BN - 1) / nvfp4::tc::BN);
   const int grid = static_cast<int>(tiles < info->sms ? tiles : info->sms);
-  nvfp4::k_gemm_tc<<<grid, nvfp4::tc::THREADS, nvfp4::tc::SMEM_BYTES, cs>>>(ta, tb, g, table);
+  nvfp4::k_gemm_tc<<<grid, nvfp4::tc::THREADS, nvfp4::tc::SMEM_BYTES, cs>>>(ta, tb, tsa, tsb, g,
+                                                                            table);
   return check_launch();
 }
 

@@ -53,6 +53,7 @@ struct GemmArgs {
   void* y;
   int64_t ldy;
   int out_fp32;
+  int sector_stores;   // y base 32-byte aligned and rows a multiple of 32 bytes
   uint64_t wait_ns;
 };
 
@@ -89,16 +90,23 @@ __device__ __forceinline__ int seg_advance(const SegTable& t, int seg, int n) {
 }
 
 // ============================================================ k_gemm_tc
-// Warp roles (12 warps):
-//   0  producer A: TMA of the activation codes + bulk copy of their scale atoms
-//   1  MMA issuer: tcgen05.mma only (one elected lane), TMEM allocation
-//   2  scale copier: tcgen05.cp of the stage's scale atoms into that stage's
-//      TMEM scale region, so the copies overlap the MMAs of the previous stage
-//   3  producer B: TMA of the weight codes + bulk copies of their scale atoms
-//   4-11 epilogue: warp w drains TMEM lane quarter w % 4, column half (w-4)/4
-// Per stage s the scale region is TMEM columns [256 + 48 s, 256 + 48 s + 48):
-// 16 columns of activation scales (4 MMAs x 4) then 32 of weight scales
-// (4 MMAs x 8).  The accumulator is columns [0, 256).
+// Warp roles (16 warps, four warpgroups):
+//   WG0  warp 0 producer A: TMA of the activation codes; warp 1 MMA issuer
+//        (tcgen05.mma only) and TMEM owner; warp 2 producer B: TMA of the
+//        weight codes; warp 3 producer S: TMA of both operands' scale atoms
+//        on a barrier of their own, so the scale writers need not wait for
+//        the 48 KB of codes.
+//   WG1  warps 4-7 scale writers: warp w reads, from the stage in shared
+//        memory, the scale bytes TMEM lane quarter w % 4 needs and writes
+//        them with tcgen05.st into that stage's TMEM scale region.  A
+//        tcgen05.cp costs the tensor pipe ~70-150 cycles whatever its size,
+//        and a k-tile needs 12 of them; register stores of the same bytes
+//        take ~40 cycles per stage and run beside the MMAs.
+//   WG2-3 warps 8-15 epilogue: warp w drains lane quarter w % 4, column
+//        half (w - 8) / 4.
+// TMEM: accumulator columns [0, 256); stage s scale region [256 + 48 s, +48):
+// 16 columns of activation scales (MMA kk reads column 4 kk + quarter) then
+// 32 of weight scales (MMA kk reads columns 8 kk + n / 32).
 namespace tc {
 constexpr int BM = 128;
 constexpr int BN = 256;
@@ -110,9 +118,13 @@ constexpr int B_BYTES = BN * BKB;       // 32 KB
 constexpr int SFA_BYTES = 4 * 512;      // 4 atoms (K = 64 each) x 128 rows
 constexpr int SFB_BYTES = 2 * 4 * 512;  // 2 row blocks of 128
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 54 KB
+constexpr int SFW_WARP0 = 4;            // scale writers: warps 4-7
+constexpr int EPI_WARP0 = 8;            // epilogue: warps 8-15
 constexpr int EPI_WARPS = 8;
-constexpr int EPI_WARP0 = 4;
-constexpr int THREADS = 32 * (EPI_WARP0 + EPI_WARPS);
+constexpr int THREADS = 512;
+constexpr uint32_t REGS_SMALL = 72;     // WG0 and WG1 after setmaxnreg
+constexpr uint32_t REGS_EPI = 184;      // WG2 and WG3 after setmaxnreg
+static_assert(2 * 128 * REGS_SMALL + 2 * 128 * REGS_EPI <= 65536, "register split");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
 constexpr uint32_t SF_COL = 256;        // + 48 * stage
@@ -123,16 +135,20 @@ static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
 static_assert(SF_COL + STAGES * SF_STRIDE <= TMEM_COLS, "TMEM budget");
 }  // namespace tc
 
+// tmA / tmB: code matrices [rows, K/2] (box 128 bytes x 128 / 256 rows, 128-byte
+// swizzle).  tmSA / tmSB: scale buffers viewed as [row blocks][K/64 atoms][64
+// u64] (box 64 x 4 x 1 / 2, i.e. one stage's atoms of 1 / 2 row blocks).
 __global__ void __launch_bounds__(tc::THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
               const GemmArgs g, const __grid_constant__ SegTable seg) {
   using namespace tc;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-  // bars: full[S], empty[S], sf_ready[S], tmem_full, tmem_empty, drain_mma, drain_sf
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 4);
+  // bars: full[S], empty[S], sf_ready[S], sf_full[S], tmem_full, tmem_empty, drain_mma
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 * STAGES + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -141,31 +157,31 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
   const int num_n = (g.N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
   const int num_kt = (g.K + BK - 1) / BK;
-  const int64_t kb4 = g.K / 64;            // scale atoms per 128-row block
-  const int sfb_blocks = (g.N + 127) / 128;
 
   auto full_bar = [&](int s) { return smem_addr(bars + s); };
   auto empty_bar = [&](int s) { return smem_addr(bars + STAGES + s); };
   auto sf_bar = [&](int s) { return smem_addr(bars + 2 * STAGES + s); };
-  const uint32_t tmem_full = smem_addr(bars + 3 * STAGES);
-  const uint32_t tmem_empty = smem_addr(bars + 3 * STAGES + 1);
-  const uint32_t drain_mma = smem_addr(bars + 3 * STAGES + 2);
-  const uint32_t drain_sf = smem_addr(bars + 3 * STAGES + 3);
+  auto sfull_bar = [&](int s) { return smem_addr(bars + 3 * STAGES + s); };
+  const uint32_t tmem_full = smem_addr(bars + 4 * STAGES);
+  const uint32_t tmem_empty = smem_addr(bars + 4 * STAGES + 1);
+  const uint32_t drain_mma = smem_addr(bars + 4 * STAGES + 2);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 2);            // both producers arrive (with their bytes)
       mbar_init(empty_bar(s), 1);
-      mbar_init(sf_bar(s), 1);
+      mbar_init(sf_bar(s), 4);              // the four scale writers
+      mbar_init(sfull_bar(s), 1);           // the scale producer
     }
     mbar_init(tmem_full, 1);
     mbar_init(tmem_empty, EPI_WARPS);
     mbar_init(drain_mma, 1);
-    mbar_init(drain_sf, 1);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
+    prefetch_tensormap(&tmSA);
+    prefetch_tensormap(&tmSB);
   }
   if (warp == 1) {
     tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
@@ -176,10 +192,11 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0 || warp == 3) {
+  // Each warpgroup resizes its registers at the top of its own branch.
+  if (warp < SFW_WARP0) regs_dealloc<REGS_SMALL>();
+  if (warp == 0 || warp == 2 || warp == 3) {
     // ---------------------------------------------------- TMA producers
     if (lane == 0) {
-      const bool is_a = (warp == 0);
       const uint64_t pol = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
@@ -188,8 +205,6 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int mb = tile % num_m;
         const int nb = tile / num_m;
-        const int nb0 = nb * 2;
-        const int nsfb = min(2, sfb_blocks - nb0);
         for (int kt = 0; kt < num_kt; ++kt) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, g.wait_ns, abort_flag)) {
             if (!*abort_flag) record_error(SITE_PRODUCER_EMPTY, warp);
@@ -197,19 +212,20 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             ok = false;
             break;
           }
-          const int nk = min(4, (g.K - kt * BK) / 64);
           uint8_t* st = smem + stage * STAGE_BYTES;
-          if (is_a) {
-            mbar_arrive_expect_tx(full_bar(stage), A_BYTES + nk * 512);
+          if (warp == 0) {
+            mbar_arrive_expect_tx(full_bar(stage), A_BYTES);
             tma_load_2d(smem_addr(st), &tmA, kt * BKB, mb * BM, full_bar(stage), pol);
-            bulk_load(smem_addr(st + A_BYTES + B_BYTES), g.sfa + (mb * kb4 + kt * 4) * 512,
-                      nk * 512, full_bar(stage), pol);
-          } else {
-            mbar_arrive_expect_tx(full_bar(stage), B_BYTES + nk * 512 * nsfb);
+          } else if (warp == 2) {
+            mbar_arrive_expect_tx(full_bar(stage), B_BYTES);
             tma_load_2d(smem_addr(st + A_BYTES), &tmB, kt * BKB, nb * BN, full_bar(stage), pol);
-            for (int j = 0; j < nsfb; ++j)
-              bulk_load(smem_addr(st + A_BYTES + B_BYTES + SFA_BYTES + j * 2048),
-                        g.sfb + ((nb0 + j) * kb4 + kt * 4) * 512, nk * 512, full_bar(stage), pol);
+          } else {
+            // both boxes always transfer their full size (out-of-range atoms read as 0)
+            mbar_arrive_expect_tx(sfull_bar(stage), SFA_BYTES + SFB_BYTES);
+            tma_load_3d(smem_addr(st + A_BYTES + B_BYTES), &tmSA, 0, kt * 4, mb, sfull_bar(stage),
+                        pol);
+            tma_load_3d(smem_addr(st + A_BYTES + B_BYTES + SFA_BYTES), &tmSB, 0, kt * 4, nb * 2,
+                        sfull_bar(stage), pol);
           }
           ++issued;
           if (++stage == STAGES) {
@@ -219,52 +235,87 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         }
       }
       // every copy this thread issued must land before the CTA may exit
+      const uint32_t mine = (warp == 3) ? 1u : 0u;
       for (int s = 0; s < STAGES && s < issued; ++s) {
         const int64_t uses = (issued - 1 - s) / STAGES + 1;
-        if (!mbar_wait(full_bar(s), static_cast<uint32_t>((uses - 1) & 1), g.wait_ns, nullptr))
+        const uint32_t bar = mine ? sfull_bar(s) : full_bar(s);
+        if (!mbar_wait(bar, static_cast<uint32_t>((uses - 1) & 1), g.wait_ns, nullptr))
           record_error(SITE_DRAIN, warp);
       }
     }
     __syncwarp();
-  } else if (warp == 2) {
-    // ---------------------------------------------------- scale copier
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
+  } else if (warp >= SFW_WARP0 && warp < EPI_WARP0) {
+    // ---------------------------------------------------- scale writers
+    regs_dealloc<REGS_SMALL>();
+    const int q = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        for (int kt = 0; kt < num_kt; ++kt) {
-          if (!mbar_wait(full_bar(stage), phase, g.wait_ns, abort_flag)) {
-            if (!*abort_flag) record_error(SITE_MMA_FULL, 2);
-            *abort_flag = 1;
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const int nk = min(4, (g.K - kt * BK) / 64);
-          const uint32_t sfa_s = smem_addr(smem + stage * STAGE_BYTES + A_BYTES + B_BYTES);
-          const uint32_t sfb_s = sfa_s + SFA_BYTES;
-          const uint32_t col = tmem_base + SF_COL + SF_STRIDE * stage;
-          for (int kk = 0; kk < nk; ++kk) {
-            tmem_cp_32x128b_x4(col + 4 * kk, desc_sf_atom(sfa_s + kk * 512));
-            tmem_cp_32x128b_x4(col + 16 + 8 * kk, desc_sf_atom(sfb_s + kk * 512));
-            tmem_cp_32x128b_x4(col + 16 + 8 * kk + 4, desc_sf_atom(sfb_s + 2048 + kk * 512));
-          }
-          tc_commit(sf_bar(stage));
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
+      for (int kt = 0; kt < num_kt; ++kt) {
+        if (!mbar_wait(sfull_bar(stage), phase, g.wait_ns, abort_flag)) {
+          if (!*abort_flag) record_error(SITE_MMA_FULL, warp);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        const uint32_t sfa_s = smem_addr(smem + stage * STAGE_BYTES + A_BYTES + B_BYTES);
+        const uint32_t sfb_s = sfa_s + SFA_BYTES;
+        uint32_t r[48];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          // activation row 32 q + lane, MMA kk: 4 scale bytes at atom kk
+          const uint32_t a = ld_shared_u32(sfa_s + kk * 512 + lane * 16 + q * 4);
+          r[4 * kk + 0] = a;
+          r[4 * kk + 1] = a;
+          r[4 * kk + 2] = a;
+          r[4 * kk + 3] = a;
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            // weight rows 128 j + 32 c + lane, c = 0..3 -> columns 8 kk + 4 j + c
+            const uint4 b = ld_shared_v4(sfb_s + j * 2048 + kk * 512 + lane * 16);
+            r[16 + 8 * kk + 4 * j + 0] = b.x;
+            r[16 + 8 * kk + 4 * j + 1] = b.y;
+            r[16 + 8 * kk + 4 * j + 2] = b.z;
+            r[16 + 8 * kk + 4 * j + 3] = b.w;
           }
         }
+        const uint32_t col = tmem_base + lane_off + SF_COL + SF_STRIDE * stage;
+        tmem_st_x32(col, r);
+        tmem_st_x16(col + 32, r + 32);
+        tmem_wait_st();
+        tc_fence_before();
+        // the MMA warp waits on this barrier alone: arrive only once the
+        // stage's codes have landed too
+        if (!mbar_wait(full_bar(stage), phase, g.wait_ns, abort_flag)) {
+          if (!*abort_flag) record_error(SITE_MMA_FULL, warp);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sf_bar(stage));
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
       }
-      tc_commit(drain_sf);
-      if (!mbar_wait(drain_sf, 0, g.wait_ns, nullptr)) record_error(SITE_DRAIN, 2);
+      if (!ok) break;
     }
-    __syncwarp();
   } else if (warp == 1) {
     // -------------------------------------------------------- MMA issuer
+    // The tensor pipe accepts about one MMA ahead of the issuing thread, so
+    // the thread's own bookkeeping shows up as pipe idle time: it waits on a
+    // single barrier per stage (the scale writers arrive only once both the
+    // codes and the scales of the stage are in place), uses precomputed
+    // descriptors, and releases the previous stage right after MMA 0.
     if (lane == 0) {
       const uint32_t idesc = idesc_mxf4nvf4(BM, BN);
+      // the start-address field holds (address >> 4) and every stage lies below
+      // 256 KB, so a stage's descriptor is the first one plus stage * STAGE_BYTES / 16
+      const uint64_t adesc0 = desc_kmajor_sw128(smem_addr(smem));
+      const uint64_t bdesc0 = desc_kmajor_sw128(smem_addr(smem + A_BYTES));
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
@@ -276,11 +327,9 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
           break;
         }
         tc_fence_after();
+        int prev = -1;
         for (int kt = 0; kt < num_kt; ++kt) {
-          // the scale copies of this stage imply its operands have landed (the
-          // copier waited on the full barrier); the full wait below is free
-          if (!mbar_wait(sf_bar(stage), phase, g.wait_ns, abort_flag) ||
-              !mbar_wait(full_bar(stage), phase, g.wait_ns, abort_flag)) {
+          if (!mbar_wait(sf_bar(stage), phase, g.wait_ns, abort_flag)) {
             if (!*abort_flag) record_error(SITE_MMA_FULL, 1);
             *abort_flag = 1;
             ok = false;
@@ -288,21 +337,22 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
           }
           tc_fence_after();
           const int nk = min(4, (g.K - kt * BK) / 64);
-          const uint8_t* st = smem + stage * STAGE_BYTES;
-          const uint64_t adesc = desc_kmajor_sw128(smem_addr(st));
-          const uint64_t bdesc = desc_kmajor_sw128(smem_addr(st + A_BYTES));
+          const uint64_t soff = static_cast<uint64_t>(stage) * (STAGE_BYTES >> 4);
+          const uint64_t ad = adesc0 + soff, bd = bdesc0 + soff;
           const uint32_t col = tmem_base + SF_COL + SF_STRIDE * stage;
-          for (int kk = 0; kk < nk; ++kk) {
-            // K = 64 fp4 = 32 bytes: advance the start address inside the swizzle atom
-            mma_mxf4nvf4(tmem_base + ACC_COL, adesc + 2 * kk, bdesc + 2 * kk, idesc, col + 4 * kk,
-                         col + 16 + 8 * kk, (kt | kk) != 0);
-          }
-          tc_commit(empty_bar(stage));
+          // K = 64 fp4 = 32 bytes per MMA: advance the start address inside the swizzle atom
+          mma_mxf4nvf4(tmem_base + ACC_COL, ad, bd, idesc, col, col + 16, kt != 0);
+          if (prev >= 0) tc_commit(empty_bar(prev));
+          for (int kk = 1; kk < nk; ++kk)
+            mma_mxf4nvf4(tmem_base + ACC_COL, ad + 2 * kk, bd + 2 * kk, idesc, col + 4 * kk,
+                         col + 16 + 8 * kk, 1u);
+          prev = stage;
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
+        if (prev >= 0) tc_commit(empty_bar(prev));
         if (!ok) break;
         tc_commit(tmem_full);
       }
@@ -311,8 +361,9 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       if (!mbar_wait(drain_mma, 0, g.wait_ns, nullptr)) record_error(SITE_DRAIN, 1);
     }
     __syncwarp();
-  } else {
+  } else if (warp >= EPI_WARP0) {
     // ---------------------------------------------------------- epilogue
+    regs_alloc<REGS_EPI>();
     const int q = warp & 3;                       // TMEM lane quarter this warp may access
     const int half = (warp - EPI_WARP0) >> 2;     // columns [128*half, 128*half + 128)
     const int row_in_tile = q * 32 + lane;
@@ -370,10 +421,13 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                 const __nv_bfloat162 p = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);
                 w[i] = *reinterpret_cast<const uint32_t*>(&p);
               }
-              uint4* dst =
-                  reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.y) + gm * g.ldy + n);
-              dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-              dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+              __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.y) + gm * g.ldy + n;
+              if (g.sector_stores) {
+                st_global_v8(dst, w);   // the row's 16 columns = one full 32-byte sector
+              } else {
+                reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+              }
             }
           }
         }
@@ -388,11 +442,13 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
 }
 
 // ========================================================== k_gemm_small
-// Warp roles (8 warps): 0 producer W (weight codes + scale atoms), 1 MMA
-// issuer, 2 scale copier, 3 producer X (token codes + scale atoms), 4-7
-// epilogue (warp w reads TMEM lane quarter w % 4).  TMEM: accumulator
+// Warp roles (12 warps): 0 producer W (weight codes + scale atoms), 1 MMA
+// issuer, 2 producer X (token codes + scale atoms), 3 idle, 4-7 scale
+// writers (tcgen05.st of the stage's scale bytes for lane quarter w % 4),
+// 8-11 epilogue (warp w reads TMEM lane quarter w % 4).  TMEM: accumulator
 // columns [0, NT); stage s scale region [64 + 32 s, 64 + 32 s + 32): 16
-// columns of weight scales then 16 of token scales (4 MMAs x 4 each).
+// columns of weight scales (MMA kk reads 4 kk + quarter) then 16 of token
+// scales (MMA kk reads 16 + 4 kk + token / 32).
 namespace sm {
 constexpr int BW = 128;                 // weight rows per CTA (MMA M)
 constexpr int BK = 256;
@@ -401,8 +457,9 @@ constexpr int STAGES = 6;
 constexpr int W_BYTES = BW * BKB;       // 16 KB
 constexpr int SFW_BYTES = 4 * 512;
 constexpr int SFX_BYTES = 4 * 512;
+constexpr int SFW_WARP0 = 4;
+constexpr int EPI_WARP0 = 8;
 constexpr int EPI_WARPS = 4;
-constexpr int EPI_WARP0 = 4;
 constexpr int THREADS = 32 * (EPI_WARP0 + EPI_WARPS);
 constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t ACC_COL = 0;         // NT columns
@@ -431,8 +488,8 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
-  // bars: full[S], empty[S], sf_ready[S], acc_full, drain_mma, drain_sf
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 3);
+  // bars: full[S], empty[S], sf_ready[S], acc_full, drain_mma
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -446,17 +503,15 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
   auto sf_bar = [&](int s) { return smem_addr(bars + 2 * STAGES + s); };
   const uint32_t acc_full = smem_addr(bars + 3 * STAGES);
   const uint32_t drain_mma = smem_addr(bars + 3 * STAGES + 1);
-  const uint32_t drain_sf = smem_addr(bars + 3 * STAGES + 2);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 2);
       mbar_init(empty_bar(s), 1);
-      mbar_init(sf_bar(s), 1);
+      mbar_init(sf_bar(s), 4);
     }
     mbar_init(acc_full, 1);
     mbar_init(drain_mma, 1);
-    mbar_init(drain_sf, 1);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&tmW);
@@ -471,7 +526,7 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0 || warp == 3) {
+  if (warp == 0 || warp == 2) {
     if (lane == 0) {
       const bool is_w = (warp == 0);
       // weights stream through once; tokens are re-read by every CTA
@@ -511,35 +566,43 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 2) {
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      for (int kt = 0; kt < num_kt; ++kt) {
-        if (!mbar_wait(full_bar(stage), phase, g.wait_ns, abort_flag)) {
-          if (!*abort_flag) record_error(SITE_MMA_FULL, 2);
-          *abort_flag = 1;
-          break;
-        }
-        tc_fence_after();
-        const int nk = min(4, (g.K - kt * BK) / 64);
-        const uint32_t sfw_s = smem_addr(smem + stage * C::STAGE_BYTES + W_BYTES + C::X_BYTES);
-        const uint32_t sfx_s = sfw_s + SFW_BYTES;
-        const uint32_t col = tmem_base + SF_COL + SF_STRIDE * stage;
-        for (int kk = 0; kk < nk; ++kk) {
-          tmem_cp_32x128b_x4(col + 4 * kk, desc_sf_atom(sfw_s + kk * 512));
-          tmem_cp_32x128b_x4(col + 16 + 4 * kk, desc_sf_atom(sfx_s + kk * 512));
-        }
-        tc_commit(sf_bar(stage));
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1u;
-        }
+  } else if (warp >= SFW_WARP0 && warp < EPI_WARP0) {
+    const int q = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int kt = 0; kt < num_kt; ++kt) {
+      if (!mbar_wait(full_bar(stage), phase, g.wait_ns, abort_flag)) {
+        if (!*abort_flag) record_error(SITE_MMA_FULL, warp);
+        *abort_flag = 1;
+        break;
       }
-      tc_commit(drain_sf);
-      if (!mbar_wait(drain_sf, 0, g.wait_ns, nullptr)) record_error(SITE_DRAIN, 2);
+      const uint32_t sfw_s = smem_addr(smem + stage * C::STAGE_BYTES + W_BYTES + C::X_BYTES);
+      const uint32_t sfx_s = sfw_s + SFW_BYTES;
+      uint32_t r[32];
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint32_t a = ld_shared_u32(sfw_s + kk * 512 + lane * 16 + q * 4);
+        r[4 * kk + 0] = a;
+        r[4 * kk + 1] = a;
+        r[4 * kk + 2] = a;
+        r[4 * kk + 3] = a;
+        const uint4 b = ld_shared_v4(sfx_s + kk * 512 + lane * 16);
+        r[16 + 4 * kk + 0] = b.x;
+        r[16 + 4 * kk + 1] = b.y;
+        r[16 + 4 * kk + 2] = b.z;
+        r[16 + 4 * kk + 3] = b.w;
+      }
+      tmem_st_x32(tmem_base + lane_off + SF_COL + SF_STRIDE * stage, r);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sf_bar(stage));
+      if (++stage == STAGES) {
+        stage = 0;
+        phase ^= 1u;
+      }
     }
-    __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = idesc_mxf4nvf4(BW, NT);
@@ -574,7 +637,7 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
       if (!mbar_wait(drain_mma, 0, g.wait_ns, nullptr)) record_error(SITE_DRAIN, 1);
     }
     __syncwarp();
-  } else {
+  } else if (warp >= EPI_WARP0) {
     const int q = warp & 3;
     const int n = wt * BW + q * 32 + lane;   // output feature of this lane
     if (mbar_wait(acc_full, 0, g.wait_ns, abort_flag)) {

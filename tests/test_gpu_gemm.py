@@ -174,3 +174,22 @@ def test_output_row_stride_and_no_overwrite():
         out = y.cpu().numpy()
         assert np.all(out[:, N:] == -7.0)
         H.check_gemm_fp32(out[:, :N], ref[:m], f"ldy path {path}")
+
+
+@pytest.mark.parametrize("ldy", [152, 160])
+def test_bf16_row_stride_both_store_widths(ldy):
+    """bf16 rows of 304 bytes take 16-byte stores, rows of 320 bytes whole 32-byte sectors."""
+    M, N, K = 200, 144, 256
+    rng = np.random.default_rng(ldy)
+    ac = rng.integers(0, 16, size=(M, K)).astype(np.uint8)
+    wc = rng.integers(0, 16, size=(N, K)).astype(np.uint8)
+    as_ = rng.integers(0x30, 0x40, size=(M, K // 16)).astype(np.uint8)
+    ws = rng.integers(0x30, 0x40, size=(N, K // 16)).astype(np.uint8)
+    A, W = dev_operands(ac, as_, M, K), dev_operands(wc, ws, N, K)
+    nv.nvfp4_set_gemm_path(LARGE)
+    y32 = nv.nvfp4_linear(A[0], A[1], 0.01, W[0], W[1], 0.02, M, N, K, out_dtype=nv.OUT_FP32)
+    y = torch.full((M, ldy), 3.0, dtype=torch.bfloat16, device="cuda")
+    nv.nvfp4_linear(A[0], A[1], 0.01, W[0], W[1], 0.02, M, N, K, y=y[:, :N])
+    out = y.float().cpu().numpy()
+    assert np.all(out[:, N:] == 3.0)
+    np.testing.assert_array_equal(out[:, :N], H.bf16_round(y32.cpu().numpy()))
