@@ -145,6 +145,30 @@ nvfp4_status nvfp4_quantize_weight(const void* w_bf16, int64_t N, int64_t K, int
                                    float* w_gs_out, void* codes, void* scales,
                                    void* workspace, nvfp4_stream_t stream);
 
+/* Weight quantisation that allocates nothing and takes no workspace.
+ * The paper has no counterpart; this is a library convenience.
+ * Some callers cannot call cudaMalloc at all: a serving runtime or plugin
+ * host that owns every byte of device memory through its own arena and hands
+ * an operator only its input and output buffers, or an embedded caller whose
+ * device-memory budget is fixed when it starts.  Such callers cannot create
+ * the workspace nvfp4_quantize_weight needs.  This entry point computes the
+ * same result (same codes, scales and w_gs) with its per-module amax scratch
+ * in a fixed array inside the library: NVFP4_NOALLOC_MAX_SEGMENTS floats
+ * (128 bytes), which every GPU that loads the library keeps until the
+ * process exits.  nseg above NVFP4_NOALLOC_MAX_SEGMENTS is rejected with
+ * NVFP4_ERR_INVALID_ARG before anything runs.  The first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress) with that
+ * device current; make that first call before any stream capture.  All
+ * calls share the one array per device: the accumulators are cleared on
+ * `stream` at the start of every call, and calls whose work overlaps on the
+ * GPU (e.g. on different streams) race on it.  Arguments, layouts and the
+ * synchronisation of `stream` are those of nvfp4_quantize_weight. */
+#define NVFP4_NOALLOC_MAX_SEGMENTS 32
+nvfp4_status nvfp4_quantize_weight_noalloc(const void* w_bf16, int64_t N, int64_t K, int64_t ldw,
+                                           const int64_t* seg_offsets, int32_t nseg,
+                                           float* w_gs_out, void* codes, void* scales,
+                                           nvfp4_stream_t stream);
+
 /* Block-scaled FP4 x FP4 GEMM (step a3) with a single module (step a4 with
  * op NONE): y[m, n] = fp32(a_gs * w_gs) * sum_k xhat[m,k] * what[n,k] / (a_gs w_gs),
  * i.e. the product of the dequantised operands, accumulated in fp32.

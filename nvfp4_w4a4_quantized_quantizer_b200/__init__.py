@@ -19,7 +19,8 @@ from ._lib import (NVFP4Error, OP_GDN_DECAY, OP_NONE, OP_SIGMOID, OUT_BF16, OUT_
 
 __all__ = [
     "nvfp4_codes_bytes", "nvfp4_scale_bytes", "nvfp4_global_scale", "nvfp4_amax",
-    "nvfp4_quantize_act", "nvfp4_quantize_weight", "nvfp4_linear", "nvfp4_fused_linear",
+    "nvfp4_quantize_act", "nvfp4_quantize_weight", "nvfp4_quantize_weight_noalloc",
+    "nvfp4_linear", "nvfp4_fused_linear",
     "nvfp4_silu_mul", "nvfp4_last_device_error", "nvfp4_set_gemm_path",
     "nvfp4_set_wait_limit_ns", "nvfp4_test_e2m1", "nvfp4_test_e4m3", "nvfp4_test_wait_timeout",
     "SegmentSpec", "NVFP4Error", "OP_NONE", "OP_SIGMOID", "OP_GDN_DECAY",
@@ -98,6 +99,28 @@ def nvfp4_quantize_weight(w: torch.Tensor, seg_offsets: Optional[Sequence[int]] 
     check(lib.nvfp4_quantize_weight(_ptr(w), N, K, _ld(w), offs_c, nseg, gs_c, _ptr(codes),
                                     _ptr(scales), _ptr(workspace), _stream(stream)),
           "nvfp4_quantize_weight")
+    return codes, scales, [float(v) for v in gs_c]
+
+
+def nvfp4_quantize_weight_noalloc(w: torch.Tensor, seg_offsets: Optional[Sequence[int]] = None,
+                                  codes: Optional[torch.Tensor] = None,
+                                  scales: Optional[torch.Tensor] = None, stream=None):
+    """nvfp4_quantize_weight for callers that cannot allocate device memory: no
+    workspace; the library's fixed scratch array holds the per-module amax.
+    (This wrapper allocates outputs only when they are not passed in.)"""
+    lib = load()
+    N, K = w.shape
+    offs = list(seg_offsets) if seg_offsets is not None else [0]
+    nseg = len(offs)
+    if codes is None:
+        codes = torch.empty((N, K // 2), dtype=torch.uint8, device=w.device)
+    if scales is None:
+        scales = torch.empty(nvfp4_scale_bytes(N, K), dtype=torch.uint8, device=w.device)
+    offs_c = (ctypes.c_int64 * nseg)(*offs)
+    gs_c = (ctypes.c_float * nseg)()
+    check(lib.nvfp4_quantize_weight_noalloc(_ptr(w), N, K, _ld(w), offs_c, nseg, gs_c, _ptr(codes),
+                                            _ptr(scales), _stream(stream)),
+          "nvfp4_quantize_weight_noalloc")
     return codes, scales, [float(v) for v in gs_c]
 
 

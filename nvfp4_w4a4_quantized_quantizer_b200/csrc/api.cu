@@ -271,6 +271,39 @@ nvfp4_status build_segments(const nvfp4_segment* segs, int32_t nseg, int64_t N, 
   return NVFP4_OK;
 }
 
+// ------------------------------------------ weight quantisation, no allocation
+// Scratch of nvfp4_quantize_weight_noalloc: the per-module amax accumulators.
+// A fixed array in the library's device image; every GPU that loads the
+// library holds it (NVFP4_NOALLOC_MAX_SEGMENTS floats) until the process exits.
+static __device__ __align__(256) float g_noalloc_amax[NVFP4_NOALLOC_MAX_SEGMENTS];
+
+float* g_noalloc_ptr[MAX_DEVICES] = {};
+std::mutex g_noalloc_mu;
+
+// The array's device address on the current device.  In host code the name
+// g_noalloc_amax is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+nvfp4_status noalloc_scratch(float** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= MAX_DEVICES) return NVFP4_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_amax);
+    if (e != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return NVFP4_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return NVFP4_OK;
+}
+
 }  // namespace
 
 // =================================================================== C ABI
@@ -408,6 +441,24 @@ nvfp4_status nvfp4_quantize_weight(const void* w, int64_t N, int64_t K, int64_t 
     if (st != NVFP4_OK) return st;
   }
   return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_quantize_weight_noalloc(const void* w, int64_t N, int64_t K, int64_t ldw,
+                                           const int64_t* seg_offsets, int32_t nseg,
+                                           float* w_gs_out, void* codes, void* scales,
+                                           nvfp4_stream_t stream) {
+  if (nseg < 1 || nseg > NVFP4_NOALLOC_MAX_SEGMENTS) return NVFP4_ERR_INVALID_ARG;
+  nvfp4_status st = check_bf16_matrix(w, N, K, ldw);
+  if (st != NVFP4_OK) return st;
+  if (codes == nullptr || scales == nullptr || w_gs_out == nullptr) return NVFP4_ERR_INVALID_ARG;
+  int dev;
+  DeviceInfo* info;
+  if ((st = current_device(&dev, &info)) != NVFP4_OK) return st;
+  float* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != NVFP4_OK) return st;
+  // the workspace path clears each module's accumulator on `stream` before use
+  return nvfp4_quantize_weight(w, N, K, ldw, seg_offsets, nseg, w_gs_out, codes, scales, scratch,
+                               stream);
 }
 
 nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales, const void* w_codes,
