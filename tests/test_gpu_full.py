@@ -1,0 +1,195 @@
+"""GPU parity at the full sizes of every workload, on sampled outputs.
+
+The CUDA path runs each workload at its full size through the same calls
+bench.py times (nvfp4_quantize_act + nvfp4_fused_linear, automatic kernel
+choice).  The oracle recomputes sampled rows: the activation rows are
+quantised by the oracle (codes and scales must match bit for bit), the
+weights are quantised by the oracle with each module's own global scale
+(codes and scales of sampled weight rows must match bit for bit), and the
+sampled output rows are compared with the float64 product under the stated
+bar (fp32 max |err| <= 1e-3 rms, relative Frobenius <= 1e-5; bf16 output =
+RNE of the fp32 output; gates within their Lipschitz-propagated bounds).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+import nvfp4_w4a4_quantized_quantizer_b200 as nv
+from tests import _helpers as H
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+OPS = {"none": nv.OP_NONE, "sigmoid": nv.OP_SIGMOID, "gdn_decay": nv.OP_GDN_DECAY}
+
+
+def _sample_rows(M, n, seed):
+    rng = np.random.default_rng(seed)
+    fixed = [0, M - 1] + [r for r in (127, 128, 255, 256) if r < M]
+    rest = rng.choice(M, size=max(0, n - len(fixed)), replace=False)
+    return np.unique(np.concatenate([fixed, rest]).astype(np.int64))
+
+
+def _oracle_weights(wf, wl, rows=None):
+    """Per-module gs (whole module) and dequantised weight rows (all, or `rows`)."""
+    offs = wl.seg_offsets + [wl.N]
+    gs = [oracle.global_scale(np.abs(wf[offs[i]:offs[i + 1]]).max()) for i in range(len(wl.segments))]
+    rows = np.arange(wl.N) if rows is None else np.asarray(rows)
+    seg = np.searchsorted(np.array(offs), rows, side="right") - 1
+    codes = np.empty((len(rows), wl.K), np.uint8)
+    scales = np.empty((len(rows), wl.K // 16), np.uint8)
+    what = np.empty((len(rows), wl.K), np.float64)
+    for s in range(len(wl.segments)):
+        idx = np.nonzero(seg == s)[0]
+        for c in range(0, len(idx), 2048):
+            sel = idx[c:c + 2048]
+            q, sc = oracle.quantize(wf[rows[sel]], gs[s])
+            codes[sel], scales[sel] = q, sc
+            what[sel] = oracle.dequantize(q, sc, gs[s])
+    return gs, codes, scales, what
+
+
+def _gpu_layer(wl, xbits, wbits, calib_bits):
+    a_gs = nv.nvfp4_global_scale(nv.nvfp4_amax(H.bf16_dev(calib_bits)).item())
+    ac, as_ = nv.nvfp4_quantize_act(H.bf16_dev(xbits), a_gs)
+    wc, ws, w_gs = nv.nvfp4_quantize_weight(H.bf16_dev(wbits), seg_offsets=wl.seg_offsets)
+    gate = {}
+    if any(s.op == "gdn_decay" for s in wl.segments):
+        a_log, dt = workloads.gate_params(wl)
+        gate = dict(a_log=torch.from_numpy(a_log).cuda(), dt=torch.from_numpy(dt).cuda())
+    specs = [nv.SegmentSpec(o, w_gs[i], a_gs, OPS[s.op],
+                            gate.get("a_log") if s.op == "gdn_decay" else None,
+                            gate.get("dt") if s.op == "gdn_decay" else None)
+             for i, (s, o) in enumerate(zip(wl.segments, wl.seg_offsets))]
+    M = xbits.shape[0]
+    y32 = nv.nvfp4_fused_linear(ac, as_, wc, ws, M, wl.N, wl.K, specs, out_dtype=nv.OUT_FP32)
+    yb = nv.nvfp4_fused_linear(ac, as_, wc, ws, M, wl.N, wl.K, specs)
+    st, info = nv.nvfp4_last_device_error()
+    assert st == 0, hex(info)
+    return a_gs, w_gs, ac, as_, wc, ws, y32, yb
+
+
+def _check_layer(wl, M, rows_sample, wrow_sample, seed):
+    calib = workloads.activations(wl, calib=True)
+    xbits = workloads.activations(wl, M=M)
+    wbits = workloads.weights(wl)
+    a_gs, w_gs, ac, as_, wc, ws, y32, yb = _gpu_layer(wl, xbits, wbits, calib)
+    # calibration: exact
+    a_gs_ref = oracle.global_scale(np.abs(H.f32(calib)).max())
+    assert np.float32(a_gs) == a_gs_ref
+    # activations: sampled rows bit-exact
+    rs = _sample_rows(M, rows_sample, seed)
+    xf = H.f32(xbits[rs])
+    qx, sx = oracle.quantize(xf, a_gs_ref)
+    codes_gpu = H.unpack_codes(ac.cpu().numpy()[rs])
+    np.testing.assert_array_equal(codes_gpu, qx)
+    np.testing.assert_array_equal(H.sf_logical(as_.cpu().numpy(), M, wl.K)[rs], sx)
+    # weights: per-module gs exact, sampled rows bit-exact
+    wf = H.f32(wbits)
+    gs_ref, wq, wsc, what = _oracle_weights(wf, wl)
+    assert [np.float32(g) for g in w_gs] == gs_ref
+    ws_rows = _sample_rows(wl.N, wrow_sample, seed + 1)
+    np.testing.assert_array_equal(H.unpack_codes(wc.cpu().numpy()[ws_rows]), wq[ws_rows])
+    np.testing.assert_array_equal(H.sf_logical(ws.cpu().numpy(), wl.N, wl.K)[ws_rows], wsc[ws_rows])
+    # outputs of the sampled rows
+    pre = oracle.dequantize(qx, sx, a_gs_ref) @ what.T
+    y = y32.cpu().numpy()[rs]
+    ybf = yb.float().cpu().numpy()[rs]
+    offs = wl.seg_offsets + [wl.N]
+    for i, s in enumerate(wl.segments):
+        sl = slice(offs[i], offs[i + 1])
+        if s.op == "none":
+            H.check_gemm_fp32(y[:, sl], pre[:, sl], f"{wl.name} module {s.name}")
+            H.check_bf16_out(ybf[:, sl], y[:, sl], pre[:, sl], f"{wl.name} module {s.name}")
+            continue
+        e = 1e-3 * np.sqrt(np.mean(pre[:, sl] ** 2))
+        if s.op == "sigmoid":
+            ref = oracle.sigmoid64(pre[:, sl])
+            assert np.all(np.abs(y[:, sl] - ref) <= 0.25 * e + 2e-6), s.name
+        else:
+            a_log, dt = workloads.gate_params(wl)
+            ref = oracle.gdn_decay64(pre[:, sl], a_log[None, :], dt[None, :])
+            bound = np.exp(a_log)[None, :] * e + 2e-5 * np.abs(ref) + 1e-6
+            assert np.all(np.abs(y[:, sl] - ref) <= bound), s.name
+        np.testing.assert_array_equal(ybf[:, sl], H.bf16_round(y[:, sl]))
+
+
+def test_prefill_full():
+    _check_layer(workloads.WORKLOADS[2], 4096, 48, 256, seed=20)
+
+
+def test_gdn_inproj_full():
+    _check_layer(workloads.WORKLOADS[3], 8192, 32, 256, seed=30)
+
+
+@pytest.mark.parametrize("M", [1, 8, 32, 64])
+def test_decode_sweep_full(M):
+    _check_layer(workloads.WORKLOADS[5], M, M, 256, seed=50 + M)
+
+
+def test_mlp_pair_full():
+    """gate_up at full size (sampled rows and weight rows), then the down
+    projection at full K and N on the oracle's own SiLU(gate)*up rows, then the
+    whole GPU chain at full size as a consistency check."""
+    wl = workloads.WORKLOADS[4]
+    M, K, H2 = wl.M, wl.K, wl.N // 2
+    calib = workloads.activations(wl, calib=True)
+    xbits = workloads.activations(wl)
+    wbits = workloads.weights(wl)
+    a_gs, w_gs, ac, as_, wc, ws, y32, yb = _gpu_layer(wl, xbits, wbits, calib)
+    a_gs_ref = oracle.global_scale(np.abs(H.f32(calib)).max())
+    assert np.float32(a_gs) == a_gs_ref
+    rs = _sample_rows(M, 16, 40)
+    qx, sx = oracle.quantize(H.f32(xbits[rs]), a_gs_ref)
+    np.testing.assert_array_equal(H.unpack_codes(ac.cpu().numpy()[rs]), qx)
+    wf = H.f32(wbits)
+    del wbits
+    gs_ref, wq, wsc, what = _oracle_weights(wf, wl)
+    del wf
+    assert [np.float32(g) for g in w_gs] == gs_ref
+    wrows = _sample_rows(wl.N, 256, 41)
+    np.testing.assert_array_equal(H.unpack_codes(wc.cpu().numpy()[wrows]), wq[wrows])
+    del wq, wsc
+    gu = oracle.dequantize(qx, sx, a_gs_ref) @ what.T          # [16, 34816]
+    del what
+    y = y32.cpu().numpy()[rs]
+    for sl in (slice(0, H2), slice(H2, 2 * H2)):
+        H.check_gemm_fp32(y[:, sl], gu[:, sl], "gate_up")
+    H.check_bf16_out(yb.float().cpu().numpy()[rs], y, gu, "gate_up")
+
+    # down projection at full K = 17408, N = 5120 on the oracle's h rows
+    h_ref = oracle.silu_mul_bf16(gu[:, :H2], gu[:, H2:])        # float32 bf16 values [16, 17408]
+    h_calib = h_ref                                             # calibrated on these rows
+    a2 = oracle.global_scale(np.abs(h_calib).max())
+    w2bits = workloads.down_weights()
+    w2f = H.f32(w2bits)
+    g2 = oracle.global_scale(np.abs(w2f).max())
+    q2, s2 = oracle.quantize(w2f, g2)
+    w2hat = oracle.dequantize(q2, s2, g2)
+    del w2f
+    qh, sh = oracle.quantize(h_ref, a2)
+    hc, hs = nv.nvfp4_quantize_act(H.bf16_dev(workloads.f32_to_bf16_bits(h_ref)), a2)
+    np.testing.assert_array_equal(H.unpack_codes(hc.cpu().numpy()), qh)
+    w2c, w2s, (g2_gpu,) = nv.nvfp4_quantize_weight(H.bf16_dev(w2bits))
+    assert np.float32(g2_gpu) == g2
+    d32 = nv.nvfp4_linear(hc, hs, a2, w2c, w2s, g2_gpu, len(rs), workloads.MLP_DOWN_N,
+                          workloads.MLP_DOWN_K, out_dtype=nv.OUT_FP32).cpu().numpy()
+    dref = oracle.dequantize(qh, sh, a2) @ w2hat.T
+    H.check_gemm_fp32(d32, dref, "down")
+
+    # the full GPU chain (gate_up bf16 -> silu*up -> requantise -> down) at M = 16384.
+    # Its h differs from the oracle's by the bf16 rounding of gate / up, which
+    # moves some codes by a grid step when h is requantised, so it is held to a
+    # bound derived from the format itself: the chain's deviation from the oracle
+    # chain must stay below half of what NVFP4 quantisation of h costs.
+    d_unquantised = h_ref.astype(np.float64) @ w2hat.T
+    quant_err = np.linalg.norm(dref - d_unquantised)
+    h = nv.nvfp4_silu_mul(yb, H2)
+    hc2, hs2 = nv.nvfp4_quantize_act(h, a2)
+    d_full = nv.nvfp4_linear(hc2, hs2, a2, w2c, w2s, g2_gpu, M, workloads.MLP_DOWN_N,
+                             workloads.MLP_DOWN_K, out_dtype=nv.OUT_FP32)
+    assert nv.nvfp4_last_device_error()[0] == 0
+    d_rows = d_full.cpu().numpy()[rs]
+    assert np.all(np.isfinite(d_rows))
+    assert np.linalg.norm(d_rows - dref) <= 0.5 * quant_err
