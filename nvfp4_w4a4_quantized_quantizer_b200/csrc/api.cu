@@ -229,7 +229,16 @@ nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t K, int64_t ld,
   a.scales = static_cast<uint8_t*>(scales);
   a.pad_from = pad_from;
   a.pad_to = pad_to;
-  const int64_t units = rows * ((K + 256 * nvfp4::QUANT_UNROLL - 1) / (256 * nvfp4::QUANT_UNROLL));
+  // r[s] = fp32(1 / fp32(s_dec * gs)): IEEE fp32 host arithmetic rounds like
+  // the device's correctly rounded reciprocal; s_dec is exact in fp32
+  for (int code = 0; code < 128; ++code) {
+    const int e = (code >> 3) & 0xF, m = code & 7;
+    const float sdec = (e == 0) ? static_cast<float>(m) * 0.001953125f
+                                : std::ldexp(1.0f + static_cast<float>(m) / 8.0f, e - 7);
+    volatile float p = sdec * gs;   // volatile: keep the two fp32 roundings separate
+    a.rtab[code] = (sdec == 0.0f || code == 127) ? 0.0f : 1.0f / p;
+  }
+  const int64_t units = rows * ((K + 512 * nvfp4::QUANT_CHUNKS - 1) / (512 * nvfp4::QUANT_CHUNKS));
   if (units >= (1ll << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   const int warps_per_block = nvfp4::QUANT_THREADS / 32;
   const int grid = grid_for(units, warps_per_block, sms * 8);

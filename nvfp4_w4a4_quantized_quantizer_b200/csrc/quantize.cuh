@@ -12,13 +12,15 @@
 // Every rounding is an explicit _rn intrinsic or a .rn conversion, so the
 // compiler cannot contract or reorder it.
 //
-// Work mapping: one warp handles one (row, 256-element chunk) unit per step:
-// lane t loads elements 8t..8t+7 (one 16-byte load; the warp reads 512
-// contiguous bytes), lanes 2b and 2b+1 form 16-element block b and exchange
-// their partial amax with one shuffle, each lane writes 4 code bytes (the
-// warp writes 128 contiguous bytes), and every 8th lane gathers the four
-// scale bytes of blocks j..j+3 (contiguous in the atom layout) into one
-// 32-bit store.  Each warp keeps UNROLL units in flight.
+// Work mapping: a warp work unit is (row, 1024-element segment); lane t owns
+// one whole 16-element block per 512-element chunk (one 32-byte load; the
+// warp reads 1 KB contiguous), writes its 8 code bytes (the warp writes 256
+// contiguous bytes), and every 4th lane gathers the scale bytes of blocks
+// j..j+3 (contiguous in the atom layout) into one 32-bit store.  The block
+// reciprocal r depends only on the scale code, so the launch carries the
+// 128-entry table r[s] = fp32(1 / fp32(s_dec * gs)) (0 for s = 0), computed
+// on the host with IEEE fp32 arithmetic — the same rounding as the device
+// reciprocal — instead of a decode, a multiply and a reciprocal per block.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -78,6 +80,7 @@ struct QuantArgs {
   uint8_t* scales;         // base of the full scale buffer (atom layout)
   int64_t pad_from;        // zero scale rows [pad_from, pad_to)
   int64_t pad_to;
+  float rtab[128];         // fp32(1 / fp32(e4m3(s) * gs)), 0 for s == 0
 };
 
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
@@ -98,25 +101,36 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
 }
 
 constexpr int QUANT_THREADS = 256;
-constexpr int QUANT_UNROLL = 4;            // 256-element chunks per warp work unit
+constexpr int QUANT_CHUNKS = 2;            // 512-element chunks per warp work unit
 
-// |x| max of eight bf16 values, exact, with packed bf16x2 instructions.
-__device__ __forceinline__ float bf16x8_absmax(const uint4& v) {
-  const __nv_bfloat162 a = __habs2(*reinterpret_cast<const __nv_bfloat162*>(&v.x));
-  const __nv_bfloat162 b = __habs2(*reinterpret_cast<const __nv_bfloat162*>(&v.y));
-  const __nv_bfloat162 c = __habs2(*reinterpret_cast<const __nv_bfloat162*>(&v.z));
-  const __nv_bfloat162 d = __habs2(*reinterpret_cast<const __nv_bfloat162*>(&v.w));
-  const __nv_bfloat162 m = __hmax2(__hmax2(a, b), __hmax2(c, d));
-  return fmaxf(__low2float(m), __high2float(m));
+__device__ __forceinline__ void ld_stream_v8(const void* p, uint32_t (&w)[8]) {
+  asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]),
+                 "=r"(w[6]), "=r"(w[7])
+               : "l"(p));
 }
 
-// A warp work unit is (row, 1024-element segment of the row); the host
-// guarantees rows * segments < 2^31 so the unit index stays 32-bit.
-__global__ void __launch_bounds__(QUANT_THREADS) k_quantize(const QuantArgs a) {
+// |x| max of sixteen bf16 values (eight packed words), exact: the magnitude
+// bits of non-negative bf16 values order like unsigned integers.
+__device__ __forceinline__ float bf16x16_absmax(const uint32_t (&w)[8]) {
+  uint32_t m = __vmaxu2(w[0] & 0x7FFF7FFFu, w[1] & 0x7FFF7FFFu);
+  m = __vmaxu2(m, w[2] & 0x7FFF7FFFu);
+  m = __vmaxu2(m, w[3] & 0x7FFF7FFFu);
+  m = __vmaxu2(m, w[4] & 0x7FFF7FFFu);
+  m = __vmaxu2(m, w[5] & 0x7FFF7FFFu);
+  m = __vmaxu2(m, w[6] & 0x7FFF7FFFu);
+  m = __vmaxu2(m, w[7] & 0x7FFF7FFFu);
+  const uint32_t hi = m >> 16, lo = m & 0xFFFFu;
+  return __uint_as_float((hi > lo ? hi : lo) << 16);
+}
+
+// A warp work unit is (row, 1024-element segment); the host guarantees
+// rows * segments < 2^31 so the unit index stays 32-bit.
+__global__ void __launch_bounds__(QUANT_THREADS) k_quantize(const __grid_constant__ QuantArgs a) {
   const int lane = threadIdx.x & 31;
   const uint32_t gwarp = (blockIdx.x * QUANT_THREADS + threadIdx.x) >> 5;
   const uint32_t nwarps = (gridDim.x * QUANT_THREADS) >> 5;
-  const uint32_t segs = static_cast<uint32_t>((a.K + 256 * QUANT_UNROLL - 1) / (256 * QUANT_UNROLL));
+  const uint32_t segs = static_cast<uint32_t>((a.K + 512 * QUANT_CHUNKS - 1) / (512 * QUANT_CHUNKS));
   const uint32_t units = static_cast<uint32_t>(a.rows) * segs;
   const float c = __fmul_rn(6.0f, a.gs);
   const int64_t code_ld = a.K / 2;
@@ -124,37 +138,46 @@ __global__ void __launch_bounds__(QUANT_THREADS) k_quantize(const QuantArgs a) {
 
   for (uint32_t u = gwarp; u < units; u += nwarps) {
     const uint32_t r = u / segs;
-    const int k0 = static_cast<int>(u - r * segs) * (256 * QUANT_UNROLL) + lane * 8;
+    const int k0 = static_cast<int>(u - r * segs) * (512 * QUANT_CHUNKS) + lane * 16;
     const __nv_bfloat16* src = a.x + static_cast<int64_t>(r) * a.ldx;
-    uint4 raw[QUANT_UNROLL];
+    uint32_t w[QUANT_CHUNKS][8];
 #pragma unroll
-    for (int i = 0; i < QUANT_UNROLL; ++i) {
-      const int k = k0 + i * 256;
-      raw[i] = (k < K) ? ld_stream_v4(src + k) : make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < QUANT_CHUNKS; ++i) {
+      const int k = k0 + i * 512;
+      if (k < K) {
+        ld_stream_v8(src + k, w[i]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[i][e] = 0u;
+      }
     }
     const int64_t grow = a.row0 + r;
 #pragma unroll
-    for (int i = 0; i < QUANT_UNROLL; ++i) {
-      const int k = k0 + i * 256;
-      if (k0 - lane * 8 + i * 256 >= K) break;            // warp-uniform: chunk past the row end
-      float amax = bf16x8_absmax(raw[i]);
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    for (int i = 0; i < QUANT_CHUNKS; ++i) {
+      if (k0 - lane * 16 + i * 512 >= K) break;            // warp-uniform: chunk past the row end
+      const int k = k0 + i * 512;
+      const float amax = bf16x16_absmax(w[i]);
       const uint32_t s = cvt_e4m3(__fdiv_rn(amax, c));
-      const float sdec = e4m3_value(s);
-      const float rr = (sdec == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(sdec, a.gs));
+      const float rr = a.rtab[s];
       float f[8];
-      bf16x8_to_f32(raw[i], f);
+      uint32_t q[2];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) f[e] = __fmul_rn(f[e], rr);
-      uint32_t packed = cvt_e2m1x8(f);
-      if (sdec == 0.0f) packed = 0;
-      // scale bytes of blocks 4g..4g+3 (lanes 8g, 8g+2, 8g+4, 8g+6) -> lane 8g
-      const uint32_t s1 = __shfl_down_sync(0xffffffffu, s, 2);
-      const uint32_t s2 = __shfl_down_sync(0xffffffffu, s, 4);
-      const uint32_t s3 = __shfl_down_sync(0xffffffffu, s, 6);
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          f[2 * e] = __fmul_rn(__uint_as_float(w[i][4 * h + e] << 16), rr);
+          f[2 * e + 1] = __fmul_rn(__uint_as_float(w[i][4 * h + e] & 0xFFFF0000u), rr);
+        }
+        q[h] = cvt_e2m1x8(f);
+      }
+      if (s == 0) q[0] = q[1] = 0u;
+      // scale bytes of blocks 4g..4g+3 (lanes 4g..4g+3) -> lane 4g
+      const uint32_t s1 = __shfl_down_sync(0xffffffffu, s, 1);
+      const uint32_t s2 = __shfl_down_sync(0xffffffffu, s, 2);
+      const uint32_t s3 = __shfl_down_sync(0xffffffffu, s, 3);
       if (k < K) {
-        *reinterpret_cast<uint32_t*>(a.codes + grow * code_ld + k / 2) = packed;
-        if ((lane & 7) == 0) {
+        *reinterpret_cast<uint2*>(a.codes + grow * code_ld + k / 2) = make_uint2(q[0], q[1]);
+        if ((lane & 3) == 0) {
           const uint32_t word = s | (s1 << 8) | (s2 << 16) | (s3 << 24);
           *reinterpret_cast<uint32_t*>(a.scales + sf_offset(grow, k / 16, a.K)) = word;
         }
