@@ -211,8 +211,11 @@ const char* nvfp4_status_string(nvfp4_status status);
 nvfp4_status nvfp4_last_device_error(nvfp4_stream_t stream, uint64_t* info);
 
 /* Kernel-path selection for tests: 0 = automatic (M <= 64 -> small-M
- * kernel), 1 = always the persistent tensor-core kernel, 2 = always the
- * small-M kernel (requires M <= 64).  Process-wide. */
+ * kernel, 64 < M <= 128 -> one-CTA tensor-core kernel, M > 128 -> CTA-pair
+ * tensor-core kernel), 1 = always the one-CTA tensor-core kernel (128 x 256
+ * tiles), 2 = always the small-M kernel (requires M <= 64), 3 = always the
+ * CTA-pair tensor-core kernel (256 x 256 tiles on clusters of two CTAs).
+ * Process-wide. */
 nvfp4_status nvfp4_set_gemm_path(int32_t path);
 
 /* Time limit of every bounded in-kernel wait, in nanoseconds (default 2e9;

@@ -42,6 +42,9 @@ struct DeviceInfo {
   bool supported = false;
   int sms = 0;
   bool attr_tc = false;
+  bool attr_tc2 = false;
+  int quant_blocks = 0;   // resident k_quantize blocks per SM
+  int pairs = 0;          // co-resident clusters of two CTAs of k_gemm_tc<2>
   bool attr_small[3] = {false, false, false};
 };
 DeviceInfo g_dev[MAX_DEVICES];
@@ -217,7 +220,7 @@ int grid_for(int64_t work_items, int64_t per_block, int cap) {
 
 nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t K, int64_t ld, int64_t row0,
                              float gs, void* codes, void* scales, int64_t pad_from,
-                             int64_t pad_to, int sms, cudaStream_t st) {
+                             int64_t pad_to, DeviceInfo* info, cudaStream_t st) {
   nvfp4::QuantArgs a;
   a.x = static_cast<const __nv_bfloat16*>(x);
   a.rows = rows;
@@ -238,11 +241,25 @@ nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t K, int64_t ld,
     volatile float p = sdec * gs;   // volatile: keep the two fp32 roundings separate
     a.rtab[code] = (sdec == 0.0f || code == 127) ? 0.0f : 1.0f / p;
   }
-  const int64_t units = rows * ((K + 512 * nvfp4::QUANT_CHUNKS - 1) / (512 * nvfp4::QUANT_CHUNKS));
-  if (units >= (1ll << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  const int warps_per_block = nvfp4::QUANT_THREADS / 32;
-  const int grid = grid_for(units, warps_per_block, sms * 8);
-  nvfp4::k_quantize<<<grid, nvfp4::QUANT_THREADS, 0, st>>>(a);
+  a.wait_ns = g_wait_ns;
+  const int64_t units = rows * ((K + nvfp4::QUANT_UNIT - 1) / nvfp4::QUANT_UNIT);
+  if (units == 0 && pad_to <= pad_from) return NVFP4_OK;
+  constexpr int smem = nvfp4::QUANT_SMEM + nvfp4::QUANT_BAR_BYTES;
+  if (info->quant_blocks == 0) {
+    int blocks = 0;
+    if (cudaFuncSetAttribute(nvfp4::k_quantize, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, nvfp4::k_quantize,
+                                                      nvfp4::QUANT_THREADS, smem) != cudaSuccess ||
+        blocks < 1) {
+      cudaGetLastError();
+      return NVFP4_ERR_CUDA;
+    }
+    info->quant_blocks = blocks;
+  }
+  // persistent: one wave of resident blocks, each warp striding over the units
+  const int grid = grid_for(units, nvfp4::QUANT_WARPS, info->sms * info->quant_blocks);
+  nvfp4::k_quantize<<<grid, nvfp4::QUANT_THREADS, smem, st>>>(a);
   return check_launch();
 }
 
@@ -344,7 +361,7 @@ const char* nvfp4_status_string(nvfp4_status s) {
 }
 
 nvfp4_status nvfp4_set_gemm_path(int32_t path) {
-  if (path < 0 || path > 2) return NVFP4_ERR_INVALID_ARG;
+  if (path < 0 || path > 3) return NVFP4_ERR_INVALID_ARG;
   g_gemm_path = path;
   return NVFP4_OK;
 }
@@ -393,7 +410,7 @@ nvfp4_status nvfp4_quantize_act(const void* x, int64_t M, int64_t K, int64_t ldx
   int dev;
   DeviceInfo* info;
   if ((st = current_device(&dev, &info)) != NVFP4_OK) return st;
-  return launch_quantize(x, M, K, ldx, 0, a_gs, codes, scales, M, pad128(M), info->sms,
+  return launch_quantize(x, M, K, ldx, 0, a_gs, codes, scales, M, pad128(M), info,
                          reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -446,7 +463,7 @@ nvfp4_status nvfp4_quantize_weight(const void* w, int64_t N, int64_t K, int64_t 
     w_gs_out[s] = gs;
     const bool last = (s == nseg - 1);
     st = launch_quantize(wb + off[s] * ldw * 2, off[s + 1] - off[s], K, ldw, off[s], gs, codes,
-                         scales, last ? N : 0, last ? pad128(N) : 0, info->sms, cs);
+                         scales, last ? N : 0, last ? pad128(N) : 0, info, cs);
     if (st != NVFP4_OK) return st;
   }
   return NVFP4_OK;
@@ -531,22 +548,62 @@ nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales, const
     return launch(nvfp4::k_gemm_small<64>, nvfp4::sm::Cfg<64>::SMEM_BYTES);
   }
 
+  const bool pair = (g_gemm_path == 3) || (g_gemm_path == 0 && M > 128);
   CUtensorMap ta, tb, tsa, tsb;
   if ((st = code_map(a_codes, M, K / 2, nvfp4::tc::BM, dev, &ta)) != NVFP4_OK) return st;
-  if ((st = code_map(w_codes, N, K / 2, nvfp4::tc::BN, dev, &tb)) != NVFP4_OK) return st;
+  if ((st = code_map(w_codes, N, K / 2, nvfp4::tc::BN / (pair ? 2 : 1), dev, &tb)) != NVFP4_OK)
+    return st;
   if ((st = scale_map(a_scales, M, K, 1, dev, &tsa)) != NVFP4_OK) return st;
   if ((st = scale_map(w_scales, N, K, 2, dev, &tsb)) != NVFP4_OK) return st;
-  if (!info->attr_tc) {
-    if (cudaFuncSetAttribute(nvfp4::k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             nvfp4::tc::SMEM_BYTES) != cudaSuccess)
-      return NVFP4_ERR_CUDA;
-    info->attr_tc = true;
+  const int64_t num_n = (N + nvfp4::tc::BN - 1) / nvfp4::tc::BN;
+  if (!pair) {
+    constexpr int smem = nvfp4::tc::Cfg<1>::SMEM_BYTES;
+    if (!info->attr_tc) {
+      if (cudaFuncSetAttribute(nvfp4::k_gemm_tc<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               smem) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+      info->attr_tc = true;
+    }
+    const int64_t tiles = ((M + nvfp4::tc::BM - 1) / nvfp4::tc::BM) * num_n;
+    const int grid = static_cast<int>(tiles < info->sms ? tiles : info->sms);
+    nvfp4::k_gemm_tc<1><<<grid, nvfp4::tc::THREADS, smem, cs>>>(ta, tb, tsa, tsb, g, table);
+    return check_launch();
   }
-  const int64_t tiles = ((M + nvfp4::tc::BM - 1) / nvfp4::tc::BM) *
-                        ((N + nvfp4::tc::BN - 1) / nvfp4::tc::BN);
-  const int grid = static_cast<int>(tiles < info->sms ? tiles : info->sms);
-  nvfp4::k_gemm_tc<<<grid, nvfp4::tc::THREADS, nvfp4::tc::SMEM_BYTES, cs>>>(ta, tb, tsa, tsb, g,
-                                                                            table);
+  constexpr int smem = nvfp4::tc::Cfg<2>::SMEM_BYTES;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(nvfp4::tc::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = cs;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (!info->attr_tc2) {
+    if (cudaFuncSetAttribute(nvfp4::k_gemm_tc<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return NVFP4_ERR_CUDA;
+    // how many pairs fit at once (clusters are placed within one GPC, so an
+    // SM count that is odd inside a GPC leaves an SM out)
+    cfg.gridDim = dim3(2 * (info->sms / 2), 1, 1);
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, nvfp4::k_gemm_tc<2>, &cfg) != cudaSuccess ||
+        clusters < 1) {
+      cudaGetLastError();
+      return NVFP4_ERR_CUDA;
+    }
+    info->pairs = clusters;
+    info->attr_tc2 = true;
+  }
+  const int64_t tiles = ((M + 2 * nvfp4::tc::BM - 1) / (2 * nvfp4::tc::BM)) * num_n;
+  const int pairs = static_cast<int>(tiles < info->pairs ? tiles : info->pairs);
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  if (cudaLaunchKernelEx(&cfg, nvfp4::k_gemm_tc<2>, ta, tb, tsa, tsb, g, table) != cudaSuccess) {
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+  }
   return check_launch();
 }
 

@@ -8,24 +8,27 @@
 // gates (wiki, mechanism study part 2) in the epilogue.
 //
 // Two kernels:
-//   k_gemm_tc     persistent, warp-specialised, one 128 x 256 output tile at
-//                 a time per CTA (1 CTA per SM).  Two producer warps stream
-//                 the activation and weight codes with TMA (128-byte swizzle)
-//                 and their scale atoms with bulk copies into a 4-stage
-//                 shared-memory ring; a copier warp moves each stage's scale
-//                 atoms into a per-stage TMEM region (tcgen05.cp) while the
-//                 MMA warp issues tcgen05.mma.kind::mxf4nvf4 (K = 64 per
-//                 instruction) on the previous stage into a 128 x 256 fp32
-//                 TMEM accumulator; eight epilogue warps drain the
-//                 accumulator (each lane = one row, 128 columns), release it
-//                 to the MMA warp, then apply alpha / op and store.
+//   k_gemm_tc<CG> persistent, warp-specialised; one CTA per SM.  CG = 1: a
+//                 CTA computes one 128 x 256 output tile at a time; CG = 2: a
+//                 cluster of two CTAs computes one 256 x 256 tile with
+//                 cta_group::2 MMAs (each CTA loads half of the weight rows).
+//                 Producer warps stream the activation and weight codes and
+//                 their scale atoms with TMA (128-byte swizzle for the codes)
+//                 into a shared-memory ring; four scale-writer warps store
+//                 each stage's scale bytes into a per-stage TMEM region
+//                 (tcgen05.st) while the MMA warp issues
+//                 tcgen05.mma.kind::mxf4nvf4 (K = 64 per instruction) into a
+//                 128 x 256 fp32 TMEM accumulator per CTA; eight epilogue
+//                 warps drain the accumulator (each lane = one row, 128
+//                 columns), release it to the MMA warp, then apply alpha / op
+//                 and store.
 //   k_gemm_small  M <= 64 (decode shapes): operands swapped so the weight
 //                 rows fill the 128-row MMA side and the tokens are the MMA N
 //                 dimension (16/32/64); one CTA per 128 weight rows streams
 //                 the whole K range through a 6-stage ring.
 // Every wait is bounded (mbar_wait); a wait that runs out records the
-// device error word, raises a CTA-wide abort flag and the kernel returns
-// after draining its own copies and MMAs and freeing TMEM.
+// device error word, raises the abort flag (of both CTAs of a pair) and the
+// kernel returns after draining its own copies and MMAs and freeing TMEM.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -95,7 +98,7 @@ __device__ __forceinline__ int seg_advance(const SegTable& t, int seg, int n) {
 //        (tcgen05.mma only) and TMEM owner; warp 2 producer B: TMA of the
 //        weight codes; warp 3 producer S: TMA of both operands' scale atoms
 //        on a barrier of their own, so the scale writers need not wait for
-//        the 48 KB of codes.
+//        the codes.
 //   WG1  warps 4-7 scale writers: warp w reads, from the stage in shared
 //        memory, the scale bytes TMEM lane quarter w % 4 needs and writes
 //        them with tcgen05.st into that stage's TMEM scale region.  A
@@ -107,17 +110,21 @@ __device__ __forceinline__ int seg_advance(const SegTable& t, int seg, int n) {
 // TMEM: accumulator columns [0, 256); stage s scale region [256 + 48 s, +48):
 // 16 columns of activation scales (MMA kk reads column 4 kk + quarter) then
 // 32 of weight scales (MMA kk reads columns 8 kk + n / 32).
+//
+// CG = 1: one CTA computes a 128 x 256 tile.
+// CG = 2: a cluster of two CTAs computes a 256 x 256 tile with cta_group::2
+// MMAs issued by the even CTA: each CTA loads its own 128 activation rows,
+// half of the tile's 256 weight rows and all 256 weight rows' scales.  Per
+// k-tile a CTA then brings in 38 KB instead of 54 KB for the same number of
+// tensor-core cycles; the L2 -> shared-memory stream, not the tensor pipe,
+// is what bounds the one-CTA tile.  The odd CTA's scale writers and
+// epilogue warps arrive on the even CTA's barriers through the cluster's
+// shared window; the MMA commits arrive on both CTAs' barriers.
 namespace tc {
-constexpr int BM = 128;
-constexpr int BN = 256;
+constexpr int BM = 128;                 // rows of A per CTA
+constexpr int BN = 256;                 // tile columns (MMA N)
 constexpr int BK = 256;                 // fp4 elements per stage (128 bytes per row)
 constexpr int BKB = BK / 2;
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BKB;       // 16 KB
-constexpr int B_BYTES = BN * BKB;       // 32 KB
-constexpr int SFA_BYTES = 4 * 512;      // 4 atoms (K = 64 each) x 128 rows
-constexpr int SFB_BYTES = 2 * 4 * 512;  // 2 row blocks of 128
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 54 KB
 constexpr int SFW_WARP0 = 4;            // scale writers: warps 4-7
 constexpr int EPI_WARP0 = 8;            // epilogue: warps 8-15
 constexpr int EPI_WARPS = 8;
@@ -130,19 +137,40 @@ constexpr uint32_t ACC_COL = 0;
 constexpr uint32_t SF_COL = 256;        // + 48 * stage
 constexpr uint32_t SF_STRIDE = 48;
 constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
-static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
-static_assert(SF_COL + STAGES * SF_STRIDE <= TMEM_COLS, "TMEM budget");
+
+template <int CG>
+struct Cfg {
+  static constexpr int B_ROWS = BN / CG;                   // weight rows loaded per CTA
+  static constexpr int A_BYTES = BM * BKB;                 // 16 KB
+  static constexpr int B_BYTES = B_ROWS * BKB;             // 32 / 16 KB
+  static constexpr int SFA_BYTES = 4 * 512;                // 4 atoms (K = 64 each) x 128 rows
+  static constexpr int SFB_BYTES = 2 * 4 * 512;            // both row blocks of the tile
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 54 / 38 KB
+  static constexpr int STAGES = CG == 1 ? 4 : 5;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+  static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
+  static_assert(SF_COL + STAGES * SF_STRIDE <= TMEM_COLS, "TMEM budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
 }  // namespace tc
 
-// tmA / tmB: code matrices [rows, K/2] (box 128 bytes x 128 / 256 rows, 128-byte
-// swizzle).  tmSA / tmSB: scale buffers viewed as [row blocks][K/64 atoms][64
-// u64] (box 64 x 4 x 1 / 2, i.e. one stage's atoms of 1 / 2 row blocks).
+// tmA / tmB: code matrices [rows, K/2] (box 128 bytes x 128 / (256 / CG)
+// rows, 128-byte swizzle).  tmSA / tmSB: scale buffers viewed as [row blocks]
+// [K/64 atoms][64 u64] (box 64 x 4 x 1 / 2, i.e. one stage's atoms of 1 / 2
+// row blocks).  CG = 2 must be launched with clusters of 2 CTAs.
+template <int CG>
 __global__ void __launch_bounds__(tc::THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
               const GemmArgs g, const __grid_constant__ SegTable seg) {
   using namespace tc;
+  using C = Cfg<CG>;
+  constexpr int STAGES = C::STAGES;
+  constexpr int STAGE_BYTES = C::STAGE_BYTES;
+  constexpr int A_BYTES = C::A_BYTES;
+  constexpr int B_BYTES = C::B_BYTES;
+  constexpr int SFA_BYTES = C::SFA_BYTES;
+  constexpr int SFB_BYTES = C::SFB_BYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -153,7 +181,10 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int num_m = (g.M + BM - 1) / BM;
+  const uint32_t rank = CG == 1 ? 0u : cluster_ctarank();
+  const int unit = static_cast<int>(blockIdx.x) / CG;     // CTA (pair) index
+  const int units = static_cast<int>(gridDim.x) / CG;
+  const int num_m = (g.M + BM * CG - 1) / (BM * CG);
   const int num_n = (g.N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
   const int num_kt = (g.K + BK - 1) / BK;
@@ -166,15 +197,34 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
   const uint32_t tmem_empty = smem_addr(bars + 4 * STAGES + 1);
   const uint32_t drain_mma = smem_addr(bars + 4 * STAGES + 2);
 
+  // Barriers that the MMA issuer waits on live in the even CTA; the odd CTA
+  // arrives on them through the cluster window.
+  auto arrive_leader = [&](uint32_t bar) {
+    if constexpr (CG == 1)
+      mbar_arrive(bar);
+    else
+      mbar_arrive_remote(mapa_shared(bar, 0));
+  };
+  auto wait_pair = [&](uint32_t bar, uint32_t parity) {
+    return mbar_wait(bar, parity, g.wait_ns, abort_flag);
+  };
+  // A role that gives up raises the abort flag of both CTAs of the pair.
+  auto raise_abort = [&](uint32_t site, uint32_t role) {
+    if (!*abort_flag) record_error(site, role);
+    *abort_flag = 1;
+    if constexpr (CG == 2)
+      st_shared_remote_u32(mapa_shared(smem_addr(const_cast<int*>(abort_flag)), rank ^ 1u), 1u);
+  };
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 2);            // both producers arrive (with their bytes)
       mbar_init(empty_bar(s), 1);
-      mbar_init(sf_bar(s), 4);              // the four scale writers
+      mbar_init(sf_bar(s), 4 * CG);         // the scale writers of every CTA of the pair
       mbar_init(sfull_bar(s), 1);           // the scale producer
     }
     mbar_init(tmem_full, 1);
-    mbar_init(tmem_empty, EPI_WARPS);
+    mbar_init(tmem_empty, EPI_WARPS * CG);
     mbar_init(drain_mma, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -184,11 +234,14 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     prefetch_tensormap(&tmSB);
   }
   if (warp == 1) {
-    tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_cg<CG>(smem_addr(tmem_slot), TMEM_COLS);
+    tmem_relinquish_cg<CG>();
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 1)
+    __syncthreads();
+  else
+    cluster_sync();   // the other CTA's barriers are initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -202,28 +255,29 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       uint32_t phase = 0;
       int64_t issued = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int tile = unit; tile < num_tiles && ok; tile += units) {
         const int mb = tile % num_m;
         const int nb = tile / num_m;
+        const int arow = (mb * CG + static_cast<int>(rank)) * BM;
+        const int brow = nb * BN + static_cast<int>(rank) * C::B_ROWS;
         for (int kt = 0; kt < num_kt; ++kt) {
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, g.wait_ns, abort_flag)) {
-            if (!*abort_flag) record_error(SITE_PRODUCER_EMPTY, warp);
-            *abort_flag = 1;
+          if (!wait_pair(empty_bar(stage), phase ^ 1u)) {
+            raise_abort(SITE_PRODUCER_EMPTY, warp);
             ok = false;
             break;
           }
           uint8_t* st = smem + stage * STAGE_BYTES;
           if (warp == 0) {
             mbar_arrive_expect_tx(full_bar(stage), A_BYTES);
-            tma_load_2d(smem_addr(st), &tmA, kt * BKB, mb * BM, full_bar(stage), pol);
+            tma_load_2d(smem_addr(st), &tmA, kt * BKB, arow, full_bar(stage), pol);
           } else if (warp == 2) {
             mbar_arrive_expect_tx(full_bar(stage), B_BYTES);
-            tma_load_2d(smem_addr(st + A_BYTES), &tmB, kt * BKB, nb * BN, full_bar(stage), pol);
+            tma_load_2d(smem_addr(st + A_BYTES), &tmB, kt * BKB, brow, full_bar(stage), pol);
           } else {
             // both boxes always transfer their full size (out-of-range atoms read as 0)
             mbar_arrive_expect_tx(sfull_bar(stage), SFA_BYTES + SFB_BYTES);
-            tma_load_3d(smem_addr(st + A_BYTES + B_BYTES), &tmSA, 0, kt * 4, mb, sfull_bar(stage),
-                        pol);
+            tma_load_3d(smem_addr(st + A_BYTES + B_BYTES), &tmSA, 0, kt * 4,
+                        mb * CG + static_cast<int>(rank), sfull_bar(stage), pol);
             tma_load_3d(smem_addr(st + A_BYTES + B_BYTES + SFA_BYTES), &tmSB, 0, kt * 4, nb * 2,
                         sfull_bar(stage), pol);
           }
@@ -251,12 +305,11 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     int stage = 0;
     uint32_t phase = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    for (int tile = unit; tile < num_tiles; tile += units) {
       bool ok = true;
       for (int kt = 0; kt < num_kt; ++kt) {
         if (!mbar_wait(sfull_bar(stage), phase, g.wait_ns, abort_flag)) {
-          if (!*abort_flag) record_error(SITE_MMA_FULL, warp);
-          *abort_flag = 1;
+          raise_abort(SITE_MMA_FULL, warp);
           ok = false;
           break;
         }
@@ -289,13 +342,12 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         // the MMA warp waits on this barrier alone: arrive only once the
         // stage's codes have landed too
         if (!mbar_wait(full_bar(stage), phase, g.wait_ns, abort_flag)) {
-          if (!*abort_flag) record_error(SITE_MMA_FULL, warp);
-          *abort_flag = 1;
+          raise_abort(SITE_MMA_FULL, warp);
           ok = false;
           break;
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(sf_bar(stage));
+        if (lane == 0) arrive_leader(sf_bar(stage));
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1u;
@@ -310,8 +362,8 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     // single barrier per stage (the scale writers arrive only once both the
     // codes and the scales of the stage are in place), uses precomputed
     // descriptors, and releases the previous stage right after MMA 0.
-    if (lane == 0) {
-      const uint32_t idesc = idesc_mxf4nvf4(BM, BN);
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = idesc_mxf4nvf4(BM * CG, BN);
       // the start-address field holds (address >> 4) and every stage lies below
       // 256 KB, so a stage's descriptor is the first one plus stage * STAGE_BYTES / 16
       const uint64_t adesc0 = desc_kmajor_sw128(smem_addr(smem));
@@ -320,18 +372,16 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
-        if (!mbar_wait(tmem_empty, static_cast<uint32_t>((local & 1) ^ 1), g.wait_ns, abort_flag)) {
-          if (!*abort_flag) record_error(SITE_MMA_TMEM_EMPTY, 1);
-          *abort_flag = 1;
+      for (int tile = unit; tile < num_tiles && ok; tile += units, ++local) {
+        if (!wait_pair(tmem_empty, static_cast<uint32_t>((local & 1) ^ 1))) {
+          raise_abort(SITE_MMA_TMEM_EMPTY, 1);
           break;
         }
         tc_fence_after();
         int prev = -1;
         for (int kt = 0; kt < num_kt; ++kt) {
-          if (!mbar_wait(sf_bar(stage), phase, g.wait_ns, abort_flag)) {
-            if (!*abort_flag) record_error(SITE_MMA_FULL, 1);
-            *abort_flag = 1;
+          if (!wait_pair(sf_bar(stage), phase)) {
+            raise_abort(SITE_MMA_FULL, 1);
             ok = false;
             break;
           }
@@ -341,23 +391,23 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
           const uint64_t ad = adesc0 + soff, bd = bdesc0 + soff;
           const uint32_t col = tmem_base + SF_COL + SF_STRIDE * stage;
           // K = 64 fp4 = 32 bytes per MMA: advance the start address inside the swizzle atom
-          mma_mxf4nvf4(tmem_base + ACC_COL, ad, bd, idesc, col, col + 16, kt != 0);
-          if (prev >= 0) tc_commit(empty_bar(prev));
+          mma_mxf4nvf4_cg<CG>(tmem_base + ACC_COL, ad, bd, idesc, col, col + 16, kt != 0);
+          if (prev >= 0) tc_commit_all<CG>(empty_bar(prev));
           for (int kk = 1; kk < nk; ++kk)
-            mma_mxf4nvf4(tmem_base + ACC_COL, ad + 2 * kk, bd + 2 * kk, idesc, col + 4 * kk,
-                         col + 16 + 8 * kk, 1u);
+            mma_mxf4nvf4_cg<CG>(tmem_base + ACC_COL, ad + 2 * kk, bd + 2 * kk, idesc,
+                                col + 4 * kk, col + 16 + 8 * kk, 1u);
           prev = stage;
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
-        if (prev >= 0) tc_commit(empty_bar(prev));
+        if (prev >= 0) tc_commit_all<CG>(empty_bar(prev));
         if (!ok) break;
-        tc_commit(tmem_full);
+        tc_commit_all<CG>(tmem_full);
       }
       // all issued tensor-core work must finish before TMEM is freed
-      tc_commit(drain_mma);
+      tc_commit_local<CG>(drain_mma);
       if (!mbar_wait(drain_mma, 0, g.wait_ns, nullptr)) record_error(SITE_DRAIN, 1);
     }
     __syncwarp();
@@ -368,12 +418,11 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     const int half = (warp - EPI_WARP0) >> 2;     // columns [128*half, 128*half + 128)
     const int row_in_tile = q * 32 + lane;
     int local = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+    for (int tile = unit; tile < num_tiles; tile += units, ++local) {
       const int mb = tile % num_m;
       const int nb = tile / num_m;
-      if (!mbar_wait(tmem_full, static_cast<uint32_t>(local & 1), g.wait_ns, abort_flag)) {
-        if (!*abort_flag) record_error(SITE_EPI_TMEM_FULL, warp);
-        *abort_flag = 1;
+      if (!wait_pair(tmem_full, static_cast<uint32_t>(local & 1))) {
+        raise_abort(SITE_EPI_TMEM_FULL, warp);
         break;
       }
       tc_fence_after();
@@ -384,9 +433,9 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tmem_empty);
+      if (lane == 0) arrive_leader(tmem_empty);
 
-      const int64_t gm = static_cast<int64_t>(mb) * BM + row_in_tile;
+      const int64_t gm = static_cast<int64_t>(mb * CG + static_cast<int>(rank)) * BM + row_in_tile;
       if (gm < g.M) {
         const int n0 = nb * BN + half * 128;
         int s = seg_advance(seg, 0, n0);
@@ -435,10 +484,15 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     }
   }
 
+  // No CTA of a pair leaves (or frees TMEM) while the pair's MMAs, copies or
+  // remote arrivals may still touch it.
   tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 1)
+    __syncthreads();
+  else
+    cluster_sync();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+  if (warp == 1) tmem_dealloc_cg<CG>(tmem_base, TMEM_COLS);
 }
 
 // ========================================================== k_gemm_small

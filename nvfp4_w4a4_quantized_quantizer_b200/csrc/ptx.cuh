@@ -29,6 +29,7 @@ enum ErrorSite : uint32_t {
   SITE_MMA_TMEM_EMPTY = 3,
   SITE_EPI_TMEM_FULL = 4,
   SITE_DRAIN = 5,
+  SITE_QUANT = 6,
   SITE_TEST = 15,
 };
 
@@ -96,6 +97,44 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
     if (abort_flag != nullptr && *abort_flag) return false;
     if (globaltimer_ns() - t0 > limit_ns) return false;
   }
+}
+
+// ---------------------------------------------------------------- clusters
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address, in the cluster's shared window, of this CTA's shared address
+// `saddr` as seen in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+
+// Arrive on an mbarrier of another CTA of the cluster, named by its cluster
+// address.  Default semantics (release at CTA scope), as CUTLASS's CTA-pair
+// pipelines use them: the data behind these hand-offs (the other CTA's TMEM
+// scale columns and its TMA-written shared memory) is read only by the
+// pair's MMAs, which the tcgen05 fences order after the waiting thread's
+// wait.  Acquire / release at cluster scope on the arrive and the waits made
+// every hand-off of the CTA-pair GEMM several hundred cycles slower.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ void st_shared_remote_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.relaxed.cluster.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v)
+               : "memory");
+}
+
+// Every thread of every CTA of the cluster (like __syncthreads, cluster-wide).
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile(
+      "barrier.cluster.arrive.release.aligned;\n\t"
+      "barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 // -------------------------------------------------------- TMA / bulk copy
@@ -186,6 +225,83 @@ __device__ __forceinline__ void mma_mxf4nvf4(uint32_t d_tmem, uint64_t a_desc, u
       "p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
+}
+
+// CTA-pair forms (cta_group::2): the two CTAs of a cluster of 2 share one
+// MMA.  Allocation and release are executed by the same warp of both CTAs;
+// the MMA and the commits by one thread of the even CTA only.  Every
+// tcgen05 instruction of a kernel must use the same cta_group.
+template <int CG>
+__device__ __forceinline__ void tmem_alloc_cg(uint32_t dst_smem, uint32_t ncols) {
+  if constexpr (CG == 1)
+    tmem_alloc(dst_smem, ncols);
+  else
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     dst_smem),
+                 "r"(ncols)
+                 : "memory");
+}
+
+template <int CG>
+__device__ __forceinline__ void tmem_relinquish_cg() {
+  if constexpr (CG == 1)
+    tmem_relinquish();
+  else
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+template <int CG>
+__device__ __forceinline__ void tmem_dealloc_cg(uint32_t taddr, uint32_t ncols) {
+  if constexpr (CG == 1)
+    tmem_dealloc(taddr, ncols);
+  else
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+// Arrive once on `bar` (same shared offset) in every CTA of the pair when the
+// tcgen05 operations issued so far have completed.
+template <int CG>
+__device__ __forceinline__ void tc_commit_all(uint32_t bar) {
+  if constexpr (CG == 1)
+    tc_commit(bar);
+  else
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(bar),
+        "h"(static_cast<uint16_t>(3))
+        : "memory");
+}
+
+// Arrive once on this CTA's `bar` only.
+template <int CG>
+__device__ __forceinline__ void tc_commit_local(uint32_t bar) {
+  if constexpr (CG == 1)
+    tc_commit(bar);
+  else
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar)
+                 : "memory");
+}
+
+// With CG = 2 the MMA is M = 256: rows 0-127 come from the even CTA's shared
+// memory and TMEM, rows 128-255 from the odd CTA's at the same addresses;
+// the N rows of B are split the same way (first half even CTA); each CTA's
+// TMEM holds its own 128 accumulator rows, its own A scales and all of B's.
+template <int CG>
+__device__ __forceinline__ void mma_mxf4nvf4_cg(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t sfa_tmem,
+                                                uint32_t sfb_tmem, uint32_t accumulate) {
+  if constexpr (CG == 1)
+    mma_mxf4nvf4(d_tmem, a_desc, b_desc, idesc, sfa_tmem, sfb_tmem, accumulate);
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], "
+        "[%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
 }
 
 // Copy 32 rows x 16 bytes from shared memory to TMEM lanes 0-31 and

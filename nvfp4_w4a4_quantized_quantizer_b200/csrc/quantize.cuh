@@ -12,15 +12,16 @@
 // Every rounding is an explicit _rn intrinsic or a .rn conversion, so the
 // compiler cannot contract or reorder it.
 //
-// Work mapping: a warp work unit is (row, 1024-element segment); lane t owns
-// one whole 16-element block per 512-element chunk (one 32-byte load; the
-// warp reads 1 KB contiguous), writes its 8 code bytes (the warp writes 256
-// contiguous bytes), and every 4th lane gathers the scale bytes of blocks
-// j..j+3 (contiguous in the atom layout) into one 32-bit store.  The block
-// reciprocal r depends only on the scale code, so the launch carries the
-// 128-entry table r[s] = fp32(1 / fp32(s_dec * gs)) (0 for s = 0), computed
-// on the host with IEEE fp32 arithmetic — the same rounding as the device
-// reciprocal — instead of a decode, a multiply and a reciprocal per block.
+// Work mapping: a warp work unit is (row, 1024-element segment), streamed
+// into shared memory by a bulk copy (see "Staging" below); lane t owns one
+// whole 16-element block per 512 elements, writes its 8 code bytes (the
+// warp writes 256 contiguous bytes), and every 4th lane gathers the scale
+// bytes of blocks j..j+3 (contiguous in the atom layout) into one 32-bit
+// store.  The block reciprocal r depends only on the scale code, so the
+// launch carries the 128-entry table r[s] = fp32(1 / fp32(s_dec * gs)) (0 for
+// s = 0), computed on the host with IEEE fp32 arithmetic — the same rounding
+// as the device reciprocal — instead of a decode, a multiply and a
+// reciprocal per block.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -80,6 +81,7 @@ struct QuantArgs {
   uint8_t* scales;         // base of the full scale buffer (atom layout)
   int64_t pad_from;        // zero scale rows [pad_from, pad_to)
   int64_t pad_to;
+  uint64_t wait_ns;        // bound on each wait for a staged copy
   float rtab[128];         // fp32(1 / fp32(e4m3(s) * gs)), 0 for s == 0
 };
 
@@ -100,15 +102,18 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
   }
 }
 
+// Staging: every warp owns a ring of QUANT_SLOTS shared-memory slots and
+// streams its work units into them with cp.async.bulk (one contiguous copy
+// of a row segment per unit, completion counted on the slot's mbarrier), so
+// each SM keeps ~QUANT_SLOTS x 2 KB x (resident warps) bytes of HBM reads in
+// flight independent of registers; the warp then quantises the unit out of
+// shared memory and refills the slot with its unit QUANT_SLOTS ahead.
 constexpr int QUANT_THREADS = 256;
-constexpr int QUANT_CHUNKS = 2;            // 512-element chunks per warp work unit
-
-__device__ __forceinline__ void ld_stream_v8(const void* p, uint32_t (&w)[8]) {
-  asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]),
-                 "=r"(w[6]), "=r"(w[7])
-               : "l"(p));
-}
+constexpr int QUANT_WARPS = QUANT_THREADS / 32;
+constexpr int QUANT_UNIT = 1024;                 // elements per work unit (2 KB of bf16)
+constexpr int QUANT_SLOTS = 4;
+constexpr int QUANT_SMEM = QUANT_WARPS * QUANT_SLOTS * QUANT_UNIT * 2;   // 64 KB
+constexpr int QUANT_BAR_BYTES = QUANT_WARPS * QUANT_SLOTS * 8;
 
 // |x| max of sixteen bf16 values (eight packed words), exact: the magnitude
 // bits of non-negative bf16 values order like unsigned integers.
@@ -124,64 +129,125 @@ __device__ __forceinline__ float bf16x16_absmax(const uint32_t (&w)[8]) {
   return __uint_as_float((hi > lo ? hi : lo) << 16);
 }
 
-// A warp work unit is (row, 1024-element segment); the host guarantees
-// rows * segments < 2^31 so the unit index stays 32-bit.
+// Elements of work unit u: row u / per_row, columns [c * QUANT_UNIT, +n).
+struct QuantUnit {
+  int64_t row;
+  int col;
+  int n;
+};
+
+__device__ __forceinline__ QuantUnit quant_unit(int64_t u, int per_row, int K) {
+  QuantUnit q;
+  q.row = u / per_row;
+  q.col = static_cast<int>(u - q.row * per_row) * QUANT_UNIT;
+  q.n = min(QUANT_UNIT, K - q.col);
+  return q;
+}
+
 __global__ void __launch_bounds__(QUANT_THREADS) k_quantize(const __grid_constant__ QuantArgs a) {
+  extern __shared__ __align__(128) uint8_t qsmem[];
+  const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const uint32_t gwarp = (blockIdx.x * QUANT_THREADS + threadIdx.x) >> 5;
-  const uint32_t nwarps = (gridDim.x * QUANT_THREADS) >> 5;
-  const uint32_t segs = static_cast<uint32_t>((a.K + 512 * QUANT_CHUNKS - 1) / (512 * QUANT_CHUNKS));
-  const uint32_t units = static_cast<uint32_t>(a.rows) * segs;
+  uint8_t* ring = qsmem + warp * (QUANT_SLOTS * QUANT_UNIT * 2);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(qsmem + QUANT_SMEM) + warp * QUANT_SLOTS;
+  const int K = static_cast<int>(a.K);
+  const int per_row = (K + QUANT_UNIT - 1) / QUANT_UNIT;
+  const int64_t units = a.rows * per_row;
+  const int64_t gwarp = static_cast<int64_t>(blockIdx.x) * QUANT_WARPS + warp;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * QUANT_WARPS;
   const float c = __fmul_rn(6.0f, a.gs);
   const int64_t code_ld = a.K / 2;
-  const int K = static_cast<int>(a.K);
+  const uint64_t pol = policy_evict_first();
 
-  for (uint32_t u = gwarp; u < units; u += nwarps) {
-    const uint32_t r = u / segs;
-    const int k0 = static_cast<int>(u - r * segs) * (512 * QUANT_CHUNKS) + lane * 16;
-    const __nv_bfloat16* src = a.x + static_cast<int64_t>(r) * a.ldx;
-    uint32_t w[QUANT_CHUNKS][8];
-#pragma unroll
-    for (int i = 0; i < QUANT_CHUNKS; ++i) {
-      const int k = k0 + i * 512;
-      if (k < K) {
-        ld_stream_v8(src + k, w[i]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) w[i][e] = 0u;
-      }
+  if (lane == 0) {
+    for (int s = 0; s < QUANT_SLOTS; ++s) mbar_init(smem_addr(bars + s), 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  // lane 0 starts the copy of the warp's i-th unit into slot i % QUANT_SLOTS
+  auto issue = [&](int64_t i) {
+    const int64_t u = gwarp + i * nwarps;
+    if (u >= units) return;
+    const QuantUnit q = quant_unit(u, per_row, K);
+    const int s = static_cast<int>(i % QUANT_SLOTS);
+    const uint32_t bytes = static_cast<uint32_t>(q.n) * 2u;
+    mbar_arrive_expect_tx(smem_addr(bars + s), bytes);
+    bulk_load(smem_addr(ring + s * (QUANT_UNIT * 2)), a.x + q.row * a.ldx + q.col, bytes,
+              smem_addr(bars + s), pol);
+  };
+  if (lane == 0)
+    for (int i = 0; i < QUANT_SLOTS; ++i) issue(i);
+
+  int64_t i = 0;
+  bool ok = true;
+  for (int64_t u = gwarp; u < units; u += nwarps, ++i) {
+    const int s = static_cast<int>(i % QUANT_SLOTS);
+    if (!mbar_wait(smem_addr(bars + s), static_cast<uint32_t>((i / QUANT_SLOTS) & 1), a.wait_ns,
+                   nullptr)) {
+      if (lane == 0) record_error(SITE_QUANT, static_cast<uint32_t>(warp));
+      ok = false;
+      break;
     }
-    const int64_t grow = a.row0 + r;
+    const QuantUnit q = quant_unit(u, per_row, K);
+    const int64_t grow = a.row0 + q.row;
+    const uint32_t slot = smem_addr(ring + s * (QUANT_UNIT * 2));
 #pragma unroll
-    for (int i = 0; i < QUANT_CHUNKS; ++i) {
-      if (k0 - lane * 16 + i * 512 >= K) break;            // warp-uniform: chunk past the row end
-      const int k = k0 + i * 512;
-      const float amax = bf16x16_absmax(w[i]);
-      const uint32_t s = cvt_e4m3(__fdiv_rn(amax, c));
-      const float rr = a.rtab[s];
+    for (int p = 0; p < QUANT_UNIT / 512; ++p) {
+      const int e0 = p * 512;
+      if (e0 >= q.n) break;                               // warp-uniform
+      const int e = e0 + lane * 16;                       // this lane's block
+      const bool live = e < q.n;                          // uniform per 4 lanes (n % 64 == 0)
+      uint32_t w[8];
+      // lanes 4..7 of each group of 8 read their halves in the other order,
+      // so a quarter-warp's 16-byte reads cover all 32 banks once
+      const uint32_t h = static_cast<uint32_t>((lane >> 2) & 1) * 16u;
+      const uint4 v0 = ld_shared_v4(slot + e * 2 + h);
+      const uint4 v1 = ld_shared_v4(slot + e * 2 + (h ^ 16u));
+      const uint4 lo = h ? v1 : v0, hi = h ? v0 : v1;
+      w[0] = lo.x; w[1] = lo.y; w[2] = lo.z; w[3] = lo.w;
+      w[4] = hi.x; w[5] = hi.y; w[6] = hi.z; w[7] = hi.w;
+      const float amax = bf16x16_absmax(w);
+      const uint32_t sc = cvt_e4m3(__fdiv_rn(amax, c));
+      const float rr = a.rtab[sc];
       float f[8];
-      uint32_t q[2];
+      uint32_t qv[2];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      for (int hh = 0; hh < 2; ++hh) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          f[2 * e] = __fmul_rn(__uint_as_float(w[i][4 * h + e] << 16), rr);
-          f[2 * e + 1] = __fmul_rn(__uint_as_float(w[i][4 * h + e] & 0xFFFF0000u), rr);
+        for (int k = 0; k < 4; ++k) {
+          f[2 * k] = __fmul_rn(__uint_as_float(w[4 * hh + k] << 16), rr);
+          f[2 * k + 1] = __fmul_rn(__uint_as_float(w[4 * hh + k] & 0xFFFF0000u), rr);
         }
-        q[h] = cvt_e2m1x8(f);
+        qv[hh] = cvt_e2m1x8(f);
       }
-      if (s == 0) q[0] = q[1] = 0u;
+      if (sc == 0) qv[0] = qv[1] = 0u;
       // scale bytes of blocks 4g..4g+3 (lanes 4g..4g+3) -> lane 4g
-      const uint32_t s1 = __shfl_down_sync(0xffffffffu, s, 1);
-      const uint32_t s2 = __shfl_down_sync(0xffffffffu, s, 2);
-      const uint32_t s3 = __shfl_down_sync(0xffffffffu, s, 3);
-      if (k < K) {
-        *reinterpret_cast<uint2*>(a.codes + grow * code_ld + k / 2) = make_uint2(q[0], q[1]);
+      const uint32_t s1 = __shfl_down_sync(0xffffffffu, sc, 1);
+      const uint32_t s2 = __shfl_down_sync(0xffffffffu, sc, 2);
+      const uint32_t s3 = __shfl_down_sync(0xffffffffu, sc, 3);
+      if (live) {
+        const int k = q.col + e;
+        *reinterpret_cast<uint2*>(a.codes + grow * code_ld + k / 2) = make_uint2(qv[0], qv[1]);
         if ((lane & 3) == 0) {
-          const uint32_t word = s | (s1 << 8) | (s2 << 16) | (s3 << 24);
+          const uint32_t word = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
           *reinterpret_cast<uint32_t*>(a.scales + sf_offset(grow, k / 16, a.K)) = word;
         }
       }
+    }
+    // every lane's reads of the slot are done (their results are stored);
+    // order them before the bulk copy that refills it
+    __syncwarp();
+    if (lane == 0) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      issue(i + QUANT_SLOTS);
+    }
+  }
+  // copies still in flight (only after a failed wait) must land before exit
+  if (!ok && lane == 0) {
+    for (int64_t j = i; j < i + QUANT_SLOTS; ++j) {
+      if (gwarp + j * nwarps >= units) break;
+      mbar_wait(smem_addr(bars + (j % QUANT_SLOTS)), static_cast<uint32_t>((j / QUANT_SLOTS) & 1),
+                a.wait_ns, nullptr);
     }
   }
 

@@ -1,4 +1,4 @@
-"""GPU parity: block-scaled FP4 GEMM (both kernels) vs the float64 oracle.
+"""GPU parity: block-scaled FP4 GEMM (every kernel) vs the float64 oracle.
 
 Operands are either built directly in the device layout from random codes
 and scales (so the GEMM is checked independently of the quantiser) or come
@@ -17,7 +17,7 @@ from tests import _helpers as H
 
 pytestmark = pytest.mark.gpu
 
-LARGE, SMALL, AUTO = 1, 2, 0
+LARGE, SMALL, AUTO, PAIR = 1, 2, 0, 3
 
 
 @pytest.fixture(autouse=True)
@@ -57,7 +57,7 @@ def run(path, ac, as_, a_gs, wc, ws, w_gs, M, N, K):
     return y32.cpu().numpy(), yb.float().cpu().numpy()
 
 
-@pytest.mark.parametrize("path,M", [(LARGE, 16), (SMALL, 16)])
+@pytest.mark.parametrize("path,M", [(LARGE, 16), (SMALL, 16), (PAIR, 16)])
 @pytest.mark.parametrize("p", [0, 1, 14, 15, 16, 31, 63, 64, 127, 128, 200, 255])
 def test_all_code_pairs_single_k(path, M, p):
     """Row m holds code m, column n holds code n, both at k = p only; random scales."""
@@ -82,7 +82,11 @@ def test_all_code_pairs_single_k(path, M, p):
     (LARGE, 128, 256, 256), (LARGE, 256, 512, 512), (LARGE, 200, 272, 320),
     (LARGE, 129, 16, 64), (LARGE, 2048, 2560, 256), (LARGE, 300, 608, 1280),
     (SMALL, 1, 16, 64), (SMALL, 7, 128, 320), (SMALL, 16, 400, 1024), (SMALL, 17, 144, 256),
-    (SMALL, 33, 272, 512), (SMALL, 64, 1040, 768)])
+    (SMALL, 33, 272, 512), (SMALL, 64, 1040, 768),
+    # CTA pairs: odd CTA's rows all past M (M <= 128), a ragged last tile
+    # whose odd-CTA weight rows lie past N, several tiles per pair
+    (PAIR, 100, 272, 320), (PAIR, 256, 256, 256), (PAIR, 300, 608, 1280),
+    (PAIR, 129, 16, 64), (PAIR, 2048, 2560, 256), (PAIR, 2304, 5120, 512)])
 def test_random_codes_and_scales(path, M, N, K):
     rng = np.random.default_rng(M * 131 + N * 7 + K)
     ac = rng.integers(0, 16, size=(M, K)).astype(np.uint8)
@@ -108,7 +112,7 @@ def test_cancellation_heavy_accumulation():
     wc[:, 64::128] = 15
     as_ = rng.integers(0x08, 0x7F, size=(M, K // 16)).astype(np.uint8)
     ws = rng.integers(0x08, 0x7F, size=(N, K // 16)).astype(np.uint8)
-    for path in (LARGE,):
+    for path in (LARGE, PAIR):
         y32, yb = run(path, *dev_operands(ac, as_, M, K), 1e-3, *dev_operands(wc, ws, N, K), 2e-3,
                       M, N, K)
         ref = oracle.linear64(oracle.dequantize(ac, as_, np.float32(1e-3)),
@@ -117,6 +121,7 @@ def test_cancellation_heavy_accumulation():
 
 
 @pytest.mark.parametrize("path,M,N,K", [(LARGE, 200, 272, 320), (LARGE, 512, 768, 1024),
+                                        (PAIR, 200, 272, 320), (PAIR, 512, 768, 1024),
                                         (SMALL, 5, 144, 320), (SMALL, 64, 256, 5120),
                                         (AUTO, 64, 128, 256)])
 def test_quantize_then_gemm(path, M, N, K):
@@ -156,7 +161,7 @@ def test_tiny_workload_end_to_end():
 
 
 def test_output_row_stride_and_no_overwrite():
-    """ldy > N: columns past N are never written (large and small kernels)."""
+    """ldy > N: columns past N are never written (every kernel)."""
     M, N, K, ldy = 150, 144, 256, 160
     rng = np.random.default_rng(9)
     ac = rng.integers(0, 16, size=(M, K)).astype(np.uint8)
@@ -166,7 +171,7 @@ def test_output_row_stride_and_no_overwrite():
     A, W = dev_operands(ac, as_, M, K), dev_operands(wc, ws, N, K)
     ref = oracle.linear64(oracle.dequantize(ac, as_, np.float32(0.01)),
                           oracle.dequantize(wc, ws, np.float32(0.02)))
-    for path, m in ((LARGE, M), (SMALL, 40)):
+    for path, m in ((LARGE, M), (PAIR, M), (SMALL, 40)):
         nv.nvfp4_set_gemm_path(path)
         y = torch.full((m, ldy), -7.0, dtype=torch.float32, device="cuda")
         nv.nvfp4_linear(A[0], A[1], 0.01, W[0], W[1], 0.02, m, N, K, y=y[:, :N],
@@ -176,8 +181,9 @@ def test_output_row_stride_and_no_overwrite():
         H.check_gemm_fp32(out[:, :N], ref[:m], f"ldy path {path}")
 
 
+@pytest.mark.parametrize("path", [LARGE, PAIR])
 @pytest.mark.parametrize("ldy", [152, 160])
-def test_bf16_row_stride_both_store_widths(ldy):
+def test_bf16_row_stride_both_store_widths(ldy, path):
     """bf16 rows of 304 bytes take 16-byte stores, rows of 320 bytes whole 32-byte sectors."""
     M, N, K = 200, 144, 256
     rng = np.random.default_rng(ldy)
@@ -186,7 +192,7 @@ def test_bf16_row_stride_both_store_widths(ldy):
     as_ = rng.integers(0x30, 0x40, size=(M, K // 16)).astype(np.uint8)
     ws = rng.integers(0x30, 0x40, size=(N, K // 16)).astype(np.uint8)
     A, W = dev_operands(ac, as_, M, K), dev_operands(wc, ws, N, K)
-    nv.nvfp4_set_gemm_path(LARGE)
+    nv.nvfp4_set_gemm_path(path)
     y32 = nv.nvfp4_linear(A[0], A[1], 0.01, W[0], W[1], 0.02, M, N, K, out_dtype=nv.OUT_FP32)
     y = torch.full((M, ldy), 3.0, dtype=torch.bfloat16, device="cuda")
     nv.nvfp4_linear(A[0], A[1], 0.01, W[0], W[1], 0.02, M, N, K, y=y[:, :N])

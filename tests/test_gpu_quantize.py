@@ -74,7 +74,10 @@ def _quant_and_check(bits, gs, ld=None):
 
 
 @pytest.mark.parametrize("M,K,ld", [(1, 64, None), (3, 192, None), (100, 320, 336),
-                                    (129, 5120, None), (300, 576, 640), (64, 256, None)])
+                                    (129, 5120, None), (300, 576, 640), (64, 256, None),
+                                    # a 64-element last segment; rows 16 (not 32) bytes apart
+                                    # mod 32; more units than every warp's staging ring holds
+                                    (70, 1088, 1096), (5, 2048, None), (3000, 5120, None)])
 def test_quantize_act_matches_oracle(M, K, ld):
     bits = workloads.random_bf16((M, K), seed=M * 7 + K, std=3.0)
     gs = oracle.global_scale(np.abs(H.f32(bits)).max())
