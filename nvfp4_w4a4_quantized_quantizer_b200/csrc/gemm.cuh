@@ -249,7 +249,8 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
   if (warp < SFW_WARP0) regs_dealloc<REGS_SMALL>();
   if (warp == 0 || warp == 2 || warp == 3) {
     // ---------------------------------------------------- TMA producers
-    if (lane == 0) {
+    // warp-wide loop; one elected lane issues each copy
+    {
       const uint64_t pol = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
@@ -268,17 +269,17 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
           }
           uint8_t* st = smem + stage * STAGE_BYTES;
           if (warp == 0) {
-            mbar_arrive_expect_tx(full_bar(stage), A_BYTES);
-            tma_load_2d(smem_addr(st), &tmA, kt * BKB, arow, full_bar(stage), pol);
+            mbar_arrive_expect_tx_warp(full_bar(stage), A_BYTES);
+            tma_load_2d_warp(smem_addr(st), &tmA, kt * BKB, arow, full_bar(stage), pol);
           } else if (warp == 2) {
-            mbar_arrive_expect_tx(full_bar(stage), B_BYTES);
-            tma_load_2d(smem_addr(st + A_BYTES), &tmB, kt * BKB, brow, full_bar(stage), pol);
+            mbar_arrive_expect_tx_warp(full_bar(stage), B_BYTES);
+            tma_load_2d_warp(smem_addr(st + A_BYTES), &tmB, kt * BKB, brow, full_bar(stage), pol);
           } else {
             // both boxes always transfer their full size (out-of-range atoms read as 0)
-            mbar_arrive_expect_tx(sfull_bar(stage), SFA_BYTES + SFB_BYTES);
-            tma_load_3d(smem_addr(st + A_BYTES + B_BYTES), &tmSA, 0, kt * 4,
+            mbar_arrive_expect_tx_warp(sfull_bar(stage), SFA_BYTES + SFB_BYTES);
+            tma_load_3d_warp(smem_addr(st + A_BYTES + B_BYTES), &tmSA, 0, kt * 4,
                         mb * CG + static_cast<int>(rank), sfull_bar(stage), pol);
-            tma_load_3d(smem_addr(st + A_BYTES + B_BYTES + SFA_BYTES), &tmSB, 0, kt * 4, nb * 2,
+            tma_load_3d_warp(smem_addr(st + A_BYTES + B_BYTES + SFA_BYTES), &tmSB, 0, kt * 4, nb * 2,
                         sfull_bar(stage), pol);
           }
           ++issued;
@@ -288,7 +289,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
           }
         }
       }
-      // every copy this thread issued must land before the CTA may exit
+      // every copy this warp issued must land before the CTA may exit
       const uint32_t mine = (warp == 3) ? 1u : 0u;
       for (int s = 0; s < STAGES && s < issued; ++s) {
         const int64_t uses = (issued - 1 - s) / STAGES + 1;
@@ -358,11 +359,12 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
   } else if (warp == 1) {
     // -------------------------------------------------------- MMA issuer
     // The tensor pipe accepts about one MMA ahead of the issuing thread, so
-    // the thread's own bookkeeping shows up as pipe idle time: it waits on a
-    // single barrier per stage (the scale writers arrive only once both the
-    // codes and the scales of the stage are in place), uses precomputed
-    // descriptors, and releases the previous stage right after MMA 0.
-    if (lane == 0 && rank == 0) {
+    // the issuer's own bookkeeping shows up as pipe idle time: the whole warp
+    // runs the loop (warp-uniform descriptors, one elected lane issues each
+    // MMA and commit), waits on a single barrier per stage (the scale writers
+    // arrive only once both the codes and the scales of the stage are in
+    // place), and releases the previous stage right after MMA 0.
+    if (rank == 0) {
       const uint32_t idesc = idesc_mxf4nvf4(BM * CG, BN);
       // the start-address field holds (address >> 4) and every stage lies below
       // 256 KB, so a stage's descriptor is the first one plus stage * STAGE_BYTES / 16
@@ -391,10 +393,10 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
           const uint64_t ad = adesc0 + soff, bd = bdesc0 + soff;
           const uint32_t col = tmem_base + SF_COL + SF_STRIDE * stage;
           // K = 64 fp4 = 32 bytes per MMA: advance the start address inside the swizzle atom
-          mma_mxf4nvf4_cg<CG>(tmem_base + ACC_COL, ad, bd, idesc, col, col + 16, kt != 0);
-          if (prev >= 0) tc_commit_all<CG>(empty_bar(prev));
+          mma_mxf4nvf4_warp<CG>(tmem_base + ACC_COL, ad, bd, idesc, col, col + 16, kt != 0);
+          if (prev >= 0) tc_commit_all_warp<CG>(empty_bar(prev));
           for (int kk = 1; kk < nk; ++kk)
-            mma_mxf4nvf4_cg<CG>(tmem_base + ACC_COL, ad + 2 * kk, bd + 2 * kk, idesc,
+            mma_mxf4nvf4_warp<CG>(tmem_base + ACC_COL, ad + 2 * kk, bd + 2 * kk, idesc,
                                 col + 4 * kk, col + 16 + 8 * kk, 1u);
           prev = stage;
           if (++stage == STAGES) {
@@ -402,12 +404,12 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             phase ^= 1u;
           }
         }
-        if (prev >= 0) tc_commit_all<CG>(empty_bar(prev));
+        if (prev >= 0) tc_commit_all_warp<CG>(empty_bar(prev));
         if (!ok) break;
-        tc_commit_all<CG>(tmem_full);
+        tc_commit_all_warp<CG>(tmem_full);
       }
       // all issued tensor-core work must finish before TMEM is freed
-      tc_commit_local<CG>(drain_mma);
+      tc_commit_local_warp<CG>(drain_mma);
       if (!mbar_wait(drain_mma, 0, g.wait_ns, nullptr)) record_error(SITE_DRAIN, 1);
     }
     __syncwarp();
@@ -581,7 +583,8 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0 || warp == 2) {
-    if (lane == 0) {
+    // warp-wide loop; one elected lane issues each copy
+    {
       const bool is_w = (warp == 0);
       // weights stream through once; tokens are re-read by every CTA
       const uint64_t pol = is_w ? policy_evict_first() : policy_evict_last();
@@ -597,14 +600,14 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
         const int nk = min(4, (g.K - kt * BK) / 64);
         uint8_t* st = smem + stage * C::STAGE_BYTES;
         if (is_w) {
-          mbar_arrive_expect_tx(full_bar(stage), W_BYTES + nk * 512);
-          tma_load_2d(smem_addr(st), &tmW, kt * BKB, wt * BW, full_bar(stage), pol);
-          bulk_load(smem_addr(st + W_BYTES + C::X_BYTES), g.sfb + (wt * kb4 + kt * 4) * 512,
+          mbar_arrive_expect_tx_warp(full_bar(stage), W_BYTES + nk * 512);
+          tma_load_2d_warp(smem_addr(st), &tmW, kt * BKB, wt * BW, full_bar(stage), pol);
+          bulk_load_warp(smem_addr(st + W_BYTES + C::X_BYTES), g.sfb + (wt * kb4 + kt * 4) * 512,
                     nk * 512, full_bar(stage), pol);
         } else {
-          mbar_arrive_expect_tx(full_bar(stage), C::X_BYTES + nk * 512);
-          tma_load_2d(smem_addr(st + W_BYTES), &tmX, kt * BKB, 0, full_bar(stage), pol);
-          bulk_load(smem_addr(st + W_BYTES + C::X_BYTES + SFW_BYTES), g.sfa + (kt * 4) * 512,
+          mbar_arrive_expect_tx_warp(full_bar(stage), C::X_BYTES + nk * 512);
+          tma_load_2d_warp(smem_addr(st + W_BYTES), &tmX, kt * BKB, 0, full_bar(stage), pol);
+          bulk_load_warp(smem_addr(st + W_BYTES + C::X_BYTES + SFW_BYTES), g.sfa + (kt * 4) * 512,
                     nk * 512, full_bar(stage), pol);
         }
         ++issued;
@@ -658,7 +661,9 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    // the whole warp runs the issuing loop (warp-uniform operands); one
+    // elected lane issues each MMA and commit
+    {
       const uint32_t idesc = idesc_mxf4nvf4(BW, NT);
       int stage = 0;
       uint32_t phase = 0;
@@ -678,16 +683,16 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
         const uint64_t xdesc = desc_kmajor_sw128(smem_addr(st + W_BYTES));
         const uint32_t col = tmem_base + SF_COL + SF_STRIDE * stage;
         for (int kk = 0; kk < nk; ++kk)
-          mma_mxf4nvf4(tmem_base + ACC_COL, wdesc + 2 * kk, xdesc + 2 * kk, idesc, col + 4 * kk,
-                       col + 16 + 4 * kk, (kt | kk) != 0);
-        tc_commit(empty_bar(stage));
+          mma_mxf4nvf4_warp<1>(tmem_base + ACC_COL, wdesc + 2 * kk, xdesc + 2 * kk, idesc,
+                               col + 4 * kk, col + 16 + 4 * kk, (kt | kk) != 0);
+        tc_commit_all_warp<1>(empty_bar(stage));
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1u;
         }
       }
-      if (ok) tc_commit(acc_full);
-      tc_commit(drain_mma);
+      if (ok) tc_commit_all_warp<1>(acc_full);
+      tc_commit_all_warp<1>(drain_mma);
       if (!mbar_wait(drain_mma, 0, g.wait_ns, nullptr)) record_error(SITE_DRAIN, 1);
     }
     __syncwarp();
