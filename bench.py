@@ -192,32 +192,59 @@ class Layer:
         return self.N * self.K // 2 + self.nv.nvfp4_scale_bytes(self.N, self.K)
 
 
-def time_steps(layer: Layer, steps: int, warmup: int, stream, per_kernel: bool):
-    """Device time of `steps` back-to-back steps (events on `stream`), plus per-kernel means."""
+# Steps are replayed from CUDA graphs: a host call of the library costs more
+# than some of its kernels (the quantiser, the decode GEMM), so launches
+# issued one by one from Python would leave the GPU idle between kernels and
+# the events would time the host.  A graph of GRAPH_STEPS steps covers the
+# activation (6), weight (4) and output (2) rotations exactly.
+GRAPH_STEPS = 12
+
+
+def capture(fn, start: int, count: int, stream):
+    """CUDA graph of fn(i, stream) for i in [start, start + count)."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(start, start + count):
+            fn(i, stream)
+    return g
+
+
+def replay_ms(graphs, stream):
+    """Device time of replaying `graphs` in order on `stream` (events on the stream)."""
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for g in graphs:
+            g.replay()
+        b.record(stream)
+    b.synchronize()
+    return a.elapsed_time(b)
+
+
+def time_steps(layer: Layer, steps: int, warmup: int, stream):
+    """Device time of exactly `steps` steps (quantise + GEMM), replayed from graphs."""
+    def step(i, st):
+        layer.quantize(i, st)
+        layer.gemm(i, st)
     for i in range(warmup):
-        layer.quantize(i, stream)
-        layer.gemm(i, stream)
+        step(i, stream)
     torch.cuda.synchronize()
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3 * steps + 1)] if per_kernel else None
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for i in range(steps):
-        if per_kernel:
-            ev[3 * i].record(stream)
-        layer.quantize(i, stream)
-        if per_kernel:
-            ev[3 * i + 1].record(stream)
-        layer.gemm(i, stream)
-        if per_kernel:
-            ev[3 * i + 2].record(stream)
-    end.record(stream)
-    end.synchronize()
-    total_ms = start.elapsed_time(end)
-    q_ms = g_ms = None
-    if per_kernel:
-        q_ms = sum(ev[3 * i].elapsed_time(ev[3 * i + 1]) for i in range(steps)) / steps
-        g_ms = sum(ev[3 * i + 1].elapsed_time(ev[3 * i + 2]) for i in range(steps)) / steps
-    return total_ms, q_ms, g_ms
+    full = capture(step, 0, GRAPH_STEPS, stream)
+    tail = capture(step, 0, steps % GRAPH_STEPS, stream) if steps % GRAPH_STEPS else None
+    replay_ms([full], stream)                               # first replay uploads the graph
+    seq = [full] * (steps // GRAPH_STEPS) + ([tail] if tail is not None else [])
+    return replay_ms(seq, stream)
+
+
+def time_kernels(layer: Layer, reps: int, stream):
+    """Mean device time of each kernel alone: graphs of GRAPH_STEPS quantiser
+    launches and of GRAPH_STEPS GEMM launches, each replayed `reps` times."""
+    gq = capture(lambda i, st: layer.quantize(i, st), 0, GRAPH_STEPS, stream)
+    gg = capture(lambda i, st: layer.gemm(i, st), 0, GRAPH_STEPS, stream)
+    replay_ms([gq, gg], stream)
+    q_ms = replay_ms([gq] * reps, stream) / (reps * GRAPH_STEPS)
+    g_ms = replay_ms([gg] * reps, stream) / (reps * GRAPH_STEPS)
+    return q_ms, g_ms
 
 
 def e2e(layer: Layer, steps: int, warmup: int, stream):
@@ -247,8 +274,9 @@ def e2e(layer: Layer, steps: int, warmup: int, stream):
     return ms, xh.numel() * 2, yh.numel() * 2
 
 
-def small_m_sweep(device, stream, iters=200, warmup=10):
-    """Decode-shaped sweep on the fused GDN in-projection weights: weight-stream GB/s."""
+def small_m_sweep(device, stream, iters=240, warmup=10):
+    """Decode-shaped sweep on the fused GDN in-projection weights: weight-stream
+    GB/s of the GEMM alone (graph replays over the rotated weight copies)."""
     import nvfp4_w4a4_quantized_quantizer_b200 as nv
     wl = workloads.WORKLOADS[5]
     out = {}
@@ -266,15 +294,14 @@ def small_m_sweep(device, stream, iters=200, warmup=10):
         for i in range(warmup):
             run(i)
         torch.cuda.synchronize()
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * iters)]
-        for i in range(iters):
+
+        def gemm(i, st):
             wc, ws = base.ws[i % len(base.ws)]
-            nv.nvfp4_quantize_act(x, base.a_gs, codes=c, scales=s, stream=stream)
-            ev[2 * i].record(stream)
-            nv.nvfp4_fused_linear(c, s, wc, ws, M, base.N, base.K, base.segs, y=y, stream=stream)
-            ev[2 * i + 1].record(stream)
-        torch.cuda.synchronize()
-        g_ms = statistics.median(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(iters))
+            nv.nvfp4_fused_linear(c, s, wc, ws, M, base.N, base.K, base.segs, y=y, stream=st)
+        g = capture(gemm, 0, GRAPH_STEPS, stream)
+        replay_ms([g], stream)
+        reps = max(1, iters // GRAPH_STEPS)
+        g_ms = replay_ms([g] * reps, stream) / (reps * GRAPH_STEPS)
         out[f"M={M}"] = {"gemm_us": round(g_ms * 1e3, 2),
                          "weight_GBps": round(base.weight_bytes / (g_ms * 1e-3) / 1e9, 1),
                          "tokens_per_s": round(M / (g_ms * 1e-3), 1)}
@@ -403,7 +430,7 @@ def main():
         pg.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        total_ms, _, _ = time_steps(layer, args.steps, args.warmup, stream, per_kernel=False)
+        total_ms = time_steps(layer, args.steps, args.warmup, stream)
     torch.cuda.synchronize()
     if pg:
         pg.barrier()
@@ -415,8 +442,8 @@ def main():
     ms_step = total_ms / args.steps
     value = ws * layer.flops / (ms_step * 1e-3) / 1e12
 
-    # per-kernel device times (separate pass, events around each launch)
-    _, q_ms, g_ms = time_steps(layer, min(args.steps, 500), 5, stream, per_kernel=True)
+    # per-kernel device times (separate pass: graphs of one kernel each)
+    q_ms, g_ms = time_kernels(layer, max(4, min(args.steps, 480) // GRAPH_STEPS), stream)
     pk = peaks()
     fp4_peak = pk["bf16"] * FP4_PER_BF16
     g_tflops = layer.flops / (g_ms * 1e-3) / 1e12
@@ -433,7 +460,8 @@ def main():
         "config": {"workload": wl.name, "M": M, "N": wl.N, "K": wl.K,
                    "step": "quantize_act + fused NVFP4 GEMM (bf16 out)",
                    "l2": f"inputs rotated over {ROTATE_ACT} activation / {ROTATE_W} weight copies "
-                         "(working set > L2)", "parallelism": f"replicas x{ws}"},
+                         "(working set > L2)", "parallelism": f"replicas x{ws}",
+                   "launch": f"steps replayed from CUDA graphs of {GRAPH_STEPS} steps"},
         "roofline": {"bound": "tensor", "achieved": round(g_tflops, 1), "peak": round(fp4_peak, 1),
                      "unit": "TFLOP/s", "frac": round(g_tflops / fp4_peak, 4),
                      "traffic": traffic,

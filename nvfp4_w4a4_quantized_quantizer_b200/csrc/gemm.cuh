@@ -698,38 +698,59 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
     __syncwarp();
   } else if (warp >= EPI_WARP0) {
     const int q = warp & 3;
-    const int n = wt * BW + q * 32 + lane;   // output feature of this lane
-    if (mbar_wait(acc_full, 0, g.wait_ns, abort_flag)) {
+    const int r = q * 32 + lane;                 // accumulator row = output column n0 + r
+    const int n = wt * BW + r;
+    // Thread r holds column n for all NT tokens.  The tile goes through
+    // shared memory (the stage ring is free once every MMA has completed) so
+    // that each token's 128 columns leave as 16-byte stores of one contiguous
+    // segment instead of NT strided 2-byte stores per thread.
+    const bool ok = mbar_wait(acc_full, 0, g.wait_ns, abort_flag);
+    if (ok) {
       tc_fence_after();
       uint32_t v[NT];
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ACC_COL;
 #pragma unroll
       for (int c = 0; c < NT / 16; ++c) {
-        uint32_t (&r)[16] = *reinterpret_cast<uint32_t(*)[16]>(v + 16 * c);
-        tmem_ld_x16(taddr + 16 * c, r);
+        uint32_t (&rr)[16] = *reinterpret_cast<uint32_t(*)[16]>(v + 16 * c);
+        tmem_ld_x16(taddr + 16 * c, rr);
       }
       tmem_wait_ld();
-      if (n < g.N) {
-        const int s = seg_advance(seg, 0, n);
-        const float alpha = seg.alpha[s];
-        const int op = seg.op[s];
-        const int h = n - seg.n_off[s];
+      const int s = seg_advance(seg, 0, n < g.N ? n : g.N - 1);
+      const float alpha = seg.alpha[s];
+      const int op = seg.op[s];
+      const int h = n - seg.n_off[s];
+      float* t32 = reinterpret_cast<float*>(smem);
+      __nv_bfloat16* t16 = reinterpret_cast<__nv_bfloat16*>(smem);
 #pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          if (j < g.M) {
-            float o = __fmul_rn(alpha, __uint_as_float(v[j]));
-            if (op != 0) o = apply_op_1(o, op, seg.a_log[s], seg.dt_bias[s], h);
-            if (g.out_fp32)
-              static_cast<float*>(g.y)[static_cast<int64_t>(j) * g.ldy + n] = o;
-            else
-              static_cast<__nv_bfloat16*>(g.y)[static_cast<int64_t>(j) * g.ldy + n] =
-                  __float2bfloat16_rn(o);
-          }
-        }
+      for (int j = 0; j < NT; ++j) {
+        float o = __fmul_rn(alpha, __uint_as_float(v[j]));
+        if (op != 0) o = apply_op_1(o, op, seg.a_log[s], seg.dt_bias[s], h);
+        if (g.out_fp32)
+          t32[j * BW + r] = o;
+        else
+          t16[j * BW + r] = __float2bfloat16_rn(o);
       }
     } else {
       if (!*abort_flag) record_error(SITE_EPI_TMEM_FULL, warp);
       *abort_flag = 1;
+    }
+    // all four epilogue warps pass this barrier exactly once, whatever their wait returned
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (ok && !*abort_flag) {
+      const int64_t n0 = static_cast<int64_t>(wt) * BW;
+      const int esz = g.out_fp32 ? 4 : 2;
+      const int chunks = BW * esz / 16;                 // 16-byte chunks per token row
+      const int per = 16 / esz;                         // columns per chunk
+      const int rows = g.M < NT ? g.M : NT;
+      for (int idx = r; idx < rows * chunks; idx += 128) {
+        const int j = idx / chunks, c = idx - j * chunks;
+        const int64_t col = n0 + c * per;
+        if (col < g.N) {                                // N % 16 == 0: chunks are whole
+          const uint4 val = *reinterpret_cast<const uint4*>(smem + (j * BW + c * per) * esz);
+          char* dst = static_cast<char*>(g.y) + (static_cast<int64_t>(j) * g.ldy + col) * esz;
+          *reinterpret_cast<uint4*>(dst) = val;
+        }
+      }
     }
   }
 
