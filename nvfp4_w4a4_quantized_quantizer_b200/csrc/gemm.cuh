@@ -61,14 +61,27 @@ struct GemmArgs {
 };
 
 // ------------------------------------------------------------- epilogue op
+// GDN gates: beta = sigmoid(v); g = -exp(A_log[h]) * softplus(v + dt_bias[h]),
+// softplus(z) = max(z, 0) + log(1 + exp(-|z|)).  They use the fast
+// exponential, logarithm and division: for the arguments that matter their
+// errors change beta by under 1e-6 and g by under ~5e-6 absolute, far below
+// what the GEMM's own 1e-3 rms tolerance moves either gate, and each gate is
+// then a handful of instructions instead of a few hundred cycles of
+// dependent full-precision library code (a column's gates for 64 tokens made
+// one CTA of the decode GEMM the last to finish).
+__device__ __forceinline__ float gate_sigmoid(float v) {
+  return __fdividef(1.0f, 1.0f + __expf(-v));
+}
+
+__device__ __forceinline__ float gate_decay(float v, float ea, float dtb) {
+  const float z = v + dtb;
+  return -ea * (fmaxf(z, 0.0f) + __logf(1.0f + __expf(-fabsf(z))));
+}
+
 __device__ __forceinline__ float apply_op(float v, int op, const float* a_log,
                                           const float* dt_bias, int h) {
-  if (op == 1) return 1.0f / (1.0f + expf(-v));
-  if (op == 2) {
-    const float z = v + __ldg(dt_bias + h);
-    const float sp = fmaxf(z, 0.0f) + log1pf(expf(-fabsf(z)));
-    return -expf(__ldg(a_log + h)) * sp;
-  }
+  if (op == 1) return gate_sigmoid(v);
+  if (op == 2) return gate_decay(v, __expf(__ldg(a_log + h)), __ldg(dt_bias + h));
   return v;
 }
 
@@ -77,13 +90,8 @@ __device__ __forceinline__ float apply_op(float v, int op, const float* a_log,
 // multiply the kernels' code size.
 __device__ __noinline__ void apply_op_16(float* o, int op, const float* a_log,
                                          const float* dt_bias, int h0) {
-#pragma unroll 1
+#pragma unroll
   for (int i = 0; i < 16; ++i) o[i] = apply_op(o[i], op, a_log, dt_bias, h0 + i);
-}
-
-__device__ __noinline__ float apply_op_1(float v, int op, const float* a_log,
-                                         const float* dt_bias, int h) {
-  return apply_op(v, op, a_log, dt_bias, h);
 }
 
 // Advance `seg` so that n lies in [n_off[seg], n_off[seg+1]).
@@ -507,6 +515,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
 // scales (MMA kk reads 16 + 4 kk + token / 32).
 namespace sm {
 constexpr int BW = 128;                 // weight rows per CTA (MMA M)
+constexpr int DIRECT_M = 8;             // up to this many tokens the epilogue stores directly
 constexpr int BK = 256;
 constexpr int BKB = BK / 2;
 constexpr int STAGES = 6;
@@ -700,10 +709,11 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
     const int q = warp & 3;
     const int r = q * 32 + lane;                 // accumulator row = output column n0 + r
     const int n = wt * BW + r;
-    // Thread r holds column n for all NT tokens.  The tile goes through
-    // shared memory (the stage ring is free once every MMA has completed) so
-    // that each token's 128 columns leave as 16-byte stores of one contiguous
-    // segment instead of NT strided 2-byte stores per thread.
+    // Thread r holds column n for all NT tokens.  With more than DIRECT_M
+    // tokens the tile goes through shared memory (the stage ring is free once
+    // every MMA has completed) so that each token's 128 columns leave as
+    // 16-byte stores of one contiguous segment instead of M strided 2-byte
+    // stores per thread.
     const bool ok = mbar_wait(acc_full, 0, g.wait_ns, abort_flag);
     if (ok) {
       tc_fence_after();
@@ -715,20 +725,48 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
         tmem_ld_x16(taddr + 16 * c, rr);
       }
       tmem_wait_ld();
-      const int s = seg_advance(seg, 0, n < g.N ? n : g.N - 1);
+      // columns past N (the last tile's padding) are never stored; they take
+      // no gate, so no gate parameter past the module's heads is read
+      const bool live = n < g.N;
+      const int s = seg_advance(seg, 0, live ? n : g.N - 1);
       const float alpha = seg.alpha[s];
-      const int op = seg.op[s];
+      const int op = live ? seg.op[s] : 0;     // columns past N take no gate
       const int h = n - seg.n_off[s];
+      const float ea = op == 2 ? __expf(__ldg(seg.a_log[s] + h)) : 0.0f;
+      const float dtb = op == 2 ? __ldg(seg.dt_bias[s] + h) : 0.0f;
       float* t32 = reinterpret_cast<float*>(smem);
       __nv_bfloat16* t16 = reinterpret_cast<__nv_bfloat16*>(smem);
-#pragma unroll
-      for (int j = 0; j < NT; ++j) {
-        float o = __fmul_rn(alpha, __uint_as_float(v[j]));
-        if (op != 0) o = apply_op_1(o, op, seg.a_log[s], seg.dt_bias[s], h);
-        if (g.out_fp32)
+      auto emit = [&](int j, float o) {
+        if (g.M <= DIRECT_M) {
+          // a few tokens: each warp store is still 64 contiguous bytes
+          if (live) {
+            if (g.out_fp32)
+              static_cast<float*>(g.y)[static_cast<int64_t>(j) * g.ldy + n] = o;
+            else
+              static_cast<__nv_bfloat16*>(g.y)[static_cast<int64_t>(j) * g.ldy + n] =
+                  __float2bfloat16_rn(o);
+          }
+        } else if (g.out_fp32) {
           t32[j * BW + r] = o;
-        else
+        } else {
           t16[j * BW + r] = __float2bfloat16_rn(o);
+        }
+      };
+      // one loop per op: the tokens of a gate column are independent, so the
+      // unrolled gate loop overlaps their latencies (padding tokens are never
+      // stored)
+      if (op == 0) {
+#pragma unroll
+        for (int j = 0; j < NT; ++j)
+          if (j < g.M) emit(j, __fmul_rn(alpha, __uint_as_float(v[j])));
+      } else if (op == 1) {
+#pragma unroll
+        for (int j = 0; j < NT; ++j)
+          if (j < g.M) emit(j, gate_sigmoid(__fmul_rn(alpha, __uint_as_float(v[j]))));
+      } else {
+#pragma unroll
+        for (int j = 0; j < NT; ++j)
+          if (j < g.M) emit(j, gate_decay(__fmul_rn(alpha, __uint_as_float(v[j])), ea, dtb));
       }
     } else {
       if (!*abort_flag) record_error(SITE_EPI_TMEM_FULL, warp);
@@ -736,7 +774,7 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
     }
     // all four epilogue warps pass this barrier exactly once, whatever their wait returned
     asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (ok && !*abort_flag) {
+    if (ok && !*abort_flag && g.M > DIRECT_M) {
       const int64_t n0 = static_cast<int64_t>(wt) * BW;
       const int esz = g.out_fp32 ? 4 : 2;
       const int chunks = BW * esz / 16;                 // 16-byte chunks per token row
