@@ -138,25 +138,6 @@ __device__ __forceinline__ void cluster_sync() {
       "barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// -------------------------------------------------------- TMA / bulk copy
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int32_t x,
-                                            int32_t y, uint32_t bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
-      : "memory");
-}
-
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int32_t x,
-                                            int32_t y, int32_t z, uint32_t bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar), "l"(policy)
-      : "memory");
-}
-
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
                                           uint32_t bar, uint64_t policy) {
   asm volatile(
@@ -252,32 +233,10 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// Arrive once on `bar` when every tcgen05 operation this thread issued so
-// far has completed.
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar)
-               : "memory");
-}
-
-// D[tmem] (+)= (A * SFA) x (B * SFB)^T, E2M1 operands in shared memory
-// (K-major), UE4M3 scale vectors of 16 elements in TMEM, fp32 accumulator.
-__device__ __forceinline__ void mma_mxf4nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                             uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
-                                             uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
-      "p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-      : "memory");
-}
-
 // CTA-pair forms (cta_group::2): the two CTAs of a cluster of 2 share one
 // MMA.  Allocation and release are executed by the same warp of both CTAs;
-// the MMA and the commits by one thread of the even CTA only.  Every
-// tcgen05 instruction of a kernel must use the same cta_group.
+// the MMAs and commits by one elected lane of the even CTA's MMA warp.
+// Every tcgen05 instruction of a kernel must use the same cta_group.
 template <int CG>
 __device__ __forceinline__ void tmem_alloc_cg(uint32_t dst_smem, uint32_t ncols) {
   if constexpr (CG == 1)
@@ -306,53 +265,15 @@ __device__ __forceinline__ void tmem_dealloc_cg(uint32_t taddr, uint32_t ncols) 
                  : "memory");
 }
 
-// Arrive once on `bar` (same shared offset) in every CTA of the pair when the
-// tcgen05 operations issued so far have completed.
-template <int CG>
-__device__ __forceinline__ void tc_commit_all(uint32_t bar) {
-  if constexpr (CG == 1)
-    tc_commit(bar);
-  else
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-        " [%0], %1;" ::"r"(bar),
-        "h"(static_cast<uint16_t>(3))
-        : "memory");
-}
-
-// Arrive once on this CTA's `bar` only.
-template <int CG>
-__device__ __forceinline__ void tc_commit_local(uint32_t bar) {
-  if constexpr (CG == 1)
-    tc_commit(bar);
-  else
-    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     bar)
-                 : "memory");
-}
-
+// D[tmem] (+)= (A * SFA) x (B * SFB)^T: E2M1 operands in shared memory
+// (K-major), UE4M3 scale vectors of 16 elements in TMEM, fp32 accumulator.
 // With CG = 2 the MMA is M = 256: rows 0-127 come from the even CTA's shared
 // memory and TMEM, rows 128-255 from the odd CTA's at the same addresses;
 // the N rows of B are split the same way (first half even CTA); each CTA's
 // TMEM holds its own 128 accumulator rows, its own A scales and all of B's.
-template <int CG>
-__device__ __forceinline__ void mma_mxf4nvf4_cg(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                                uint32_t idesc, uint32_t sfa_tmem,
-                                                uint32_t sfb_tmem, uint32_t accumulate) {
-  if constexpr (CG == 1)
-    mma_mxf4nvf4(d_tmem, a_desc, b_desc, idesc, sfa_tmem, sfb_tmem, accumulate);
-  else
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], "
-        "[%6], p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-        : "memory");
-}
-
-// Warp-wide forms: every lane of the warp executes them with the same
-// (warp-uniform) operands and one lane chosen by elect.sync issues the
+//
+// These are warp-wide forms: every lane of the warp executes them with the
+// same (warp-uniform) operands and one lane chosen by elect.sync issues the
 // instruction.  Keeping the issuing loop warp-wide lets the compiler hold
 // descriptors and TMEM addresses in uniform registers; issued from inside a
 // one-lane branch, each tcgen05.mma first moved its six operands into
@@ -383,7 +304,9 @@ __device__ __forceinline__ void mma_mxf4nvf4_warp(uint32_t d_tmem, uint64_t a_de
         : "memory");
 }
 
-// tc_commit_all / tc_commit_local issued by one elected lane of the warp.
+// Arrive once on `bar` (the same shared offset) in every CTA of the pair
+// when the tcgen05 operations issued so far have completed (_local: in this
+// CTA only).  Issued by one elected lane of the warp.
 template <int CG>
 __device__ __forceinline__ void tc_commit_all_warp(uint32_t bar) {
   if constexpr (CG == 1)
@@ -414,13 +337,6 @@ __device__ __forceinline__ void tc_commit_local_warp(uint32_t bar) {
         "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
             bar)
         : "memory");
-}
-
-// Copy 32 rows x 16 bytes from shared memory to TMEM lanes 0-31 and
-// replicate them into all four 32-lane sub-partitions (4 columns each).
-__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t src_desc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc)
-               : "memory");
 }
 
 __device__ __forceinline__ void tmem_wait_st() {
@@ -529,12 +445,6 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
 // bytes, 8-row atoms of 1024 bytes stacked contiguously.
 __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
   return smem_desc(saddr, 16, 1024, 2);
-}
-
-// Scale-factor atom for tcgen05.cp 32x128b: 32 rows of 16 contiguous bytes,
-// 8-row core matrices 128 bytes apart, no swizzle.
-__device__ __forceinline__ uint64_t desc_sf_atom(uint32_t saddr) {
-  return smem_desc(saddr, 0, 128, 0);
 }
 
 // Instruction descriptor of kind::mxf4nvf4: E2M1 A and B (format code 1),
