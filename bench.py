@@ -137,6 +137,35 @@ def ncu_traffic(name: str):
     return None
 
 
+# ------------------------------------------------------------ multi-rank
+# N > 1: one process per GPU, each a replica of the whole layer on its own
+# tokens (weak scaling, no data-path collective); the timed region is
+# bracketed by a barrier and a device synchronisation on both sides and the
+# reported time is the maximum over ranks.
+def timed_region(pg, fn, sync):
+    """Barrier + sync, fn() (returns device ms), sync + barrier."""
+    if pg is not None:
+        pg.barrier()
+    sync()
+    ms = fn()
+    sync()
+    if pg is not None:
+        pg.barrier()
+    return ms
+
+
+def max_over_ranks(value: float, pg, device) -> float:
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    if pg is not None:
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, flops_per_step: float, ms_step: float) -> float:
+    """Whole-job TFLOP/s: every rank runs one step of the workload per step time."""
+    return world * flops_per_step / (ms_step * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------- workloads
 def _dev_bf16(bits, device):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
@@ -426,21 +455,13 @@ def main():
     torch.cuda.synchronize()
 
     # main timed region: barrier + sync on both sides, max over ranks
-    if pg:
-        pg.barrier()
-    torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        total_ms = time_steps(layer, args.steps, args.warmup, stream)
-    torch.cuda.synchronize()
-    if pg:
-        pg.barrier()
+        total_ms = timed_region(pg, lambda: time_steps(layer, args.steps, args.warmup, stream),
+                                torch.cuda.synchronize)
     clocks = clk.summary()
-    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-    if pg:
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, pg, device)
     ms_step = total_ms / args.steps
-    value = ws * layer.flops / (ms_step * 1e-3) / 1e12
+    value = job_value(ws, layer.flops, ms_step)
 
     # per-kernel device times (separate pass: graphs of one kernel each)
     q_ms, g_ms = time_kernels(layer, max(4, min(args.steps, 480) // GRAPH_STEPS), stream)
