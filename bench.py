@@ -8,7 +8,11 @@ Default workload: the single prefill projection M=4096, K=5120, N=5120
 N(0, 1/sqrt(K)), static activation scale calibrated on a 512-row batch).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--workload prefill|gdn_inproj|decode]
+                    [--workload prefill|gdn_inproj|mlp|decode]
+
+--workload mlp times the MLP pair as one step (quantise, gate_up with two
+modules, SiLU(gate)*up, requantise, down GEMM); its roofline line is the
+gate_up GEMM, the down GEMM and the glue kernels are reported beside it.
 
 Prints one JSON line on rank 0.  Multi-GPU runs (torchrun, one rank per GPU)
 are weak-scaled replicas: every rank runs the same layer on its own batch, no
@@ -221,6 +225,82 @@ class Layer:
         return self.N * self.K // 2 + self.nv.nvfp4_scale_bytes(self.N, self.K)
 
 
+class MlpChain:
+    """The MLP pair as one step: quantise x, gate_up (two modules, one fused
+    GEMM), h = bf16(SiLU(gate) * up), requantise h under its calibrated global
+    scale, down GEMM.  Activation copies rotate over 3, weight sets over 2
+    (working set > L2)."""
+
+    def __init__(self, device, rotate_act=3, rotate_w=2):
+        import nvfp4_w4a4_quantized_quantizer_b200 as nv
+        wl = workloads.WORKLOADS[4]
+        self.nv, self.wl = nv, wl
+        self.M, self.K, self.N = wl.M, wl.K, wl.N
+        self.H, self.N2 = wl.N // 2, workloads.MLP_DOWN_N
+        assert workloads.MLP_DOWN_K == self.H
+        calib = _dev_bf16(workloads.activations(wl, calib=True), device)
+        self.a_gs = nv.nvfp4_global_scale(nv.nvfp4_amax(calib).item())
+        self.x_host = workloads.activations(wl)
+        x = _dev_bf16(self.x_host, device)
+        self.xs = [x] + [x.clone() for _ in range(rotate_act - 1)]
+        wbits = _dev_bf16(workloads.weights(wl), device)
+        wc, ws, self.w_gs = nv.nvfp4_quantize_weight(wbits, seg_offsets=wl.seg_offsets)
+        del wbits
+        w2bits = _dev_bf16(workloads.down_weights(), device)
+        w2c, w2s, (self.w2_gs,) = nv.nvfp4_quantize_weight(w2bits)
+        del w2bits
+        self.segs = [nv.SegmentSpec(off, g, self.a_gs) for off, g in zip(wl.seg_offsets, self.w_gs)]
+        # the down input's static global scale: the chain on the calibration batch
+        cc, cs = nv.nvfp4_quantize_act(calib, self.a_gs)
+        gu_cal = nv.nvfp4_fused_linear(cc, cs, wc, ws, calib.shape[0], self.N, self.K, self.segs)
+        h_cal = nv.nvfp4_silu_mul(gu_cal, self.H)
+        self.a2_gs = nv.nvfp4_global_scale(nv.nvfp4_amax(h_cal).item())
+        del calib, cc, cs, gu_cal, h_cal
+        self.ws = [(wc, ws, w2c, w2s)] + [tuple(t.clone() for t in (wc, ws, w2c, w2s))
+                                          for _ in range(rotate_w - 1)]
+        self.xc = torch.empty((self.M, self.K // 2), dtype=torch.uint8, device=device)
+        self.xsc = torch.empty(nv.nvfp4_scale_bytes(self.M, self.K), dtype=torch.uint8, device=device)
+        self.gu = torch.empty((self.M, self.N), dtype=torch.bfloat16, device=device)
+        self.h = torch.empty((self.M, self.H), dtype=torch.bfloat16, device=device)
+        self.hc = torch.empty((self.M, self.H // 2), dtype=torch.uint8, device=device)
+        self.hsc = torch.empty(nv.nvfp4_scale_bytes(self.M, self.H), dtype=torch.uint8, device=device)
+        self.y = torch.empty((self.M, self.N2), dtype=torch.bfloat16, device=device)
+        self.ys = [self.y, self.y]
+
+    def quantize(self, i, stream, x=None):
+        xx = self.xs[i % len(self.xs)] if x is None else x
+        self.nv.nvfp4_quantize_act(xx, self.a_gs, codes=self.xc, scales=self.xsc, stream=stream)
+
+    def gate_up(self, i, stream):
+        wc, ws, _, _ = self.ws[i % len(self.ws)]
+        self.nv.nvfp4_fused_linear(self.xc, self.xsc, wc, ws, self.M, self.N, self.K, self.segs,
+                                   y=self.gu, stream=stream)
+
+    def silu(self, i, stream):
+        self.nv.nvfp4_silu_mul(self.gu, self.H, h=self.h, stream=stream)
+
+    def requantize(self, i, stream):
+        self.nv.nvfp4_quantize_act(self.h, self.a2_gs, codes=self.hc, scales=self.hsc, stream=stream)
+
+    def down(self, i, stream):
+        _, _, w2c, w2s = self.ws[i % len(self.ws)]
+        self.nv.nvfp4_linear(self.hc, self.hsc, self.a2_gs, w2c, w2s, self.w2_gs, self.M, self.N2,
+                             self.H, y=self.y, stream=stream)
+
+    def gemm(self, i, stream):
+        """Everything after the first quantisation."""
+        self.gate_up(i, stream)
+        self.silu(i, stream)
+        self.requantize(i, stream)
+        self.down(i, stream)
+
+    launches_per_step = 5
+
+    @property
+    def flops(self):
+        return 2.0 * self.M * self.K * self.N + 2.0 * self.M * self.H * self.N2
+
+
 # Steps are replayed from CUDA graphs: a host call of the library costs more
 # than some of its kernels (the quantiser, the decode GEMM), so launches
 # issued one by one from Python would leave the GPU idle between kernels and
@@ -265,6 +345,14 @@ def time_steps(layer: Layer, steps: int, warmup: int, stream):
     return replay_ms(seq, stream)
 
 
+def time_each(fns, reps: int, stream):
+    """Mean device time (ms) of each named launch alone: a graph of
+    GRAPH_STEPS launches of it, replayed `reps` times."""
+    graphs = {name: capture(fn, 0, GRAPH_STEPS, stream) for name, fn in fns.items()}
+    replay_ms(list(graphs.values()), stream)
+    return {name: replay_ms([g] * reps, stream) / (reps * GRAPH_STEPS) for name, g in graphs.items()}
+
+
 def time_kernels(layer: Layer, reps: int, stream):
     """Mean device time of each kernel alone: graphs of GRAPH_STEPS quantiser
     launches and of GRAPH_STEPS GEMM launches, each replayed `reps` times."""
@@ -280,7 +368,7 @@ def e2e(layer: Layer, steps: int, warmup: int, stream):
     """Same metric through the public API from pinned host buffers: H2D of the
     step's activations, quantise, GEMM, D2H of the bf16 output, every step."""
     xh = torch.from_numpy(layer.x_host.view(np.int16)).view(torch.bfloat16).pin_memory()
-    yh = torch.empty((layer.M, layer.N), dtype=torch.bfloat16).pin_memory()
+    yh = torch.empty(tuple(layer.ys[0].shape), dtype=torch.bfloat16).pin_memory()
     xd = torch.empty_like(layer.xs[0])
 
     def one(i):
@@ -396,7 +484,7 @@ def cpu_baseline(wl: workloads.Workload, target_s: float = 12.0, rows: int = 32)
 
 
 # ------------------------------------------------------------------ main
-WORKLOAD_BY_NAME = {"prefill": 2, "gdn_inproj": 3, "decode": 5}
+WORKLOAD_BY_NAME = {"prefill": 2, "gdn_inproj": 3, "mlp": 4, "decode": 5}
 
 
 def main():
@@ -451,7 +539,8 @@ def main():
                                 device_id=device)
         pg = dist
     stream = torch.cuda.Stream(device)
-    layer = Layer(wl, M, device)
+    mlp = args.workload == "mlp"
+    layer = MlpChain(device) if mlp else Layer(wl, M, device)
     torch.cuda.synchronize()
 
     # main timed region: barrier + sync on both sides, max over ranks
@@ -464,13 +553,37 @@ def main():
     value = job_value(ws, layer.flops, ms_step)
 
     # per-kernel device times (separate pass: graphs of one kernel each)
-    q_ms, g_ms = time_kernels(layer, max(4, min(args.steps, 480) // GRAPH_STEPS), stream)
+    reps = max(4, min(args.steps, 480) // GRAPH_STEPS)
     pk = peaks()
     fp4_peak = pk["bf16"] * FP4_PER_BF16
-    g_tflops = layer.flops / (g_ms * 1e-3) / 1e12
+    if mlp:
+        t = time_each({"quantize": layer.quantize, "gate_up": layer.gate_up, "silu_mul": layer.silu,
+                       "requantize": layer.requantize, "down": layer.down}, max(2, reps // 4), stream)
+        q_ms, g_ms = t["quantize"], t["gate_up"]
+        g_flops = 2.0 * layer.M * layer.K * layer.N           # the dominant kernel: gate_up
+        d_tflops = 2.0 * layer.M * layer.H * layer.N2 / (t["down"] * 1e-3) / 1e12
+        rq_bytes = layer.M * layer.H * 2 + layer.M * layer.H // 2 + nv.nvfp4_scale_bytes(layer.M, layer.H)
+        extra = {"down_us": round(t["down"] * 1e3, 2), "down_tflops": round(d_tflops, 1),
+                 "down_frac": round(d_tflops / fp4_peak, 4),
+                 "silu_mul_us": round(t["silu_mul"] * 1e3, 2),
+                 "requantize_us": round(t["requantize"] * 1e3, 2),
+                 "requantize_GBps": round(rq_bytes / (t["requantize"] * 1e-3) / 1e9, 1)}
+        step_desc = ("quantize_act + gate_up (2 modules) + silu_mul + quantize_act + down GEMM "
+                     "(bf16 out)")
+        cfg_shape = {"M": layer.M, "K": layer.K, "N_gate_up": layer.N, "N_down": layer.N2,
+                     "K_down": layer.H}
+        profile = f"gemm_tc_{wl.name}.md"
+    else:
+        q_ms, g_ms = time_kernels(layer, reps, stream)
+        g_flops = layer.flops
+        extra = {}
+        step_desc = "quantize_act + fused NVFP4 GEMM (bf16 out)"
+        cfg_shape = {"M": M, "N": wl.N, "K": wl.K}
+        profile = f"gemm_tc_{wl.name}.md"
+    g_tflops = g_flops / (g_ms * 1e-3) / 1e12
     q_bytes = layer.M * layer.K * 2 + layer.M * layer.K // 2 + nv.nvfp4_scale_bytes(layer.M, layer.K)
     q_gbs = q_bytes / (q_ms * 1e-3) / 1e9
-    traffic = ncu_traffic(f"gemm_tc_{wl.name}.md")
+    traffic = ncu_traffic(profile)
 
     e_ms, h2d, d2h = e2e(layer, max(20, min(200, args.steps // 20)), 3, stream)
     line = {
@@ -478,9 +591,9 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4",
         "data": "synthetic",
-        "config": {"workload": wl.name, "M": M, "N": wl.N, "K": wl.K,
-                   "step": "quantize_act + fused NVFP4 GEMM (bf16 out)",
-                   "l2": f"inputs rotated over {ROTATE_ACT} activation / {ROTATE_W} weight copies "
+        "config": {"workload": wl.name, **cfg_shape,
+                   "step": step_desc,
+                   "l2": f"inputs rotated over {len(layer.xs)} activation / {len(layer.ws)} weight copies "
                          "(working set > L2)", "parallelism": f"replicas x{ws}",
                    "launch": f"steps replayed from CUDA graphs of {GRAPH_STEPS} steps"},
         "roofline": {"bound": "tensor", "achieved": round(g_tflops, 1), "peak": round(fp4_peak, 1),
@@ -489,10 +602,10 @@ def main():
                      "peak_note": f"{pk['source']} bf16 burst {pk['bf16']} x {FP4_PER_BF16} nominal FP4/BF16"},
         "kernels": {"gemm_us": round(g_ms * 1e3, 2), "gemm_tflops": round(g_tflops, 1),
                     "quantize_us": round(q_ms * 1e3, 2), "quantize_GBps": round(q_gbs, 1),
-                    "quantize_hbm_frac": round(q_gbs / pk["hbm"], 4)},
+                    "quantize_hbm_frac": round(q_gbs / pk["hbm"], 4), **extra},
         "e2e": {"value": round(layer.flops / (e_ms * 1e-3) / 1e12, 2), "unit": "TFLOPS",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": (layer.launches_per_step if mlp else 2) * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and not args.no_small_m and ws == 1:

@@ -214,8 +214,10 @@ nvfp4_status nvfp4_last_device_error(nvfp4_stream_t stream, uint64_t* info);
  * kernel, 64 < M <= 128 -> one-CTA tensor-core kernel, M > 128 -> CTA-pair
  * tensor-core kernel), 1 = always the one-CTA tensor-core kernel (128 x 256
  * tiles), 2 = always the small-M kernel (requires M <= 64), 3 = always the
- * CTA-pair tensor-core kernel (256 x 256 tiles on clusters of two CTAs).
- * Process-wide. */
+ * CTA-pair tensor-core kernel (256 x 256 tiles on clusters of two CTAs),
+ * 4 = the CTA-pair kernel with its tiles walked N fastest (the order chosen
+ * automatically when the activation codes exceed 64 MB and the weight codes
+ * are smaller).  Process-wide. */
 nvfp4_status nvfp4_set_gemm_path(int32_t path);
 
 /* Time limit of every bounded in-kernel wait, in nanoseconds (default 2e9;

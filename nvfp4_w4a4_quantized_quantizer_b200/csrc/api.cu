@@ -361,7 +361,7 @@ const char* nvfp4_status_string(nvfp4_status s) {
 }
 
 nvfp4_status nvfp4_set_gemm_path(int32_t path) {
-  if (path < 0 || path > 3) return NVFP4_ERR_INVALID_ARG;
+  if (path < 0 || path > 4) return NVFP4_ERR_INVALID_ARG;
   g_gemm_path = path;
   return NVFP4_OK;
 }
@@ -524,6 +524,15 @@ nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales, const
   g.sector_stores = ((reinterpret_cast<uintptr_t>(y) & 31u) == 0) &&
                     ((ldy * (g.out_fp32 ? 4 : 2)) % 32 == 0);
   g.wait_ns = g_wait_ns;
+  // Tile raster.  Consecutive CTAs (pairs) run tiles that share one operand
+  // tile, and the rest of that operand is re-read from L2 for each of the
+  // other operand's tiles.  By default they share weight tiles (M fastest),
+  // which keeps the activations L2-resident; when the activation codes are
+  // too large to stay in the 126 MB L2 (e.g. the MLP down projection's
+  // 16384 x 17408 input, 143 MB) and the weights are smaller, they share
+  // activation tiles instead, so the activations stream from HBM once.
+  const int64_t a_bytes = M * (K / 2), w_bytes = N * (K / 2);
+  g.n_fastest = (g_gemm_path == 4) || (a_bytes > (64ll << 20) && w_bytes < a_bytes);
 
   const bool small = (g_gemm_path == 2) || (g_gemm_path == 0 && M <= 64);
   if (small) {
@@ -548,7 +557,7 @@ nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales, const
     return launch(nvfp4::k_gemm_small<64>, nvfp4::sm::Cfg<64>::SMEM_BYTES);
   }
 
-  const bool pair = (g_gemm_path == 3) || (g_gemm_path == 0 && M > 128);
+  const bool pair = (g_gemm_path >= 3) || (g_gemm_path == 0 && M > 128);
   CUtensorMap ta, tb, tsa, tsb;
   if ((st = code_map(a_codes, M, K / 2, nvfp4::tc::BM, dev, &ta)) != NVFP4_OK) return st;
   if ((st = code_map(w_codes, N, K / 2, nvfp4::tc::BN / (pair ? 2 : 1), dev, &tb)) != NVFP4_OK)

@@ -57,6 +57,8 @@ struct GemmArgs {
   int64_t ldy;
   int out_fp32;
   int sector_stores;   // y base 32-byte aligned and rows a multiple of 32 bytes
+  int n_fastest;       // tile raster: 0 = M fastest (consecutive CTAs share a weight tile),
+                       // 1 = N fastest (they share an activation tile)
   uint64_t wait_ns;
 };
 
@@ -265,8 +267,8 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       int64_t issued = 0;
       bool ok = true;
       for (int tile = unit; tile < num_tiles && ok; tile += units) {
-        const int mb = tile % num_m;
-        const int nb = tile / num_m;
+        const int mb = g.n_fastest ? tile / num_n : tile % num_m;
+        const int nb = g.n_fastest ? tile % num_n : tile / num_m;
         const int arow = (mb * CG + static_cast<int>(rank)) * BM;
         const int brow = nb * BN + static_cast<int>(rank) * C::B_ROWS;
         for (int kt = 0; kt < num_kt; ++kt) {
@@ -429,8 +431,8 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     const int row_in_tile = q * 32 + lane;
     int local = 0;
     for (int tile = unit; tile < num_tiles; tile += units, ++local) {
-      const int mb = tile % num_m;
-      const int nb = tile / num_m;
+      const int mb = g.n_fastest ? tile / num_n : tile % num_m;
+      const int nb = g.n_fastest ? tile % num_n : tile / num_m;
       if (!wait_pair(tmem_full, static_cast<uint32_t>(local & 1))) {
         raise_abort(SITE_EPI_TMEM_FULL, warp);
         break;

@@ -128,7 +128,7 @@ def test_linear_and_weight_validation(lib):
 
 
 def test_misc_validation(lib):
-    assert lib.nvfp4_set_gemm_path(4) == INVALID
+    assert lib.nvfp4_set_gemm_path(5) == INVALID
     assert lib.nvfp4_set_gemm_path(0) == 0
     assert lib.nvfp4_set_wait_limit_ns(0) == INVALID
     assert lib.nvfp4_silu_mul(P, 4, 12, 24, P, 12, NUL) == SHAPE       # H % 8

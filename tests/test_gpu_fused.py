@@ -20,7 +20,7 @@ from tests import _helpers as H
 
 pytestmark = pytest.mark.gpu
 
-LARGE, SMALL, AUTO, PAIR = 1, 2, 0, 3
+LARGE, SMALL, AUTO, PAIR, PAIR_NFAST = 1, 2, 0, 3, 4
 OPS = {"none": nv.OP_NONE, "sigmoid": nv.OP_SIGMOID, "gdn_decay": nv.OP_GDN_DECAY}
 
 
@@ -79,7 +79,7 @@ def _run_fused(path, M, K, seed):
 
 
 @pytest.mark.parametrize("path,M,K", [(LARGE, 200, 320), (LARGE, 384, 1024), (PAIR, 200, 320),
-                                      (PAIR, 600, 1024), (SMALL, 5, 320),
+                                      (PAIR, 600, 1024), (PAIR_NFAST, 600, 1024), (SMALL, 5, 320),
                                       (SMALL, 64, 512), (AUTO, 1, 256)])
 def test_fused_gdn_segments_and_gates(path, M, K):
     widths, offs, ops, a_log, y32, yb, ref, pre, _ = _run_fused(path, M, K, seed=M + K)

@@ -17,7 +17,7 @@ from tests import _helpers as H
 
 pytestmark = pytest.mark.gpu
 
-LARGE, SMALL, AUTO, PAIR = 1, 2, 0, 3
+LARGE, SMALL, AUTO, PAIR, PAIR_NFAST = 1, 2, 0, 3, 4
 
 
 @pytest.fixture(autouse=True)
@@ -57,7 +57,7 @@ def run(path, ac, as_, a_gs, wc, ws, w_gs, M, N, K):
     return y32.cpu().numpy(), yb.float().cpu().numpy()
 
 
-@pytest.mark.parametrize("path,M", [(LARGE, 16), (SMALL, 16), (PAIR, 16)])
+@pytest.mark.parametrize("path,M", [(LARGE, 16), (SMALL, 16), (PAIR, 16), (PAIR_NFAST, 16)])
 @pytest.mark.parametrize("p", [0, 1, 14, 15, 16, 31, 63, 64, 127, 128, 200, 255])
 def test_all_code_pairs_single_k(path, M, p):
     """Row m holds code m, column n holds code n, both at k = p only; random scales."""
@@ -86,7 +86,9 @@ def test_all_code_pairs_single_k(path, M, p):
     # CTA pairs: odd CTA's rows all past M (M <= 128), a ragged last tile
     # whose odd-CTA weight rows lie past N, several tiles per pair
     (PAIR, 100, 272, 320), (PAIR, 256, 256, 256), (PAIR, 300, 608, 1280),
-    (PAIR, 129, 16, 64), (PAIR, 2048, 2560, 256), (PAIR, 2304, 5120, 512)])
+    (PAIR, 129, 16, 64), (PAIR, 2048, 2560, 256), (PAIR, 2304, 5120, 512),
+    # tiles walked N fastest (ragged M and N tiles, several tiles per pair)
+    (PAIR_NFAST, 300, 608, 1280), (PAIR_NFAST, 2304, 5120, 512), (PAIR_NFAST, 129, 16, 64)])
 def test_random_codes_and_scales(path, M, N, K):
     rng = np.random.default_rng(M * 131 + N * 7 + K)
     ac = rng.integers(0, 16, size=(M, K)).astype(np.uint8)
@@ -171,7 +173,7 @@ def test_output_row_stride_and_no_overwrite():
     A, W = dev_operands(ac, as_, M, K), dev_operands(wc, ws, N, K)
     ref = oracle.linear64(oracle.dequantize(ac, as_, np.float32(0.01)),
                           oracle.dequantize(wc, ws, np.float32(0.02)))
-    for path, m in ((LARGE, M), (PAIR, M), (SMALL, 40)):
+    for path, m in ((LARGE, M), (PAIR, M), (PAIR_NFAST, M), (SMALL, 40)):
         nv.nvfp4_set_gemm_path(path)
         y = torch.full((m, ldy), -7.0, dtype=torch.float32, device="cuda")
         nv.nvfp4_linear(A[0], A[1], 0.01, W[0], W[1], 0.02, m, N, K, y=y[:, :N],
