@@ -22,6 +22,8 @@ Pinning status (what each function is checked against in ``tests/``):
   fused_linear64             -- closed-form mismatch ratio, per-segment
                                 decomposition
   sigmoid64 / gdn_decay64    -- Lipschitz bounds, limits, closed values
+  silu_mul_bf16              -- ml_dtypes bfloat16 RNE (random and exact ties),
+                                closed values and limits of SiLU
 No function is "parity unpinned".
 """
 from .nvfp4 import (  # noqa: F401

@@ -175,3 +175,46 @@ def test_gates_contract_relative_error(op):
     rel_in = np.linalg.norm(y_noisy - y) / np.linalg.norm(y)
     rel_out = np.linalg.norm(out_n - out) / np.linalg.norm(out)
     assert rel_out < rel_in
+
+
+# ------------------------------------------------- MLP glue (SiLU(gate) * up)
+def test_silu_mul_bf16_rounding_matches_ml_dtypes():
+    """The bf16 rounding step against an independent RNE: ml_dtypes' bfloat16
+    cast of the same float32 products (random, ties at every exponent, and
+    values whose low 16 bits are exactly 0x8000)."""
+    rng = np.random.default_rng(21)
+    g = rng.standard_normal(20000) * 4
+    u = rng.standard_normal(20000) * 3
+    h = oracle.silu_mul_bf16(g, u)
+    prod32 = (g * (1.0 / (1.0 + np.exp(-g))) * u).astype(np.float32)
+    want = prod32.astype(ml_dtypes.bfloat16).astype(np.float32)
+    # the oracle's product is float64 rounded once to float32, as here; allow
+    # the rare case where the two float64 evaluations land on different float32s
+    diff = h != want
+    assert diff.mean() < 1e-3
+    ulp = np.abs(want[diff]) * 2.0 ** -7
+    assert np.all(np.abs(h[diff] - want[diff]) <= ulp)
+    # exact ties: float32 values halfway between two bf16 values round to even
+    base = np.array([1.0, 1.5, -3.25, 1000.0], np.float32).view(np.uint32)
+    ties = (base | 0x8000).view(np.float32)
+    # silu(50) = 50 exactly in float64 (sigmoid(50) rounds to 1), and
+    # 50 * (tie / 50) in float64 rounds back to the float32 tie
+    got = oracle.silu_mul_bf16(np.full(4, 50.0), ties.astype(np.float64) / 50.0)
+    np.testing.assert_array_equal(got, ties.astype(ml_dtypes.bfloat16).astype(np.float32))
+
+
+def test_silu_mul_bf16_closed_values_and_limits():
+    up = np.array([3.0, -2.0, 0.5], np.float64)
+    # silu(0) = 0
+    np.testing.assert_array_equal(oracle.silu_mul_bf16(np.zeros(3), up), np.zeros(3, np.float32))
+    # silu(g) -> g for large g, -> 0 for very negative g
+    big = oracle.silu_mul_bf16(np.full(3, 40.0), up)
+    np.testing.assert_allclose(big, (40.0 * up).astype(np.float32), rtol=2.0 ** -8)
+    neg = oracle.silu_mul_bf16(np.full(3, -60.0), up)
+    assert np.all(np.abs(neg) < 1e-20)
+    # silu(1) * 1 = 1 / (1 + e^-1), to bf16 precision
+    one = oracle.silu_mul_bf16(np.array([1.0]), np.array([1.0]))
+    assert abs(float(one[0]) - 1.0 / (1.0 + np.exp(-1.0))) <= 2.0 ** -9
+    # the output holds bf16 values only
+    h = oracle.silu_mul_bf16(np.linspace(-8, 8, 999), np.linspace(3, -3, 999))
+    assert np.all((h.view(np.uint32) & 0xFFFF) == 0)
