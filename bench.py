@@ -121,10 +121,37 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source with comments and blank lines removed (string literals kept)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c == '"' or c == "'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            i = text.find("\n", i)
+            i = n if i < 0 else i
+        elif text.startswith("/*", i):
+            i = text.find("*/", i + 2)
+            i = n if i < 0 else i + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (ln.rstrip() for ln in "".join(out).splitlines())
+    return "\n".join(ln for ln in lines if ln.strip())
+
+
 def source_digest():
+    """Digest of the kernel sources' code (comments do not count): a profile's
+    counters apply while this matches the digest recorded with them."""
     h = hashlib.sha256()
     for f in ("ptx.cuh", "gemm.cuh", "quantize.cuh", "api.cu"):
-        h.update(open(os.path.join(ROOT, "nvfp4_w4a4_quantized_quantizer_b200", "csrc", f), "rb").read())
+        text = open(os.path.join(ROOT, "nvfp4_w4a4_quantized_quantizer_b200", "csrc", f)).read()
+        h.update(_code_only(text).encode())
     return h.hexdigest()[:16]
 
 

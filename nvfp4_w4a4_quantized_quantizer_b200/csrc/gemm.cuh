@@ -105,16 +105,18 @@ __device__ __forceinline__ int seg_advance(const SegTable& t, int seg, int n) {
 // ============================================================ k_gemm_tc
 // Warp roles (16 warps, four warpgroups):
 //   WG0  warp 0 producer A: TMA of the activation codes; warp 1 MMA issuer
-//        (tcgen05.mma only) and TMEM owner; warp 2 producer B: TMA of the
-//        weight codes; warp 3 producer S: TMA of both operands' scale atoms
-//        on a barrier of their own, so the scale writers need not wait for
-//        the codes.
+//        and TMEM owner (the whole warp runs the loop, one elected lane
+//        issues each MMA and commit); warp 2 producer B: TMA of the weight
+//        codes; warp 3 producer S: TMA of both operands' scale atoms on a
+//        barrier of their own, so the scale writers need not wait for the
+//        codes.
 //   WG1  warps 4-7 scale writers: warp w reads, from the stage in shared
 //        memory, the scale bytes TMEM lane quarter w % 4 needs and writes
-//        them with tcgen05.st into that stage's TMEM scale region.  A
-//        tcgen05.cp costs the tensor pipe ~70-150 cycles whatever its size,
-//        and a k-tile needs 12 of them; register stores of the same bytes
-//        take ~40 cycles per stage and run beside the MMAs.
+//        them with tcgen05.st into that stage's TMEM scale region.  A k-tile
+//        needs 12 tcgen05.cp copies of scale atoms, each holding the issuing
+//        thread ~100-150 cycles (issued by the MMA thread they made the
+//        prefill GEMM about twice as slow); register stores of the same
+//        bytes take ~40 cycles per stage and run beside the MMAs.
 //   WG2-3 warps 8-15 epilogue: warp w drains lane quarter w % 4, column
 //        half (w - 8) / 4.
 // TMEM: accumulator columns [0, 256); stage s scale region [256 + 48 s, +48):
@@ -126,10 +128,15 @@ __device__ __forceinline__ int seg_advance(const SegTable& t, int seg, int n) {
 // MMAs issued by the even CTA: each CTA loads its own 128 activation rows,
 // half of the tile's 256 weight rows and all 256 weight rows' scales.  Per
 // k-tile a CTA then brings in 38 KB instead of 54 KB for the same number of
-// tensor-core cycles; the L2 -> shared-memory stream, not the tensor pipe,
-// is what bounds the one-CTA tile.  The odd CTA's scale writers and
-// epilogue warps arrive on the even CTA's barriers through the cluster's
-// shared window; the MMA commits arrive on both CTAs' barriers.
+// tensor-core cycles (prefill 4096 x 5120 x 5120: 498 MB of L2 -> shared
+// memory traffic instead of 708 MB, 49.6 us instead of 57).  The odd CTA's
+// scale writers and epilogue warps arrive on the even CTA's barriers
+// through the cluster's shared window; the MMA commits arrive on both CTAs'
+// barriers.
+//
+// Tiles are walked M fastest (consecutive CTAs share a weight tile and the
+// activations stay in L2) or, when GemmArgs::n_fastest is set, N fastest
+// (they share an activation tile: for activations too large for the L2).
 namespace tc {
 constexpr int BM = 128;                 // rows of A per CTA
 constexpr int BN = 256;                 // tile columns (MMA N)
