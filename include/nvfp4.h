@@ -126,13 +126,21 @@ nvfp4_status nvfp4_amax(const void* x_bf16, int64_t R, int64_t K, int64_t ldx,
 
 /* Activation quantisation (step a1): bf16 x [M, K] -> codes [M, K/2] and
  * scales (atom layout, padding rows zeroed) under the static global scale
- * a_gs > 0.  All pointers are device pointers. */
+ * a_gs > 0.  The operation is the NVFP4 16-element block scaling of the
+ * activations (bayesiansapien wiki, "The four-part mechanism study", part 1;
+ * nefut abstract: all linear layers W4A4) under a calibrated static scale
+ * (aimodeling, "Where the taboo came from": calibration-only PTQ).  All
+ * pointers are caller-owned device memory; x is read, codes and scales are
+ * overwritten.  Arguments are checked before any launch (INVALID_ARG,
+ * ALIGNMENT, UNSUPPORTED_SHAPE); the kernel is queued on `stream`. */
 nvfp4_status nvfp4_quantize_act(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
                                 float a_gs, void* codes, void* scales,
                                 nvfp4_stream_t stream);
 
-/* Weight quantisation (step a2, offline).  W [N, K] bf16 is split into
- * modules at seg_offsets (HOST array of nseg ascending row offsets, first 0,
+/* Weight quantisation (step a2, offline; the W4 half of W4A4, nefut
+ * abstract, with one global scale per module as the fused-projection repair
+ * needs: bayesiansapien wiki, "Two practical repairs").  W [N, K] bf16 is
+ * split into modules at seg_offsets (HOST array of nseg ascending row offsets, first 0,
  * each a multiple of 16; NULL with nseg == 1 means one module).  Each module
  * gets its own w_gs = amax(module)/2688, written to w_gs_out (HOST array of
  * nseg floats), and is quantised with it into the shared codes / scales
@@ -170,10 +178,13 @@ nvfp4_status nvfp4_quantize_weight_noalloc(const void* w_bf16, int64_t N, int64_
                                            nvfp4_stream_t stream);
 
 /* Block-scaled FP4 x FP4 GEMM (step a3) with a single module (step a4 with
- * op NONE): y[m, n] = fp32(a_gs * w_gs) * sum_k xhat[m,k] * what[n,k] / (a_gs w_gs),
- * i.e. the product of the dequantised operands, accumulated in fp32.
- * a_* describe the quantised activations [M, K], w_* the quantised weights
- * [N, K] (both K-major, y = x W^T).  Device pointers. */
+ * op NONE): y[m, n] = fp32(a_gs * w_gs) * sum_k e2m1(qa[m,k]) sa[m,k/16]
+ * e2m1(qw[n,k]) sw[n,k/16], accumulated in fp32 — the product of the
+ * dequantised operands (nefut abstract: W4A4 linear layers).  a_* describe
+ * the quantised activations [M, K], w_* the quantised weights [N, K] (both
+ * K-major, y = x W^T), y is bf16 (or fp32) [M, N] with row stride ldy.
+ * Caller-owned device pointers; y is overwritten, nothing else is written.
+ * Errors as for nvfp4_fused_linear. */
 nvfp4_status nvfp4_linear(const void* a_codes, const void* a_scales, float a_gs,
                           const void* w_codes, const void* w_scales, float w_gs,
                           int64_t M, int64_t N, int64_t K,
@@ -181,12 +192,21 @@ nvfp4_status nvfp4_linear(const void* a_codes, const void* a_scales, float a_gs,
                           nvfp4_stream_t stream);
 
 /* Fused multi-module projection (steps a3 + a4): one GEMM over the
- * concatenated weight [N, K]; the epilogue applies each module's own alpha
- * and op (the pages' global-scale mismatch repair, plus the optional GDN
- * gates).  segs: HOST array of nseg (1..NVFP4_MAX_SEGMENTS) entries, n_offset
+ * concatenated weight [N, K]; the epilogue applies each module's own alpha =
+ * fp32(a_gs * w_gs) — the repair of the global-scale mismatch of fused
+ * kernels (bayesiansapien wiki, "Two practical repairs"; aimodeling, "What
+ * engineers should actually take away") — and its op: none, beta =
+ * sigmoid(y), or g = -exp(A_log[h]) * softplus(y + dt_bias[h]) with h the
+ * column within the module (the GDN gates: wiki, mechanism study part 2).
+ * segs: HOST array of nseg (1..NVFP4_MAX_SEGMENTS) entries, n_offset
  * strictly ascending, first 0, each a multiple of 16 and < N; copied during
- * the call.  For M <= 64 the small-M weight-streaming kernel is used (step
- * a5), otherwise the persistent tensor-core kernel. */
+ * the call; a_log / dt_bias are device arrays of the module's width (decay
+ * modules only).  For M <= 64 the small-M weight-streaming kernel is used
+ * (step a5), otherwise the persistent tensor-core kernel.  Requires K % 64
+ * == 0, N % 16 == 0, 16-byte aligned pointers, ldy >= N (a multiple of 8
+ * bf16 / 4 fp32 elements); violations return before any launch.  The
+ * kernel is queued on `stream`; a bounded in-kernel wait that runs out is
+ * reported by nvfp4_last_device_error. */
 nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales,
                                 const void* w_codes, const void* w_scales,
                                 int64_t M, int64_t N, int64_t K,
