@@ -159,6 +159,12 @@ __global__ void __launch_bounds__(QUANT_THREADS) k_quantize(const __grid_constan
   const int64_t code_ld = a.K / 2;
   const uint64_t pol = policy_evict_first();
 
+  // With launch overlap this grid may start before the kernel ahead of it
+  // has finished: let the kernel behind it be scheduled, then wait before
+  // reading x or writing codes and scales.
+  griddep_launch_dependents();
+  griddep_wait();
+
   if (lane == 0) {
     for (int s = 0; s < QUANT_SLOTS; ++s) mbar_init(smem_addr(bars + s), 1);
     fence_mbar_init();
