@@ -146,7 +146,8 @@ nvfp4_status nvfp4_quantize_act(const void* x_bf16, int64_t M, int64_t K, int64_
  * nseg floats), and is quantised with it into the shared codes / scales
  * buffers (padding rows zeroed).  `workspace` is caller-owned DEVICE scratch
  * of nvfp4_quantize_weight_workspace_bytes(nseg) bytes (the per-module amax
- * reduction); its contents on entry do not matter.  Synchronises `stream`. */
+ * reduction); its contents on entry do not matter.  Synchronises `stream`
+ * and returns once the codes and scales are written. */
 size_t nvfp4_quantize_weight_workspace_bytes(int32_t nseg);
 nvfp4_status nvfp4_quantize_weight(const void* w_bf16, int64_t N, int64_t K, int64_t ldw,
                                    const int64_t* seg_offsets, int32_t nseg,
@@ -239,6 +240,21 @@ nvfp4_status nvfp4_last_device_error(nvfp4_stream_t stream, uint64_t* info);
  * automatically when the activation codes exceed 64 MB and the weight codes
  * are smaller).  Process-wide. */
 nvfp4_status nvfp4_set_gemm_path(int32_t path);
+
+/* Launch overlap (process-wide, off by default; on = 1, off = 0): the
+ * activation quantiser and the small-M GEMM (M <= 64) are launched with
+ * programmatic stream serialization, so that each may start while the
+ * kernel ahead of it on the stream is still running and the next call's
+ * weight stream overlaps this call's tail (the decode loop of consecutive
+ * layers).  The quantiser waits for the kernel ahead before it reads x or
+ * writes codes and scales.  The GEMM waits for it before it reads the
+ * activation codes and scales and before it writes y, but streams the
+ * weight codes and scales from its start: with overlap on, the kernel
+ * launched just ahead of a small-M GEMM on the same stream must not write
+ * that GEMM's weight codes or scales (weights quantised offline, or any
+ * other kernel in between, satisfy this).  Results are identical with
+ * overlap on or off. */
+nvfp4_status nvfp4_set_launch_overlap(int32_t on);
 
 /* Time limit of every bounded in-kernel wait, in nanoseconds (default 2e9;
  * also read once from the environment variable NVFP4_SPIN_LIMIT_NS). */

@@ -21,7 +21,7 @@ __all__ = [
     "nvfp4_codes_bytes", "nvfp4_scale_bytes", "nvfp4_global_scale", "nvfp4_amax",
     "nvfp4_quantize_act", "nvfp4_quantize_weight", "nvfp4_quantize_weight_noalloc",
     "nvfp4_linear", "nvfp4_fused_linear",
-    "nvfp4_silu_mul", "nvfp4_last_device_error", "nvfp4_set_gemm_path",
+    "nvfp4_silu_mul", "nvfp4_last_device_error", "nvfp4_set_gemm_path", "nvfp4_set_launch_overlap",
     "nvfp4_set_wait_limit_ns", "nvfp4_test_e2m1", "nvfp4_test_e4m3", "nvfp4_test_wait_timeout",
     "SegmentSpec", "NVFP4Error", "OP_NONE", "OP_SIGMOID", "OP_GDN_DECAY",
 ]
@@ -184,6 +184,10 @@ def nvfp4_last_device_error(stream=None) -> Tuple[int, int]:
 
 def nvfp4_set_gemm_path(path: int) -> None:
     check(load().nvfp4_set_gemm_path(path), "nvfp4_set_gemm_path")
+
+
+def nvfp4_set_launch_overlap(on: bool) -> None:
+    check(load().nvfp4_set_launch_overlap(1 if on else 0), "nvfp4_set_launch_overlap")
 
 
 def nvfp4_set_wait_limit_ns(limit_ns: int) -> None:

@@ -47,6 +47,7 @@ SIGNATURES = {
     "nvfp4_status_string": (ctypes.c_char_p, [_st]),
     "nvfp4_last_device_error": (_st, [_vp, ctypes.POINTER(ctypes.c_uint64)]),
     "nvfp4_set_gemm_path": (_st, [_i32]),
+    "nvfp4_set_launch_overlap": (_st, [_i32]),
     "nvfp4_set_wait_limit_ns": (_st, [_u64]),
     "nvfp4_test_e2m1": (_st, [_vp, _vp, _i64, _vp]),
     "nvfp4_test_e4m3": (_st, [_vp, _vp, _i64, _vp]),

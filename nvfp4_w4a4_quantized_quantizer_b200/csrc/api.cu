@@ -34,6 +34,34 @@ uint64_t read_env_wait_ns() {
 
 uint64_t g_wait_ns = read_env_wait_ns();
 int g_gemm_path = 0;
+bool g_overlap = false;
+
+// Launch with programmatic stream serialization when launch overlap is on:
+// the kernel may then start before the kernel ahead of it on the stream has
+// finished (it waits for it with griddepcontrol.wait where it must).
+template <typename Kernel, typename... Args>
+nvfp4_status launch_maybe_overlapped(Kernel kernel, dim3 grid, dim3 block, int smem,
+                                     cudaStream_t st, Args... args) {
+  if (!g_overlap) {
+    kernel<<<grid, block, smem, st>>>(args...);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, args...) != cudaSuccess) {
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+  }
+  return NVFP4_OK;
+}
 
 // ----------------------------------------------------------- device info
 constexpr int MAX_DEVICES = 64;
@@ -259,8 +287,8 @@ nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t K, int64_t ld,
   }
   // persistent: one wave of resident blocks, each warp striding over the units
   const int grid = grid_for(units, nvfp4::QUANT_WARPS, info->sms * info->quant_blocks);
-  nvfp4::k_quantize<<<grid, nvfp4::QUANT_THREADS, smem, st>>>(a);
-  return check_launch();
+  return launch_maybe_overlapped(nvfp4::k_quantize, dim3(grid), dim3(nvfp4::QUANT_THREADS), smem,
+                                 st, a);
 }
 
 nvfp4_status launch_amax(const void* x, int64_t rows, int64_t K, int64_t ld, float* out, int sms,
@@ -366,6 +394,12 @@ nvfp4_status nvfp4_set_gemm_path(int32_t path) {
   return NVFP4_OK;
 }
 
+nvfp4_status nvfp4_set_launch_overlap(int32_t on) {
+  if (on != 0 && on != 1) return NVFP4_ERR_INVALID_ARG;
+  g_overlap = (on == 1);
+  return NVFP4_OK;
+}
+
 nvfp4_status nvfp4_set_wait_limit_ns(uint64_t limit_ns) {
   if (limit_ns == 0) return NVFP4_ERR_INVALID_ARG;
   g_wait_ns = limit_ns;
@@ -466,6 +500,12 @@ nvfp4_status nvfp4_quantize_weight(const void* w, int64_t N, int64_t K, int64_t 
                          scales, last ? N : 0, last ? pad128(N) : 0, info, cs);
     if (st != NVFP4_OK) return st;
   }
+  // the codes and scales are complete on return, so that a GEMM launched
+  // with launch overlap may stream them from its start
+  if (cudaStreamSynchronize(cs) != cudaSuccess) {
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+  }
   return NVFP4_OK;
 }
 
@@ -549,8 +589,8 @@ nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales, const
           return NVFP4_ERR_CUDA;
         info->attr_small[which] = true;
       }
-      kernel<<<grid, nvfp4::sm::THREADS, smem, cs>>>(tw, tx, g, table);
-      return check_launch();
+      return launch_maybe_overlapped(kernel, dim3(grid), dim3(nvfp4::sm::THREADS), smem, cs, tw,
+                                     tx, g, table);
     };
     if (nt == 16) return launch(nvfp4::k_gemm_small<16>, nvfp4::sm::Cfg<16>::SMEM_BYTES);
     if (nt == 32) return launch(nvfp4::k_gemm_small<32>, nvfp4::sm::Cfg<32>::SMEM_BYTES);

@@ -527,7 +527,6 @@ constexpr int BW = 128;                 // weight rows per CTA (MMA M)
 constexpr int DIRECT_M = 8;             // up to this many tokens the epilogue stores directly
 constexpr int BK = 256;
 constexpr int BKB = BK / 2;
-constexpr int STAGES = 6;
 constexpr int W_BYTES = BW * BKB;       // 16 KB
 constexpr int SFW_BYTES = 4 * 512;
 constexpr int SFX_BYTES = 4 * 512;
@@ -540,24 +539,33 @@ constexpr uint32_t ACC_COL = 0;         // NT columns
 constexpr uint32_t SF_COL = 64;         // + 32 * stage
 constexpr uint32_t SF_STRIDE = 32;
 constexpr int BAR_BYTES = 256;
-static_assert(SF_COL + STAGES * SF_STRIDE <= TMEM_COLS, "TMEM budget");
+// Two CTAs fit on one SM (shared memory, 256 TMEM columns and <= 80
+// registers per thread each), so that with launch overlap the next call's
+// CTAs start streaming their weights beside this call's.
+constexpr int SMEM_PER_SM = 233472;     // 228 KB
+constexpr int SMEM_RESERVED = 1024;     // per CTA
 template <int NT>
 struct Cfg {
   static constexpr int X_BYTES = NT * BKB;   // NT rows x 128 bytes
   static constexpr int STAGE_BYTES = W_BYTES + X_BYTES + SFW_BYTES + SFX_BYTES;
+  static constexpr int STAGES = NT <= 16 ? 5 : (NT <= 32 ? 4 : 3);   // 22 / 24 / 28 KB stages
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
+  static_assert(SF_COL + STAGES * SF_STRIDE <= TMEM_COLS, "TMEM budget");
+  static_assert(2 * (SMEM_BYTES + SMEM_RESERVED) <= SMEM_PER_SM, "two CTAs per SM");
+  static_assert(NT * BW * 4 <= STAGES * STAGE_BYTES, "the epilogue's transpose fits the ring");
 };
 }  // namespace sm
 
 // tmW: weight codes [N, K/2]; tmX: token codes [M, K/2].  D (TMEM) is
 // [128 weight rows] x [NT tokens]; y[token, n] is written transposed back.
 template <int NT>
-__global__ void __launch_bounds__(sm::THREADS, 1)
+__global__ void __launch_bounds__(sm::THREADS, 2)
     k_gemm_small(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                  const GemmArgs g, const __grid_constant__ SegTable seg) {
   using namespace sm;
   using C = Cfg<NT>;
+  constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -599,11 +607,17 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // With launch overlap the next kernel may now be scheduled beside this one.
+  // Only the weight stream starts before the kernel ahead has finished: the
+  // token producer and the epilogue wait for it (griddep_wait) before they
+  // read the token operands or write y.
+  griddep_launch_dependents();
 
   if (warp == 0 || warp == 2) {
     // warp-wide loop; one elected lane issues each copy
     {
       const bool is_w = (warp == 0);
+      if (!is_w) griddep_wait();   // the token operands may come from the kernel ahead
       // weights stream through once; tokens are re-read by every CTA
       const uint64_t pol = is_w ? policy_evict_first() : policy_evict_last();
       int stage = 0;
@@ -723,6 +737,7 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
     // every MMA has completed) so that each token's 128 columns leave as
     // 16-byte stores of one contiguous segment instead of M strided 2-byte
     // stores per thread.
+    griddep_wait();   // y may still be read or written by the kernel ahead
     const bool ok = mbar_wait(acc_full, 0, g.wait_ns, abort_flag);
     if (ok) {
       tc_fence_after();

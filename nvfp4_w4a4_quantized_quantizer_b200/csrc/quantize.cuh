@@ -177,6 +177,12 @@ __global__ void __launch_bounds__(QUANT_THREADS) k_quantize(const __grid_constan
   const int64_t step_rows = nwarps / per_row;
   const int step_cols = static_cast<int>(nwarps - step_rows * per_row);
 
+  // With launch overlap this grid may start before the kernel ahead of it
+  // has finished: let the kernel behind it be scheduled, then wait before
+  // reading x or writing codes and scales.
+  griddep_launch_dependents();
+  griddep_wait();
+
   if (lane == 0) {
     for (int s = 0; s < QUANT_SLOTS; ++s) mbar_init(smem_addr(bars + s), 1);
     fence_mbar_init();

@@ -125,7 +125,12 @@ def test_gdn_inproj_full():
 
 @pytest.mark.parametrize("M", [1, 8, 32, 64])
 def test_decode_sweep_full(M):
-    _check_layer(workloads.WORKLOADS[5], M, M, 256, seed=50 + M)
+    # with launch overlap, as bench.py runs the decode workload
+    nv.nvfp4_set_launch_overlap(True)
+    try:
+        _check_layer(workloads.WORKLOADS[5], M, M, 256, seed=50 + M)
+    finally:
+        nv.nvfp4_set_launch_overlap(False)
 
 
 def test_mlp_pair_full():

@@ -201,3 +201,71 @@ def test_bf16_row_stride_both_store_widths(ldy, path):
     out = y.float().cpu().numpy()
     assert np.all(out[:, N:] == 3.0)
     np.testing.assert_array_equal(out[:, :N], H.bf16_round(y32.cpu().numpy()))
+
+
+# ------------------------------------------------------------ launch overlap
+@pytest.fixture
+def overlap():
+    nv.nvfp4_set_launch_overlap(True)
+    yield
+    nv.nvfp4_set_launch_overlap(False)
+
+
+def _decode_layer(M, N, K, seed):
+    xb = workloads.random_bf16((M, K), seed=seed, std=1.0)
+    wb = workloads.random_bf16((N, K), seed=seed + 1, std=1 / np.sqrt(K))
+    a_gs = float(oracle.global_scale(np.abs(H.f32(xb)).max()))
+    wc, ws, (w_gs,) = nv.nvfp4_quantize_weight(H.bf16_dev(wb))
+    return xb, wb, a_gs, wc, ws, w_gs
+
+
+@pytest.mark.parametrize("M", [1, 8, 17, 40, 64])
+def test_overlap_gives_identical_results(M, overlap):
+    """quantise + small-M GEMM chains with launch overlap on equal the plain launches bit for bit."""
+    N, K = 1040, 2048
+    xb, _, a_gs, wc, ws, w_gs = _decode_layer(M, N, K, seed=M)
+    nv.nvfp4_set_launch_overlap(False)
+    ac, as_ = nv.nvfp4_quantize_act(H.bf16_dev(xb), a_gs)
+    ref = nv.nvfp4_linear(ac, as_, a_gs, wc, ws, w_gs, M, N, K, out_dtype=nv.OUT_FP32).cpu()
+    nv.nvfp4_set_launch_overlap(True)
+    x = H.bf16_dev(xb)
+    for _ in range(3):
+        ac2, as2 = nv.nvfp4_quantize_act(x, a_gs)
+        y = nv.nvfp4_linear(ac2, as2, a_gs, wc, ws, w_gs, M, N, K, out_dtype=nv.OUT_FP32)
+        assert torch.equal(y.cpu(), ref)
+        assert torch.equal(ac2.cpu(), ac.cpu()) and torch.equal(as2.cpu(), as_.cpu())
+    assert nv.nvfp4_last_device_error()[0] == 0
+
+
+def test_overlap_keeps_stream_order_of_shared_buffers(overlap):
+    """Consecutive layers sharing one code buffer and one output buffer: the
+    quantiser of layer i+1 must not overwrite the codes layer i's GEMM still
+    reads, and each GEMM must read the codes just written (read-after-write,
+    write-after-read and write-after-write through the same buffers)."""
+    M, N, K = 16, 2064, 1024
+    layers = [_decode_layer(M, N, K, seed=100 + 7 * i) for i in range(4)]
+    nv.nvfp4_set_launch_overlap(False)
+    expect = []
+    for xb, _, a_gs, wc, ws, w_gs in layers:
+        ac, as_ = nv.nvfp4_quantize_act(H.bf16_dev(xb), a_gs)
+        expect.append(nv.nvfp4_linear(ac, as_, a_gs, wc, ws, w_gs, M, N, K, out_dtype=nv.OUT_FP32).cpu())
+    nv.nvfp4_set_launch_overlap(True)
+    xs = [H.bf16_dev(l[0]) for l in layers]
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+    scales = torch.empty(nv.nvfp4_scale_bytes(M, K), dtype=torch.uint8, device="cuda")
+    outs = [torch.empty((M, N), dtype=torch.float32, device="cuda") for _ in layers]
+    y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    for rep in range(5):
+        # one code buffer, back-to-back quantise / GEMM launches
+        for i, (_, _, a_gs, wc, ws, w_gs) in enumerate(layers):
+            nv.nvfp4_quantize_act(xs[i], a_gs, codes=codes, scales=scales)
+            nv.nvfp4_linear(codes, scales, a_gs, wc, ws, w_gs, M, N, K, y=outs[i],
+                            out_dtype=nv.OUT_FP32)
+        for i in range(len(layers)):
+            assert torch.equal(outs[i].cpu(), expect[i]), (rep, i)
+        # one output buffer: the last GEMM's result stays
+        for i, (_, _, a_gs, wc, ws, w_gs) in enumerate(layers):
+            nv.nvfp4_quantize_act(xs[i], a_gs, codes=codes, scales=scales)
+            nv.nvfp4_linear(codes, scales, a_gs, wc, ws, w_gs, M, N, K, y=y, out_dtype=nv.OUT_FP32)
+        assert torch.equal(y.cpu(), expect[-1]), rep
+    assert nv.nvfp4_last_device_error()[0] == 0
