@@ -222,6 +222,8 @@ class Layer:
         self.scales = [torch.empty(nv.nvfp4_scale_bytes(M, self.K), dtype=torch.uint8, device=device)
                        for _ in range(2)]
         self.ys = [torch.empty((M, self.N), dtype=torch.bfloat16, device=device) for _ in range(2)]
+        # lets the CTA-pair GEMM split its last partial wave of tiles along K
+        self.work = nv.nvfp4_gemm_workspace(device)
         self.segs = []
         gate_dev = {}
         if any(s.op == "gdn_decay" for s in wl.segments):
@@ -241,7 +243,8 @@ class Layer:
     def gemm(self, i, stream):
         wc, ws = self.ws[i % len(self.ws)]
         self.nv.nvfp4_fused_linear(self.codes[i % 2], self.scales[i % 2], wc, ws, self.M, self.N,
-                                   self.K, self.segs, y=self.ys[i % 2], stream=stream)
+                                   self.K, self.segs, y=self.ys[i % 2], stream=stream,
+                                   workspace=self.work)
 
     @property
     def flops(self):
@@ -277,11 +280,13 @@ class MlpChain:
         w2c, w2s, (self.w2_gs,) = nv.nvfp4_quantize_weight(w2bits)
         del w2bits
         self.segs = [nv.SegmentSpec(off, g, self.a_gs) for off, g in zip(wl.seg_offsets, self.w_gs)]
+        self.work = nv.nvfp4_gemm_workspace(device)
         # the down input's static global scale: the chain on the calibration batch
         cc, cs = nv.nvfp4_quantize_act(calib, self.a_gs)
         gu_cal = nv.nvfp4_fused_linear(cc, cs, wc, ws, calib.shape[0], self.N, self.K, self.segs)
         h_cal = nv.nvfp4_silu_mul(gu_cal, self.H)
         self.a2_gs = nv.nvfp4_global_scale(nv.nvfp4_amax(h_cal).item())
+        self.segs2 = [nv.SegmentSpec(0, self.w2_gs, self.a2_gs)]
         del calib, cc, cs, gu_cal, h_cal
         self.ws = [(wc, ws, w2c, w2s)] + [tuple(t.clone() for t in (wc, ws, w2c, w2s))
                                           for _ in range(rotate_w - 1)]
@@ -301,7 +306,7 @@ class MlpChain:
     def gate_up(self, i, stream):
         wc, ws, _, _ = self.ws[i % len(self.ws)]
         self.nv.nvfp4_fused_linear(self.xc, self.xsc, wc, ws, self.M, self.N, self.K, self.segs,
-                                   y=self.gu, stream=stream)
+                                   y=self.gu, stream=stream, workspace=self.work)
 
     def silu(self, i, stream):
         self.nv.nvfp4_silu_mul(self.gu, self.H, h=self.h, stream=stream)
@@ -311,8 +316,8 @@ class MlpChain:
 
     def down(self, i, stream):
         _, _, w2c, w2s = self.ws[i % len(self.ws)]
-        self.nv.nvfp4_linear(self.hc, self.hsc, self.a2_gs, w2c, w2s, self.w2_gs, self.M, self.N2,
-                             self.H, y=self.y, stream=stream)
+        self.nv.nvfp4_fused_linear(self.hc, self.hsc, w2c, w2s, self.M, self.N2, self.H, self.segs2,
+                                   y=self.y, stream=stream, workspace=self.work)
 
     def gemm(self, i, stream):
         """Everything after the first quantisation."""

@@ -215,6 +215,39 @@ nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales,
                                 void* y, int64_t ldy, nvfp4_out_dtype out_dtype,
                                 nvfp4_stream_t stream);
 
+/* Workspace of nvfp4_fused_linear_ws: NVFP4_GEMM_WS_COUNTER_BYTES of
+ * arrival counters followed by one 256 KB fp32 partial tile per K-part. */
+#define NVFP4_GEMM_WS_COUNTER_BYTES 4096
+#define NVFP4_GEMM_WS_MAX_UNITS 128
+
+/* Bytes of a workspace that never limits the split of
+ * nvfp4_fused_linear_ws (NVFP4_GEMM_WS_COUNTER_BYTES + 128 partial tiles,
+ * about 32 MB).  Any device. */
+size_t nvfp4_gemm_workspace_bytes(void);
+
+/* nvfp4_fused_linear with a caller-owned device workspace that lets the
+ * CTA-pair kernel balance its last, partial wave of tiles: each tile of that
+ * wave is computed as up to 4 K-parts by pairs that would otherwise idle;
+ * each part writes an fp32 partial tile to the workspace and the last part
+ * to arrive sums the parts in part order (the same order whichever arrives
+ * last, so results do not depend on timing) and applies the epilogue.  The
+ * sum differs from the unsplit kernel's by fp32 rounding only.
+ * workspace: 16-byte aligned; its first NVFP4_GEMM_WS_COUNTER_BYTES must be
+ * zero before its first use (every call leaves them zero, also after a
+ * bounded wait ran out); it must not be in use by another call that may run
+ * at the same time.  workspace_bytes below nvfp4_gemm_workspace_bytes()
+ * limits the number of parts; NULL (or too small for two parts) runs the
+ * last wave as whole tiles, exactly like nvfp4_fused_linear.  Other
+ * arguments, layouts and errors as for nvfp4_fused_linear; an unaligned
+ * workspace returns NVFP4_ERR_ALIGNMENT. */
+nvfp4_status nvfp4_fused_linear_ws(const void* a_codes, const void* a_scales,
+                                   const void* w_codes, const void* w_scales,
+                                   int64_t M, int64_t N, int64_t K,
+                                   const nvfp4_segment* segs, int32_t nseg,
+                                   void* y, int64_t ldy, nvfp4_out_dtype out_dtype,
+                                   void* workspace, size_t workspace_bytes,
+                                   nvfp4_stream_t stream);
+
 /* MLP glue between the two projections of the MLP pair (not an NVFP4 step):
  * h[m, j] = bf16(silu(gu[m, j]) * gu[m, H + j]) for j < H, computed in fp32.
  * gu: bf16 [M, ld_in] with ld_in >= 2H; h: bf16 [M, ld_out], ld_out >= H.

@@ -20,7 +20,7 @@ from ._lib import (NVFP4Error, OP_GDN_DECAY, OP_NONE, OP_SIGMOID, OUT_BF16, OUT_
 __all__ = [
     "nvfp4_codes_bytes", "nvfp4_scale_bytes", "nvfp4_global_scale", "nvfp4_amax",
     "nvfp4_quantize_act", "nvfp4_quantize_weight", "nvfp4_quantize_weight_noalloc",
-    "nvfp4_linear", "nvfp4_fused_linear",
+    "nvfp4_linear", "nvfp4_fused_linear", "nvfp4_gemm_workspace_bytes", "nvfp4_gemm_workspace",
     "nvfp4_silu_mul", "nvfp4_last_device_error", "nvfp4_set_gemm_path", "nvfp4_set_launch_overlap",
     "nvfp4_set_wait_limit_ns", "nvfp4_test_e2m1", "nvfp4_test_e4m3", "nvfp4_test_wait_timeout",
     "SegmentSpec", "NVFP4Error", "OP_NONE", "OP_SIGMOID", "OP_GDN_DECAY",
@@ -155,14 +155,33 @@ def nvfp4_linear(a_codes, a_scales, a_gs: float, w_codes, w_scales, w_gs: float,
     return y
 
 
+def nvfp4_gemm_workspace_bytes() -> int:
+    return load().nvfp4_gemm_workspace_bytes()
+
+
+def nvfp4_gemm_workspace(device=None) -> torch.Tensor:
+    """A zeroed workspace of nvfp4_gemm_workspace_bytes() for nvfp4_fused_linear."""
+    return torch.zeros(nvfp4_gemm_workspace_bytes(), dtype=torch.uint8, device=device)
+
+
 def nvfp4_fused_linear(a_codes, a_scales, w_codes, w_scales, M: int, N: int, K: int,
                        segments: Sequence[SegmentSpec], y: Optional[torch.Tensor] = None,
-                       out_dtype: int = OUT_BF16, stream=None) -> torch.Tensor:
+                       out_dtype: int = OUT_BF16, stream=None,
+                       workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """With `workspace` (see nvfp4_gemm_workspace) the call is
+    nvfp4_fused_linear_ws, which splits the last partial wave along K."""
     y = _out(y, M, N, out_dtype, a_codes.device)
     segs = (Segment * len(segments))(*[s.c() for s in segments])
-    check(load().nvfp4_fused_linear(_ptr(a_codes), _ptr(a_scales), _ptr(w_codes), _ptr(w_scales),
-                                    M, N, K, segs, len(segments), _ptr(y), _ld(y), out_dtype,
-                                    _stream(stream)), "nvfp4_fused_linear")
+    if workspace is None:
+        check(load().nvfp4_fused_linear(_ptr(a_codes), _ptr(a_scales), _ptr(w_codes),
+                                        _ptr(w_scales), M, N, K, segs, len(segments), _ptr(y),
+                                        _ld(y), out_dtype, _stream(stream)), "nvfp4_fused_linear")
+    else:
+        check(load().nvfp4_fused_linear_ws(_ptr(a_codes), _ptr(a_scales), _ptr(w_codes),
+                                           _ptr(w_scales), M, N, K, segs, len(segments), _ptr(y),
+                                           _ld(y), out_dtype, _ptr(workspace),
+                                           workspace.numel() * workspace.element_size(),
+                                           _stream(stream)), "nvfp4_fused_linear_ws")
     return y
 
 

@@ -227,6 +227,10 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 constexpr int64_t kMaxDim = (1ll << 31) - 1;
 
+// One K-part's fp32 partial tile: 2 CTAs x 128 rows x 256 columns.
+constexpr size_t kPartialBytes = 2ull * nvfp4::tc::BM * nvfp4::tc::BN * 4;
+constexpr int64_t kMaxSplit = 4;
+
 nvfp4_status check_bf16_matrix(const void* x, int64_t R, int64_t K, int64_t ld) {
   if (x == nullptr) return NVFP4_ERR_INVALID_ARG;
   if (R < 0 || K < 64 || K % 64 != 0 || R > kMaxDim || K > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -527,13 +531,20 @@ nvfp4_status nvfp4_quantize_weight_noalloc(const void* w, int64_t N, int64_t K, 
                                stream);
 }
 
-nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales, const void* w_codes,
-                                const void* w_scales, int64_t M, int64_t N, int64_t K,
-                                const nvfp4_segment* segs, int32_t nseg, void* y, int64_t ldy,
-                                nvfp4_out_dtype out_dtype, nvfp4_stream_t stream) {
+size_t nvfp4_gemm_workspace_bytes(void) {
+  return static_cast<size_t>(NVFP4_GEMM_WS_COUNTER_BYTES) +
+         static_cast<size_t>(NVFP4_GEMM_WS_MAX_UNITS) * kPartialBytes;
+}
+
+nvfp4_status nvfp4_fused_linear_ws(const void* a_codes, const void* a_scales, const void* w_codes,
+                                   const void* w_scales, int64_t M, int64_t N, int64_t K,
+                                   const nvfp4_segment* segs, int32_t nseg, void* y, int64_t ldy,
+                                   nvfp4_out_dtype out_dtype, void* workspace,
+                                   size_t workspace_bytes, nvfp4_stream_t stream) {
   if (a_codes == nullptr || a_scales == nullptr || w_codes == nullptr || w_scales == nullptr ||
       y == nullptr)
     return NVFP4_ERR_INVALID_ARG;
+  if (workspace != nullptr && !aligned16(workspace)) return NVFP4_ERR_ALIGNMENT;
   if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_FP32) return NVFP4_ERR_INVALID_ARG;
   if (M < 0 || M > kMaxDim || N < 16 || N % 16 != 0 || N > kMaxDim || K < 64 || K % 64 != 0 ||
       K > kMaxDim || ldy < N)
@@ -564,6 +575,11 @@ nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales, const
   g.sector_stores = ((reinterpret_cast<uintptr_t>(y) & 31u) == 0) &&
                     ((ldy * (g.out_fp32 ? 4 : 2)) % 32 == 0);
   g.wait_ns = g_wait_ns;
+  g.full_tiles = 0;
+  g.split = 1;
+  g.split_units = 0;
+  g.partial = nullptr;
+  g.counters = nullptr;
   // Tile raster.  Consecutive CTAs (pairs) run tiles that share one operand
   // tile, and the rest of that operand is re-read from L2 for each of the
   // other operand's tiles.  By default they share weight tiles (M fastest),
@@ -649,11 +665,43 @@ nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales, const
   const int64_t tiles = ((M + 2 * nvfp4::tc::BM - 1) / (2 * nvfp4::tc::BM)) * num_n;
   const int pairs = static_cast<int>(tiles < info->pairs ? tiles : info->pairs);
   cfg.gridDim = dim3(2 * pairs, 1, 1);
+  // Last partial wave: when the tiles are not a multiple of the pairs, each
+  // tile of the last wave is split into S K-parts run by otherwise idle
+  // pairs (S = pairs / leftover tiles, at most 4, at most the k-tiles and
+  // within the workspace); the parts meet in the caller's workspace.
+  if (workspace != nullptr && tiles > pairs) {
+    const int64_t num_kt = (K + nvfp4::tc::BK - 1) / nvfp4::tc::BK;
+    const int64_t left = tiles % pairs;
+    const int64_t max_units =
+        workspace_bytes > NVFP4_GEMM_WS_COUNTER_BYTES
+            ? static_cast<int64_t>((workspace_bytes - NVFP4_GEMM_WS_COUNTER_BYTES) / kPartialBytes)
+            : 0;
+    int64_t S = left > 0 ? pairs / left : 0;
+    if (S > kMaxSplit) S = kMaxSplit;
+    if (S > num_kt) S = num_kt;
+    while (S >= 2 && left * S > max_units) --S;
+    if (S >= 2 && left * 2 * 4 <= NVFP4_GEMM_WS_COUNTER_BYTES) {
+      g.full_tiles = static_cast<int>(tiles - left);
+      g.split = static_cast<int>(S);
+      g.split_units = static_cast<int>(left * S);
+      g.counters = static_cast<unsigned*>(workspace);
+      g.partial = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                           NVFP4_GEMM_WS_COUNTER_BYTES);
+    }
+  }
   if (cudaLaunchKernelEx(&cfg, nvfp4::k_gemm_tc<2>, ta, tb, tsa, tsb, g, table) != cudaSuccess) {
     cudaGetLastError();
     return NVFP4_ERR_CUDA;
   }
   return check_launch();
+}
+
+nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales, const void* w_codes,
+                                const void* w_scales, int64_t M, int64_t N, int64_t K,
+                                const nvfp4_segment* segs, int32_t nseg, void* y, int64_t ldy,
+                                nvfp4_out_dtype out_dtype, nvfp4_stream_t stream) {
+  return nvfp4_fused_linear_ws(a_codes, a_scales, w_codes, w_scales, M, N, K, segs, nseg, y, ldy,
+                               out_dtype, nullptr, 0, stream);
 }
 
 nvfp4_status nvfp4_linear(const void* a_codes, const void* a_scales, float a_gs,

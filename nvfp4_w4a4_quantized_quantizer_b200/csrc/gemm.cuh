@@ -59,6 +59,18 @@ struct GemmArgs {
   int sector_stores;   // y base 32-byte aligned and rows a multiple of 32 bytes
   int n_fastest;       // tile raster: 0 = M fastest (consecutive CTAs share a weight tile),
                        // 1 = N fastest (they share an activation tile)
+  // Last-wave K split (CTA-pair kernel): tiles [full_tiles, num_tiles) are each
+  // computed as `split` K-parts by split_units = (num_tiles - full_tiles) * split
+  // units; unit u (u < split_units) takes part u % split of tile
+  // full_tiles + u / split after its whole tiles.  split <= 1: no split.
+  // The parts meet in a caller-owned workspace: one arrival counter per
+  // (split tile, CTA of the pair), all zero between launches (the last part
+  // wraps its counter back to 0), and one fp32 partial tile per unit.
+  int full_tiles;
+  int split;
+  int split_units;
+  float* partial;      // [split_units][2 CTAs][2 halves][32 chunks][128 rows] float4
+  unsigned* counters;  // [num_tiles - full_tiles][2 CTAs]
   uint64_t wait_ns;
 };
 
@@ -137,6 +149,44 @@ __device__ __forceinline__ int seg_advance(const SegTable& t, int seg, int n) {
 // Tiles are walked M fastest (consecutive CTAs share a weight tile and the
 // activations stay in L2) or, when GemmArgs::n_fastest is set, N fastest
 // (they share an activation tile: for activations too large for the L2).
+// One unit of work of a CTA (pair): a whole tile (part < 0) or one K-part of
+// a tile of the last partial wave.
+struct WorkItem {
+  int tile;
+  int kt0, kt1;   // k-tiles [kt0, kt1)
+  int part;
+};
+
+__device__ __forceinline__ int work_full(const GemmArgs& g, int num_tiles) {
+  return g.split > 1 ? g.full_tiles : num_tiles;
+}
+
+__device__ __forceinline__ int work_count(const GemmArgs& g, int unit, int units, int num_tiles) {
+  const int full = work_full(g, num_tiles);
+  int n = unit < full ? (full - 1 - unit) / units + 1 : 0;
+  if (g.split > 1 && unit < g.split_units) ++n;
+  return n;
+}
+
+__device__ __forceinline__ WorkItem work_item(const GemmArgs& g, int unit, int units,
+                                              int num_tiles, int num_kt, int i) {
+  const int full = work_full(g, num_tiles);
+  const int nfull = unit < full ? (full - 1 - unit) / units + 1 : 0;
+  WorkItem w;
+  if (i < nfull) {
+    w.tile = unit + i * units;
+    w.kt0 = 0;
+    w.kt1 = num_kt;
+    w.part = -1;
+  } else {
+    w.tile = full + unit / g.split;
+    w.part = unit % g.split;
+    w.kt0 = w.part * num_kt / g.split;
+    w.kt1 = (w.part + 1) * num_kt / g.split;
+  }
+  return w;
+}
+
 namespace tc {
 constexpr int BM = 128;                 // rows of A per CTA
 constexpr int BN = 256;                 // tile columns (MMA N)
@@ -205,6 +255,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
   const int num_n = (g.N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
   const int num_kt = (g.K + BK - 1) / BK;
+  const int n_items = work_count(g, unit, units, num_tiles);
 
   auto full_bar = [&](int s) { return smem_addr(bars + s); };
   auto empty_bar = [&](int s) { return smem_addr(bars + STAGES + s); };
@@ -273,12 +324,14 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       uint32_t phase = 0;
       int64_t issued = 0;
       bool ok = true;
-      for (int tile = unit; tile < num_tiles && ok; tile += units) {
+      for (int it = 0; it < n_items && ok; ++it) {
+        const WorkItem w = work_item(g, unit, units, num_tiles, num_kt, it);
+        const int tile = w.tile;
         const int mb = g.n_fastest ? tile / num_n : tile % num_m;
         const int nb = g.n_fastest ? tile % num_n : tile / num_m;
         const int arow = (mb * CG + static_cast<int>(rank)) * BM;
         const int brow = nb * BN + static_cast<int>(rank) * C::B_ROWS;
-        for (int kt = 0; kt < num_kt; ++kt) {
+        for (int kt = w.kt0; kt < w.kt1; ++kt) {
           if (!wait_pair(empty_bar(stage), phase ^ 1u)) {
             raise_abort(SITE_PRODUCER_EMPTY, warp);
             ok = false;
@@ -323,9 +376,10 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     int stage = 0;
     uint32_t phase = 0;
-    for (int tile = unit; tile < num_tiles; tile += units) {
+    for (int it = 0; it < n_items; ++it) {
+      const WorkItem w = work_item(g, unit, units, num_tiles, num_kt, it);
       bool ok = true;
-      for (int kt = 0; kt < num_kt; ++kt) {
+      for (int kt = w.kt0; kt < w.kt1; ++kt) {
         if (!mbar_wait(sfull_bar(stage), phase, g.wait_ns, abort_flag)) {
           raise_abort(SITE_MMA_FULL, warp);
           ok = false;
@@ -391,14 +445,15 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
-      for (int tile = unit; tile < num_tiles && ok; tile += units, ++local) {
+      for (int it = 0; it < n_items && ok; ++it, ++local) {
+        const WorkItem w = work_item(g, unit, units, num_tiles, num_kt, it);
         if (!wait_pair(tmem_empty, static_cast<uint32_t>((local & 1) ^ 1))) {
           raise_abort(SITE_MMA_TMEM_EMPTY, 1);
           break;
         }
         tc_fence_after();
         int prev = -1;
-        for (int kt = 0; kt < num_kt; ++kt) {
+        for (int kt = w.kt0; kt < w.kt1; ++kt) {
           if (!wait_pair(sf_bar(stage), phase)) {
             raise_abort(SITE_MMA_FULL, 1);
             ok = false;
@@ -410,7 +465,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
           const uint64_t ad = adesc0 + soff, bd = bdesc0 + soff;
           const uint32_t col = tmem_base + SF_COL + SF_STRIDE * stage;
           // K = 64 fp4 = 32 bytes per MMA: advance the start address inside the swizzle atom
-          mma_mxf4nvf4_warp<CG>(tmem_base + ACC_COL, ad, bd, idesc, col, col + 16, kt != 0);
+          mma_mxf4nvf4_warp<CG>(tmem_base + ACC_COL, ad, bd, idesc, col, col + 16, kt != w.kt0);
           if (prev >= 0) tc_commit_all_warp<CG>(empty_bar(prev));
           for (int kk = 1; kk < nk; ++kk)
             mma_mxf4nvf4_warp<CG>(tmem_base + ACC_COL, ad + 2 * kk, bd + 2 * kk, idesc,
@@ -436,69 +491,151 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     const int q = warp & 3;                       // TMEM lane quarter this warp may access
     const int half = (warp - EPI_WARP0) >> 2;     // columns [128*half, 128*half + 128)
     const int row_in_tile = q * 32 + lane;
-    int local = 0;
-    for (int tile = unit; tile < num_tiles; tile += units, ++local) {
-      const int mb = g.n_fastest ? tile / num_n : tile % num_m;
-      const int nb = g.n_fastest ? tile % num_n : tile / num_m;
-      if (!wait_pair(tmem_full, static_cast<uint32_t>(local & 1))) {
-        raise_abort(SITE_EPI_TMEM_FULL, warp);
-        break;
-      }
-      tc_fence_after();
-      uint32_t v[128];
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ACC_COL + half * 128;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld_x32(taddr + c * 32, v + c * 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) arrive_leader(tmem_empty);
-
+    // The output of one tile row: alpha / op, bf16 RNE (or fp32), store.
+    // fetch(grp, a) yields the fp32 accumulator bits of columns
+    // 16 grp .. 16 grp + 15 of this thread's 128.
+    // Rows past M skip only the stores: fetch may issue warp-collective
+    // TMEM loads, so every lane of the warp runs it.
+    auto store_row = [&](int mb, int nb, auto&& fetch) {
       const int64_t gm = static_cast<int64_t>(mb * CG + static_cast<int>(rank)) * BM + row_in_tile;
-      if (gm < g.M) {
-        const int n0 = nb * BN + half * 128;
-        int s = seg_advance(seg, 0, n0);
+      const bool row_live = gm < g.M;
+      const int n0 = nb * BN + half * 128;
+      int s = seg_advance(seg, 0, n0);
 #pragma unroll
-        for (int grp = 0; grp < 8; ++grp) {
-          const int n = n0 + grp * 16;
-          if (n < g.N) {
-            s = seg_advance(seg, s, n);
-            const float alpha = seg.alpha[s];
-            const int op = seg.op[s];
-            const int h0 = n - seg.n_off[s];
-            float o[16];
+      for (int grp = 0; grp < 8; ++grp) {
+        const int n = n0 + grp * 16;
+        if (n < g.N) {
+          s = seg_advance(seg, s, n);
+          const float alpha = seg.alpha[s];
+          const int op = seg.op[s];
+          const int h0 = n - seg.n_off[s];
+          uint32_t a[16];
+          fetch(grp, a);
+          float o[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) o[i] = __fmul_rn(alpha, __uint_as_float(v[grp * 16 + i]));
-            if (op != 0) {
-              float t[16];
+          for (int i = 0; i < 16; ++i) o[i] = __fmul_rn(alpha, __uint_as_float(a[i]));
+          if (op != 0) {
+            float t[16];
 #pragma unroll
-              for (int i = 0; i < 16; ++i) t[i] = o[i];
-              apply_op_16(t, op, seg.a_log[s], seg.dt_bias[s], h0);
+            for (int i = 0; i < 16; ++i) t[i] = o[i];
+            apply_op_16(t, op, seg.a_log[s], seg.dt_bias[s], h0);
 #pragma unroll
-              for (int i = 0; i < 16; ++i) o[i] = t[i];
+            for (int i = 0; i < 16; ++i) o[i] = t[i];
+          }
+          if (row_live && g.out_fp32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.y) + gm * g.ldy + n);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+          } else if (row_live) {
+            uint32_t w[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const __nv_bfloat162 p = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);
+              w[i] = *reinterpret_cast<const uint32_t*>(&p);
             }
-            if (g.out_fp32) {
-              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.y) + gm * g.ldy + n);
-#pragma unroll
-              for (int i = 0; i < 4; ++i)
-                dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.y) + gm * g.ldy + n;
+            if (g.sector_stores) {
+              st_global_v8(dst, w);   // the row's 16 columns = one full 32-byte sector
             } else {
-              uint32_t w[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const __nv_bfloat162 p = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);
-                w[i] = *reinterpret_cast<const uint32_t*>(&p);
-              }
-              __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.y) + gm * g.ldy + n;
-              if (g.sector_stores) {
-                st_global_v8(dst, w);   // the row's 16 columns = one full 32-byte sector
-              } else {
-                reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
-              }
+              reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+              reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
             }
           }
         }
+      }
+    };
+    // K-parts: chunk c (columns 4c..4c+3 of this thread's 128) of unit u's
+    // partial tile; for one chunk a warp's 32 rows are 512 contiguous bytes
+    auto part_chunk = [&](int u, int c) {
+      return reinterpret_cast<float4*>(g.partial) +
+             ((((static_cast<size_t>(u) * 2 + rank) * 2 + half) * 32 + c) * BM + row_in_tile);
+    };
+    volatile int* last_flag = abort_flag + 1;
+    int local = 0;
+    bool dead = false;   // a wait ran out: skip the work, keep every barrier
+    for (int it = 0; it < n_items; ++it, ++local) {
+      const WorkItem wi = work_item(g, unit, units, num_tiles, num_kt, it);
+      const int mb = g.n_fastest ? wi.tile / num_n : wi.tile % num_m;
+      const int nb = g.n_fastest ? wi.tile % num_n : wi.tile / num_m;
+      bool ok = !dead;
+      if (ok && !wait_pair(tmem_full, static_cast<uint32_t>(local & 1))) {
+        raise_abort(SITE_EPI_TMEM_FULL, warp);
+        dead = true;
+        ok = false;
+      }
+      uint32_t v[128];
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ACC_COL + half * 128;
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld_x32(taddr + c * 32, v + c * 32);
+        tmem_wait_ld();
+        // A K-part is always a CTA's last item: no MMA waits for its
+        // accumulator, which stays in TMEM for the sum below.
+        if (wi.part < 0) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) arrive_leader(tmem_empty);
+        }
+      }
+      if (wi.part < 0) {
+        if (ok)
+          store_row(mb, nb, [&](int grp, uint32_t (&a)[16]) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) a[i] = v[grp * 16 + i];
+          });
+        continue;
+      }
+      // one K-part of a last-wave tile: publish it; the CTA that publishes
+      // the tile's last part sums all parts in part order and stores
+      if (ok) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          __stcg(part_chunk(unit, c),
+                 make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]),
+                             __uint_as_float(v[4 * c + 2]), __uint_as_float(v[4 * c + 3])));
+        __threadfence();
+      }
+      // Every epilogue warp passes both barriers once per part and every part
+      // counts itself, whatever its waits returned, so that each counter
+      // wraps back to zero (atomicInc with limit split - 1) in every launch.
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (warp == EPI_WARP0 && lane == 0) {
+        const unsigned idx = static_cast<unsigned>((wi.tile - g.full_tiles) * 2) + rank;
+        const unsigned lim = static_cast<unsigned>(g.split - 1);
+        *last_flag = atomicInc(g.counters + idx, lim) == lim;
+      }
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (ok && *last_flag && !*abort_flag) {
+        __threadfence();
+        // sum the parts in part order, whichever CTA is last, 16 columns at
+        // a time: this CTA's own part is re-read from TMEM (a K-part is a
+        // CTA's last item, so its accumulator was not released), the others
+        // come from the workspace
+        const int u0 = (wi.tile - g.full_tiles) * g.split;
+        const int mine = wi.part;
+        store_row(mb, nb, [&](int grp, uint32_t (&a)[16]) {
+          for (int p = 0; p < g.split; ++p) {
+            uint32_t t[16];
+            if (p == mine) {
+              tmem_ld_x16(taddr + grp * 16, t);
+              tmem_wait_ld();
+            } else {
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const float4 x = __ldcg(part_chunk(u0 + p, grp * 4 + c));
+                t[4 * c] = __float_as_uint(x.x);
+                t[4 * c + 1] = __float_as_uint(x.y);
+                t[4 * c + 2] = __float_as_uint(x.z);
+                t[4 * c + 3] = __float_as_uint(x.w);
+              }
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              a[i] = p == 0 ? t[i] : __float_as_uint(__uint_as_float(a[i]) + __uint_as_float(t[i]));
+          }
+        });
       }
     }
   }

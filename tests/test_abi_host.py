@@ -113,6 +113,19 @@ def test_fused_linear_validation(lib):
     assert f(*args(ok, 2, M=0)) == 0                          # no-op
 
 
+def test_gemm_workspace(lib):
+    # arrival counters + 128 fp32 partial tiles of 2 x 128 x 256
+    assert lib.nvfp4_gemm_workspace_bytes() == 4096 + 128 * 2 * 128 * 256 * 4
+    f = lib.nvfp4_fused_linear_ws
+    ok = _segs((0, 0), (32, 1))
+    args = lambda work, M=8, K=128: (P, P, P, P, M, 64, K, ok, 2, P, 64, 0, work,  # noqa: E731
+                                     lib.nvfp4_gemm_workspace_bytes(), NUL)
+    assert f(*args(P_MIS)) == ALIGN                           # workspace not 16-byte aligned
+    assert f(*args(P, K=96)) == SHAPE                         # the fused_linear checks apply
+    assert f(*args(P, M=0)) == 0
+    assert f(*args(NUL, M=0)) == 0                            # no workspace: plain fused_linear
+
+
 def test_linear_and_weight_validation(lib):
     assert lib.nvfp4_linear(P, P, 1.0, P, P, 1.0, 4, 64, 64, NUL, 64, 0, NUL) == INVALID
     assert lib.nvfp4_linear(P, P, -1.0, P, P, 1.0, 4, 64, 64, P, 64, 0, NUL) == INVALID
