@@ -201,8 +201,7 @@ constexpr uint32_t REGS_EPI = 184;      // WG2 and WG3 after setmaxnreg
 static_assert(2 * 128 * REGS_SMALL + 2 * 128 * REGS_EPI <= 65536, "register split");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
-constexpr uint32_t SF_COL = 256;        // + 48 * stage
-constexpr uint32_t SF_STRIDE = 48;
+constexpr uint32_t SF_COL = 256;        // + SF_STRIDE * stage
 constexpr int BAR_BYTES = 256;
 
 template <int CG>
@@ -211,9 +210,16 @@ struct Cfg {
   static constexpr int A_BYTES = BM * BKB;                 // 16 KB
   static constexpr int B_BYTES = B_ROWS * BKB;             // 32 / 16 KB
   static constexpr int SFA_BYTES = 4 * 512;                // 4 atoms (K = 64 each) x 128 rows
-  static constexpr int SFB_BYTES = 2 * 4 * 512;            // both row blocks of the tile
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 54 / 38 KB
-  static constexpr int STAGES = CG == 1 ? 4 : 5;
+  // Weight scales: a one-CTA tile needs both 128-row blocks of its 256 rows;
+  // in a pair each CTA's MMA half reads the scales of the weight rows that
+  // CTA loaded, from its own TMEM, so each CTA loads only its own block.
+  static constexpr int SFB_BYTES = (CG == 1 ? 2 : 1) * 4 * 512;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 54 / 36 KB
+  static constexpr int STAGES = CG == 1 ? 4 : 6;
+  // TMEM scale region per stage: SFA 16 columns, then SFB 8 (CG 1) or 4
+  // (CG 2) columns per MMA
+  static constexpr uint32_t SFB_PER_MMA = CG == 1 ? 8 : 4;
+  static constexpr uint32_t SF_STRIDE = 16 + 4 * SFB_PER_MMA;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
   static_assert(SF_COL + STAGES * SF_STRIDE <= TMEM_COLS, "TMEM budget");
@@ -238,6 +244,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
   constexpr int B_BYTES = C::B_BYTES;
   constexpr int SFA_BYTES = C::SFA_BYTES;
   constexpr int SFB_BYTES = C::SFB_BYTES;
+  constexpr uint32_t SF_STRIDE = C::SF_STRIDE;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -349,8 +356,9 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             mbar_arrive_expect_tx_warp(sfull_bar(stage), SFA_BYTES + SFB_BYTES);
             tma_load_3d_warp(smem_addr(st + A_BYTES + B_BYTES), &tmSA, 0, kt * 4,
                         mb * CG + static_cast<int>(rank), sfull_bar(stage), pol);
-            tma_load_3d_warp(smem_addr(st + A_BYTES + B_BYTES + SFA_BYTES), &tmSB, 0, kt * 4, nb * 2,
-                        sfull_bar(stage), pol);
+            // CG 2: this CTA's own weight-row block (tmSB has 1-block boxes)
+            tma_load_3d_warp(smem_addr(st + A_BYTES + B_BYTES + SFA_BYTES), &tmSB, 0, kt * 4,
+                             nb * 2 + (CG == 2 ? static_cast<int>(rank) : 0), sfull_bar(stage), pol);
           }
           ++issued;
           if (++stage == STAGES) {
@@ -397,18 +405,19 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
           r[4 * kk + 2] = a;
           r[4 * kk + 3] = a;
 #pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            // weight rows 128 j + 32 c + lane, c = 0..3 -> columns 8 kk + 4 j + c
+          for (int j = 0; j < (CG == 1 ? 2 : 1); ++j) {
+            // weight rows 128 j + 32 c + lane of the stage's blocks, c = 0..3
+            // -> columns SFB_PER_MMA kk + 4 j + c
             const uint4 b = ld_shared_v4(sfb_s + j * 2048 + kk * 512 + lane * 16);
-            r[16 + 8 * kk + 4 * j + 0] = b.x;
-            r[16 + 8 * kk + 4 * j + 1] = b.y;
-            r[16 + 8 * kk + 4 * j + 2] = b.z;
-            r[16 + 8 * kk + 4 * j + 3] = b.w;
+            r[16 + C::SFB_PER_MMA * kk + 4 * j + 0] = b.x;
+            r[16 + C::SFB_PER_MMA * kk + 4 * j + 1] = b.y;
+            r[16 + C::SFB_PER_MMA * kk + 4 * j + 2] = b.z;
+            r[16 + C::SFB_PER_MMA * kk + 4 * j + 3] = b.w;
           }
         }
         const uint32_t col = tmem_base + lane_off + SF_COL + SF_STRIDE * stage;
         tmem_st_x32(col, r);
-        tmem_st_x16(col + 32, r + 32);
+        if constexpr (CG == 1) tmem_st_x16(col + 32, r + 32);
         tmem_wait_st();
         tc_fence_before();
         // the MMA warp waits on this barrier alone: arrive only once the
@@ -469,7 +478,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
           if (prev >= 0) tc_commit_all_warp<CG>(empty_bar(prev));
           for (int kk = 1; kk < nk; ++kk)
             mma_mxf4nvf4_warp<CG>(tmem_base + ACC_COL, ad + 2 * kk, bd + 2 * kk, idesc,
-                                col + 4 * kk, col + 16 + 8 * kk, 1u);
+                                col + 4 * kk, col + 16 + C::SFB_PER_MMA * kk, 1u);
           prev = stage;
           if (++stage == STAGES) {
             stage = 0;
