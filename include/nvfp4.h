@@ -248,6 +248,30 @@ nvfp4_status nvfp4_fused_linear_ws(const void* a_codes, const void* a_scales,
                                    void* workspace, size_t workspace_bytes,
                                    nvfp4_stream_t stream);
 
+/* The MLP pair's first half in one kernel (gate_up GEMM, SiLU(gate) * up
+ * and the NVFP4 quantisation of the product that the down projection
+ * consumes; the all-linear-layers W4A4 recipe: nefut abstract).  The weight
+ * [2H, K] holds the gate module's H rows, then the up module's H rows, each
+ * quantised with its own global scale (w_gs_gate, w_gs_up).  For every
+ * activation row m and h < H:
+ *   g = bf16(fp32(a_gs * w_gs_gate) * acc_gate[m, h]),
+ *   u = bf16(fp32(a_gs * w_gs_up) * acc_up[m, h]),
+ *   h = bf16(g / (1 + exp(-g)) * u)        (fp32 steps, as nvfp4_silu_mul),
+ * and h [M, H] is quantised under the static global scale h_gs exactly as
+ * nvfp4_quantize_act quantises it: h_codes [M, H/2], h_scales
+ * nvfp4_scale_bytes(M, H) bytes in the atom layout (padding rows zero).
+ * The result equals nvfp4_fused_linear (bf16 out, segments gate | up) ->
+ * nvfp4_silu_mul -> nvfp4_quantize_act bit for bit, without the bf16
+ * [M, 2H] and [M, H] intermediates.  Requires H % 128 == 0, K % 64 == 0,
+ * 16-byte aligned caller-owned device pointers, finite positive scales;
+ * violations return before any launch.  Queued on `stream`. */
+nvfp4_status nvfp4_gate_up_silu_quantize(const void* a_codes, const void* a_scales,
+                                          const void* w_codes, const void* w_scales,
+                                          int64_t M, int64_t H, int64_t K,
+                                          float a_gs, float w_gs_gate, float w_gs_up,
+                                          float h_gs, void* h_codes, void* h_scales,
+                                          nvfp4_stream_t stream);
+
 /* MLP glue between the two projections of the MLP pair (not an NVFP4 step):
  * h[m, j] = bf16(silu(gu[m, j]) * gu[m, H + j]) for j < H, computed in fp32.
  * gu: bf16 [M, ld_in] with ld_in >= 2H; h: bf16 [M, ld_out], ld_out >= H.

@@ -21,7 +21,8 @@ __all__ = [
     "nvfp4_codes_bytes", "nvfp4_scale_bytes", "nvfp4_global_scale", "nvfp4_amax",
     "nvfp4_quantize_act", "nvfp4_quantize_weight", "nvfp4_quantize_weight_noalloc",
     "nvfp4_linear", "nvfp4_fused_linear", "nvfp4_gemm_workspace_bytes", "nvfp4_gemm_workspace",
-    "nvfp4_silu_mul", "nvfp4_last_device_error", "nvfp4_set_gemm_path", "nvfp4_set_launch_overlap",
+    "nvfp4_gate_up_silu_quantize", "nvfp4_silu_mul", "nvfp4_last_device_error", "nvfp4_set_gemm_path",
+    "nvfp4_set_launch_overlap",
     "nvfp4_set_wait_limit_ns", "nvfp4_test_e2m1", "nvfp4_test_e4m3", "nvfp4_test_wait_timeout",
     "SegmentSpec", "NVFP4Error", "OP_NONE", "OP_SIGMOID", "OP_GDN_DECAY",
 ]
@@ -183,6 +184,24 @@ def nvfp4_fused_linear(a_codes, a_scales, w_codes, w_scales, M: int, N: int, K: 
                                            workspace.numel() * workspace.element_size(),
                                            _stream(stream)), "nvfp4_fused_linear_ws")
     return y
+
+
+def nvfp4_gate_up_silu_quantize(a_codes, a_scales, w_codes, w_scales, M: int, H: int, K: int,
+                                a_gs: float, w_gs_gate: float, w_gs_up: float, h_gs: float,
+                                h_codes: Optional[torch.Tensor] = None,
+                                h_scales: Optional[torch.Tensor] = None,
+                                stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    dev = a_codes.device
+    if h_codes is None:
+        h_codes = torch.empty((M, H // 2), dtype=torch.uint8, device=dev)
+    if h_scales is None:
+        h_scales = torch.empty(nvfp4_scale_bytes(M, H), dtype=torch.uint8, device=dev)
+    check(load().nvfp4_gate_up_silu_quantize(
+        _ptr(a_codes), _ptr(a_scales), _ptr(w_codes), _ptr(w_scales), M, H, K,
+        ctypes.c_float(a_gs), ctypes.c_float(w_gs_gate), ctypes.c_float(w_gs_up),
+        ctypes.c_float(h_gs), _ptr(h_codes), _ptr(h_scales), _stream(stream)),
+        "nvfp4_gate_up_silu_quantize")
+    return h_codes, h_scales
 
 
 def nvfp4_silu_mul(gu: torch.Tensor, H: int, h: Optional[torch.Tensor] = None,

@@ -46,6 +46,8 @@ SIGNATURES = {
     "nvfp4_gemm_workspace_bytes": (_sz, []),
     "nvfp4_fused_linear_ws": (_st, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.POINTER(Segment),
                                     _i32, _vp, _i64, _st, _vp, _sz, _vp]),
+    "nvfp4_gate_up_silu_quantize": (_st, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _f32, _f32, _f32,
+                                          _f32, _vp, _vp, _vp]),
     "nvfp4_silu_mul": (_st, [_vp, _i64, _i64, _i64, _vp, _i64, _vp]),
     "nvfp4_status_string": (ctypes.c_char_p, [_st]),
     "nvfp4_last_device_error": (_st, [_vp, ctypes.POINTER(ctypes.c_uint64)]),

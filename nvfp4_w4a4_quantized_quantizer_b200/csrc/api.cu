@@ -71,8 +71,10 @@ struct DeviceInfo {
   int sms = 0;
   bool attr_tc = false;
   bool attr_tc2 = false;
+  bool attr_tc2_swiglu = false;
   int quant_blocks = 0;   // resident k_quantize blocks per SM
   int pairs = 0;          // co-resident clusters of two CTAs of k_gemm_tc<2>
+  int swiglu_pairs = 0;   // the same for k_gemm_tc<2, true>
   bool attr_small[3] = {false, false, false};
 };
 DeviceInfo g_dev[MAX_DEVICES];
@@ -702,6 +704,90 @@ nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales, const
                                 nvfp4_out_dtype out_dtype, nvfp4_stream_t stream) {
   return nvfp4_fused_linear_ws(a_codes, a_scales, w_codes, w_scales, M, N, K, segs, nseg, y, ldy,
                                out_dtype, nullptr, 0, stream);
+}
+
+nvfp4_status nvfp4_gate_up_silu_quantize(const void* a_codes, const void* a_scales,
+                                          const void* w_codes, const void* w_scales, int64_t M,
+                                          int64_t H, int64_t K, float a_gs, float w_gs_gate,
+                                          float w_gs_up, float h_gs, void* h_codes, void* h_scales,
+                                          nvfp4_stream_t stream) {
+  if (a_codes == nullptr || a_scales == nullptr || w_codes == nullptr || w_scales == nullptr ||
+      h_codes == nullptr || h_scales == nullptr)
+    return NVFP4_ERR_INVALID_ARG;
+  if (M < 0 || M > kMaxDim || H < 128 || H % 128 != 0 || 2 * H > kMaxDim || K < 64 ||
+      K % 64 != 0 || K > kMaxDim)
+    return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(w_codes) ||
+      !aligned16(w_scales) || !aligned16(h_codes) || !aligned16(h_scales))
+    return NVFP4_ERR_ALIGNMENT;
+  if (!good_scale(a_gs) || !good_scale(w_gs_gate) || !good_scale(w_gs_up) || !good_scale(h_gs))
+    return NVFP4_ERR_INVALID_ARG;
+  if (M == 0) return NVFP4_OK;
+  int dev;
+  DeviceInfo* info;
+  nvfp4_status st = current_device(&dev, &info);
+  if (st != NVFP4_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+
+  nvfp4::GemmArgs g = {};
+  g.M = static_cast<int>(M);
+  g.N = static_cast<int>(2 * H);
+  g.K = static_cast<int>(K);
+  g.wait_ns = g_wait_ns;
+  g.H = static_cast<int>(H);
+  g.alpha_gate = a_gs * w_gs_gate;   // fp32 products, as the segment table forms them
+  g.alpha_up = a_gs * w_gs_up;
+  g.h_gs = h_gs;
+  g.h_codes = static_cast<uint8_t*>(h_codes);
+  g.h_scales = static_cast<uint8_t*>(h_scales);
+  const int64_t a_bytes = M * (K / 2), w_bytes = 2 * H * (K / 2);
+  g.n_fastest = a_bytes > (64ll << 20) && w_bytes < a_bytes;
+  nvfp4_segment one = {0, w_gs_gate, a_gs, NVFP4_OP_NONE, nullptr, nullptr};
+  SegTable table;
+  if ((st = build_segments(&one, 1, 2 * H, &table)) != NVFP4_OK) return st;
+
+  CUtensorMap ta, tb, tsa, tsb;
+  if ((st = code_map(a_codes, M, K / 2, nvfp4::tc::BM, dev, &ta)) != NVFP4_OK) return st;
+  if ((st = code_map(w_codes, 2 * H, K / 2, nvfp4::tc::BN / 2, dev, &tb)) != NVFP4_OK) return st;
+  if ((st = scale_map(a_scales, M, K, 1, dev, &tsa)) != NVFP4_OK) return st;
+  if ((st = scale_map(w_scales, 2 * H, K, 1, dev, &tsb)) != NVFP4_OK) return st;
+
+  constexpr int smem = nvfp4::tc::Cfg<2>::SMEM_BYTES;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(nvfp4::tc::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = cs;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (!info->attr_tc2_swiglu) {
+    if (cudaFuncSetAttribute(nvfp4::k_gemm_tc<2, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return NVFP4_ERR_CUDA;
+    cfg.gridDim = dim3(2 * (info->sms / 2), 1, 1);
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, nvfp4::k_gemm_tc<2, true>, &cfg) !=
+            cudaSuccess ||
+        clusters < 1) {
+      cudaGetLastError();
+      return NVFP4_ERR_CUDA;
+    }
+    info->swiglu_pairs = clusters;
+    info->attr_tc2_swiglu = true;
+  }
+  const int64_t tiles = ((M + 2 * nvfp4::tc::BM - 1) / (2 * nvfp4::tc::BM)) * (H / 128);
+  const int pairs = static_cast<int>(tiles < info->swiglu_pairs ? tiles : info->swiglu_pairs);
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  if (cudaLaunchKernelEx(&cfg, nvfp4::k_gemm_tc<2, true>, ta, tb, tsa, tsb, g, table) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+  }
+  return check_launch();
 }
 
 nvfp4_status nvfp4_linear(const void* a_codes, const void* a_scales, float a_gs,

@@ -35,6 +35,7 @@
 #include <cstdint>
 
 #include "ptx.cuh"
+#include "quantize.cuh"
 
 namespace nvfp4 {
 
@@ -72,6 +73,16 @@ struct GemmArgs {
   float* partial;      // [split_units][2 CTAs][2 halves][32 chunks][128 rows] float4
   unsigned* counters;  // [num_tiles - full_tiles][2 CTAs]
   uint64_t wait_ns;
+  // SwiGLU epilogue (k_gemm_tc<2, true>): the weight is [gate; up], H rows
+  // each; tile column nb covers h columns [128 nb, 128 nb + 128) -- the even
+  // CTA loads those gate rows, the odd CTA the matching up rows -- and the
+  // epilogue writes h = bf16(silu(g) * u), g = bf16(alpha_gate * acc_gate),
+  // u = bf16(alpha_up * acc_up), quantised under h_gs: codes [M, H/2] and
+  // scales in the atom layout (the down projection's activation operand).
+  int H;
+  float alpha_gate, alpha_up, h_gs;
+  uint8_t* h_codes;
+  uint8_t* h_scales;
 };
 
 // ------------------------------------------------------------- epilogue op
@@ -187,6 +198,51 @@ __device__ __forceinline__ WorkItem work_item(const GemmArgs& g, int unit, int u
   return w;
 }
 
+// SwiGLU epilogue of one output row: g = bf16(alpha_gate * acc) for the 64
+// gate columns in v[0..63], u = bf16(alpha_up * acc) for the up columns in
+// v[64..127], h = bf16(silu(g) * u) (silu_mul_f32, as the standalone MLP
+// glue kernel computes it), then NVFP4 quantisation of h's four 16-blocks
+// under g.h_gs with exactly k_quantize's arithmetic: 32 code bytes at
+// h_codes[gm, h0 / 2] and the four scale bytes (one 32-bit word) at the
+// atom-layout position of blocks h0/16 .. h0/16 + 3.  Rows gm >= M store
+// only their scale word (zero).
+__device__ __forceinline__ void swiglu_store_row(const GemmArgs& g, int64_t gm, int h0,
+                                                 const uint32_t (&v)[128]) {
+  const float c = __fmul_rn(6.0f, g.h_gs);
+  uint32_t codes[8];
+  uint32_t word = 0;
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    float h[16];
+    uint32_t amax_bits = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float gv = __bfloat162float(__float2bfloat16_rn(__fmul_rn(g.alpha_gate, __uint_as_float(v[16 * b + i]))));
+      const float uv = __bfloat162float(__float2bfloat16_rn(__fmul_rn(g.alpha_up, __uint_as_float(v[64 + 16 * b + i]))));
+      h[i] = __bfloat162float(__float2bfloat16_rn(silu_mul_f32(gv, uv)));
+      // |h| max on the bit patterns (h is bf16-valued: exact)
+      const uint32_t mag = __float_as_uint(h[i]) & 0x7FFFFFFFu;
+      amax_bits = mag > amax_bits ? mag : amax_bits;
+    }
+    const uint32_t sc = cvt_e4m3(__fdiv_rn(__uint_as_float(amax_bits), c));
+    const float r = block_reciprocal(sc, g.h_gs);
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      float f[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) f[k] = __fmul_rn(h[8 * hh + k], r);
+      codes[2 * b + hh] = sc == 0 ? 0u : cvt_e2m1x8(f);
+    }
+    word |= sc << (8 * b);
+  }
+  if (gm < g.M) {
+    uint4* dst = reinterpret_cast<uint4*>(g.h_codes + gm * (g.H / 2) + h0 / 2);
+    dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+    dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+  }
+  *reinterpret_cast<uint32_t*>(g.h_scales + sf_offset(gm, h0 / 16, g.H)) = word;
+}
+
 namespace tc {
 constexpr int BM = 128;                 // rows of A per CTA
 constexpr int BN = 256;                 // tile columns (MMA N)
@@ -230,12 +286,14 @@ struct Cfg {
 // tmA / tmB: code matrices [rows, K/2] (box 128 bytes x 128 / (256 / CG)
 // rows, 128-byte swizzle).  tmSA / tmSB: scale buffers viewed as [row blocks]
 // [K/64 atoms][64 u64] (box 64 x 4 x 1 / 2, i.e. one stage's atoms of 1 / 2
-// row blocks).  CG = 2 must be launched with clusters of 2 CTAs.
-template <int CG>
+// row blocks).  CG = 2 must be launched with clusters of 2 CTAs.  SWIGLU
+// (CG = 2 only): the epilogue is the SwiGLU one described at GemmArgs::H.
+template <int CG, bool SWIGLU = false>
 __global__ void __launch_bounds__(tc::THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
               const GemmArgs g, const __grid_constant__ SegTable seg) {
+  static_assert(!SWIGLU || CG == 2, "the SwiGLU epilogue pairs gate and up rows across a CTA pair");
   using namespace tc;
   using C = Cfg<CG>;
   constexpr int STAGES = C::STAGES;
@@ -259,7 +317,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
   const int unit = static_cast<int>(blockIdx.x) / CG;     // CTA (pair) index
   const int units = static_cast<int>(gridDim.x) / CG;
   const int num_m = (g.M + BM * CG - 1) / (BM * CG);
-  const int num_n = (g.N + BN - 1) / BN;
+  const int num_n = SWIGLU ? g.H / 128 : (g.N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
   const int num_kt = (g.K + BK - 1) / BK;
   const int n_items = work_count(g, unit, units, num_tiles);
@@ -337,7 +395,9 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         const int mb = g.n_fastest ? tile / num_n : tile % num_m;
         const int nb = g.n_fastest ? tile % num_n : tile / num_m;
         const int arow = (mb * CG + static_cast<int>(rank)) * BM;
-        const int brow = nb * BN + static_cast<int>(rank) * C::B_ROWS;
+        // SwiGLU: the even CTA's half of the tile is gate rows, the odd CTA's the up rows
+        const int brow = SWIGLU ? nb * 128 + (rank ? g.H : 0)
+                                : nb * BN + static_cast<int>(rank) * C::B_ROWS;
         for (int kt = w.kt0; kt < w.kt1; ++kt) {
           if (!wait_pair(empty_bar(stage), phase ^ 1u)) {
             raise_abort(SITE_PRODUCER_EMPTY, warp);
@@ -356,9 +416,12 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             mbar_arrive_expect_tx_warp(sfull_bar(stage), SFA_BYTES + SFB_BYTES);
             tma_load_3d_warp(smem_addr(st + A_BYTES + B_BYTES), &tmSA, 0, kt * 4,
                         mb * CG + static_cast<int>(rank), sfull_bar(stage), pol);
-            // CG 2: this CTA's own weight-row block (tmSB has 1-block boxes)
+            // CG 2: this CTA's own weight-row block (tmSB has 1-block boxes);
+            // SwiGLU: the gate block nb (even CTA) or the up block H/128 + nb
+            const int sfb_block = SWIGLU ? nb + (rank ? g.H / 128 : 0)
+                                         : nb * 2 + (CG == 2 ? static_cast<int>(rank) : 0);
             tma_load_3d_warp(smem_addr(st + A_BYTES + B_BYTES + SFA_BYTES), &tmSB, 0, kt * 4,
-                             nb * 2 + (CG == 2 ? static_cast<int>(rank) : 0), sfull_bar(stage), pol);
+                             sfb_block, sfull_bar(stage), pol);
           }
           ++issued;
           if (++stage == STAGES) {
@@ -577,8 +640,19 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ACC_COL + half * 128;
       if (ok) {
         tc_fence_after();
+        if constexpr (SWIGLU) {
+          // this warp's 64 h columns: gate accumulator columns [64 half, +64)
+          // into v[0..63], the matching up columns [128 + 64 half, +64) into v[64..127]
+          const uint32_t lane_base = taddr - half * 128;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld_x32(taddr + c * 32, v + c * 32);
+          for (int c = 0; c < 2; ++c) {
+            tmem_ld_x32(lane_base + half * 64 + c * 32, v + c * 32);
+            tmem_ld_x32(lane_base + 128 + half * 64 + c * 32, v + 64 + c * 32);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld_x32(taddr + c * 32, v + c * 32);
+        }
         tmem_wait_ld();
         // A K-part is always a CTA's last item: no MMA waits for its
         // accumulator, which stays in TMEM for the sum below.
@@ -588,7 +662,15 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
           if (lane == 0) arrive_leader(tmem_empty);
         }
       }
-      if (wi.part < 0) {
+      if constexpr (SWIGLU) {
+        // whole tiles only (the host never splits this launch); rows past M
+        // inside the last 128-row block still write their (zero) scale
+        // bytes: the scale buffer's padding rows must hold zeros
+        const int64_t gm = static_cast<int64_t>(mb * CG + static_cast<int>(rank)) * BM + row_in_tile;
+        const int64_t rows_padded = (static_cast<int64_t>(g.M) + 127) / 128 * 128;
+        if (ok && gm < rows_padded) swiglu_store_row(g, gm, nb * 128 + half * 64, v);
+        continue;
+      } else if (wi.part < 0) {
         if (ok)
           store_row(mb, nb, [&](int grp, uint32_t (&a)[16]) {
 #pragma unroll

@@ -328,6 +328,21 @@ __global__ void __launch_bounds__(AMAX_THREADS) k_amax(const __nv_bfloat16* __re
 }
 
 // ------------------------------------------------------- MLP glue (SiLU*up)
+// h = fp32(silu(g) * u) for bf16-valued g and u: g / (1 + e^-g) with an
+// IEEE divide, then the product, each step rounded to nearest and none
+// contracted (the fused gate_up epilogue computes the same function, so
+// both paths give identical h).
+__device__ __forceinline__ float silu_mul_f32(float g, float u) {
+  return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+}
+
+// Block reciprocal of scale code `code` under global scale gs:
+// fp32(1 / fp32(e4m3(code) * gs)), 0 for code 0 -- the entry of k_quantize's
+// host-built table, computed on the device with the same two roundings.
+__device__ __forceinline__ float block_reciprocal(uint32_t code, float gs) {
+  return code == 0 ? 0.0f : __frcp_rn(__fmul_rn(e4m3_value(code), gs));
+}
+
 constexpr int SILU_THREADS = 256;
 
 __global__ void __launch_bounds__(SILU_THREADS) k_silu_mul(const __nv_bfloat16* __restrict__ gu,
@@ -346,8 +361,8 @@ __global__ void __launch_bounds__(SILU_THREADS) k_silu_mul(const __nv_bfloat16* 
     uint32_t w[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float a0 = __fmul_rn(__fdiv_rn(g[2 * e], 1.0f + expf(-g[2 * e])), u[2 * e]);
-      const float a1 = __fmul_rn(__fdiv_rn(g[2 * e + 1], 1.0f + expf(-g[2 * e + 1])), u[2 * e + 1]);
+      const float a0 = silu_mul_f32(g[2 * e], u[2 * e]);
+      const float a1 = silu_mul_f32(g[2 * e + 1], u[2 * e + 1]);
       const __nv_bfloat162 p = __floats2bfloat162_rn(a0, a1);
       w[e] = *reinterpret_cast<const uint32_t*>(&p);
     }

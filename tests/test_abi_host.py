@@ -140,6 +140,20 @@ def test_linear_and_weight_validation(lib):
     assert w(P, 64, 64, 64, None, 1, gs, P, P, NUL, NUL) == INVALID  # workspace required
 
 
+def test_gate_up_silu_quantize_validation(lib):
+    f = lib.nvfp4_gate_up_silu_quantize
+    args = lambda M=8, H=128, K=128, hc=P, gs=1.0: (P, P, P, P, M, H, K, 1.0, 1.0, 1.0, gs, hc, P,  # noqa: E731
+                                                   NUL)
+    assert f(*args(H=192)) == SHAPE                           # H % 128
+    assert f(*args(H=0)) == SHAPE
+    assert f(*args(K=96)) == SHAPE                            # K % 64
+    assert f(*args(hc=NUL)) == INVALID
+    assert f(*args(hc=P_MIS)) == ALIGN
+    assert f(*args(gs=0.0)) == INVALID
+    assert f(*args(gs=float("nan"))) == INVALID
+    assert f(*args(M=0)) == 0
+
+
 def test_misc_validation(lib):
     assert lib.nvfp4_set_gemm_path(5) == INVALID
     assert lib.nvfp4_set_gemm_path(0) == 0

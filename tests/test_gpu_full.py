@@ -202,6 +202,12 @@ def test_mlp_pair_full():
     quant_err = np.linalg.norm(dref - d_unquantised)
     h = nv.nvfp4_silu_mul(yb, H2)
     hc2, hs2 = nv.nvfp4_quantize_act(h, a2)
+    del h
+    # the one-kernel form of gate_up -> silu_mul -> quantise (as bench.py runs
+    # the MLP step) gives the same codes and scales bit for bit
+    fc, fs = nv.nvfp4_gate_up_silu_quantize(ac, as_, wc, ws, M, H2, K, a_gs, w_gs[0], w_gs[1], a2)
+    assert torch.equal(fc, hc2) and torch.equal(fs, hs2)
+    del fc, fs
     d_full = nv.nvfp4_linear(hc2, hs2, a2, w2c, w2s, g2_gpu, M, workloads.MLP_DOWN_N,
                              workloads.MLP_DOWN_K, out_dtype=nv.OUT_FP32)
     assert nv.nvfp4_last_device_error()[0] == 0

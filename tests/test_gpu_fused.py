@@ -18,6 +18,8 @@ import workloads
 import nvfp4_w4a4_quantized_quantizer_b200 as nv
 from tests import _helpers as H
 
+_H = H  # the helpers, where a parameter named H (the MLP hidden size) shadows them
+
 pytestmark = pytest.mark.gpu
 
 LARGE, SMALL, AUTO, PAIR, PAIR_NFAST = 1, 2, 0, 3, 4
@@ -120,3 +122,53 @@ def test_repair_vs_shared_scale():
                                    atol=1e-6 * np.abs(yb[:, sl]).max())
         if i > 0:
             assert abs(ratio - 1) > 1e-3        # the modules really do differ
+
+
+# ------------------------------------------ MLP first half in one kernel
+def _gate_up_operands(M, H, K, seed):
+    rng = np.random.default_rng(seed)
+    xb = workloads.random_bf16((M, K), seed=seed, std=1.0)
+    std_g, std_u = 1 / np.sqrt(K), 3 / np.sqrt(K)          # up weights 3x the gate's scale
+    wb = np.concatenate([workloads.random_bf16((H, K), seed=seed + 1, std=std_g),
+                         workloads.random_bf16((H, K), seed=seed + 2, std=std_u)])
+    a_gs = float(oracle.global_scale(np.abs(_H.f32(xb)).max()))
+    ac, as_ = nv.nvfp4_quantize_act(_H.bf16_dev(xb), a_gs)
+    wc, ws, (g_gs, u_gs) = nv.nvfp4_quantize_weight(_H.bf16_dev(wb), seg_offsets=[0, H])
+    return ac, as_, wc, ws, a_gs, g_gs, u_gs, rng
+
+
+
+@pytest.mark.parametrize("M,H,K", [(100, 128, 256), (256, 384, 512), (300, 256, 1280),
+                                   (600, 640, 320), (2304, 1024, 256)])
+def test_gate_up_silu_quantize_equals_the_unfused_chain(M, H, K):
+    """One kernel = fused_linear (bf16, gate | up) -> silu_mul -> quantize_act, bit for bit,
+    padding rows of the scale buffer included."""
+    ac, as_, wc, ws, a_gs, g_gs, u_gs, _ = _gate_up_operands(M, H, K, seed=M + H + K)
+    segs = [nv.SegmentSpec(0, g_gs, a_gs), nv.SegmentSpec(H, u_gs, a_gs)]
+    gu = nv.nvfp4_fused_linear(ac, as_, wc, ws, M, 2 * H, K, segs)
+    h = nv.nvfp4_silu_mul(gu, H)
+    h_gs = float(oracle.global_scale(float(h.float().abs().max().item())))
+    ref_c, ref_s = nv.nvfp4_quantize_act(h, h_gs)
+    hc = torch.full((M, H // 2), 0xAB, dtype=torch.uint8, device="cuda")
+    hs = torch.full((nv.nvfp4_scale_bytes(M, H),), 0xCD, dtype=torch.uint8, device="cuda")
+    nv.nvfp4_gate_up_silu_quantize(ac, as_, wc, ws, M, H, K, a_gs, g_gs, u_gs, h_gs,
+                                   h_codes=hc, h_scales=hs)
+    st, info = nv.nvfp4_last_device_error()
+    assert st == 0, f"device error word {info:#x}"
+    assert torch.equal(hc, ref_c)
+    assert torch.equal(hs, ref_s)
+
+
+def test_silu_mul_matches_the_oracle_within_one_bf16_step():
+    """nvfp4_silu_mul (fp32 steps) against the float64 oracle on the same bf16 gate / up."""
+    M, Hd = 64, 4096
+    rng = np.random.default_rng(3)
+    g = workloads.f32_to_bf16_bits(rng.normal(0, 3, (M, Hd)).astype(np.float32))
+    u = workloads.f32_to_bf16_bits(rng.normal(0, 2, (M, Hd)).astype(np.float32))
+    gu = np.concatenate([g, u], axis=1)
+    h = nv.nvfp4_silu_mul(H.bf16_dev(gu), Hd).float().cpu().numpy()
+    ref = oracle.silu_mul_bf16(H.f32(g), H.f32(u))
+    # both are bf16-rounded: at most one bf16 step apart (fp32 vs float64 inner steps)
+    step = np.abs(ref).astype(np.float64) * 2.0 ** -7 + 1e-30
+    assert np.all(np.abs(h.astype(np.float64) - ref) <= step)
+    assert np.mean(h == ref) > 0.99
