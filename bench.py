@@ -294,8 +294,9 @@ class MlpChain:
         self.xsc = torch.empty(nv.nvfp4_scale_bytes(self.M, self.K), dtype=torch.uint8, device=device)
         self.hc = torch.empty((self.M, self.H // 2), dtype=torch.uint8, device=device)
         self.hsc = torch.empty(nv.nvfp4_scale_bytes(self.M, self.H), dtype=torch.uint8, device=device)
-        self.y = torch.empty((self.M, self.N2), dtype=torch.bfloat16, device=device)
-        self.ys = [self.y, self.y]
+        # two output buffers: a step's read-back may overlap the next step's kernels
+        self.ys = [torch.empty((self.M, self.N2), dtype=torch.bfloat16, device=device)
+                   for _ in range(2)]
 
     def quantize(self, i, stream, x=None):
         xx = self.xs[i % len(self.xs)] if x is None else x
@@ -311,7 +312,7 @@ class MlpChain:
     def down(self, i, stream):
         _, _, w2c, w2s = self.ws[i % len(self.ws)]
         self.nv.nvfp4_fused_linear(self.hc, self.hsc, w2c, w2s, self.M, self.N2, self.H, self.segs2,
-                                   y=self.y, stream=stream, workspace=self.work)
+                                   y=self.ys[i % 2], stream=stream, workspace=self.work)
 
     def gemm(self, i, stream):
         """Everything after the first quantisation."""
@@ -389,30 +390,52 @@ def time_kernels(layer: Layer, reps: int, stream):
 
 
 def e2e(layer: Layer, steps: int, warmup: int, stream):
-    """Same metric through the public API from pinned host buffers: H2D of the
-    step's activations, quantise, GEMM, D2H of the bf16 output, every step."""
+    """Same metric through the public API from pinned host buffers: every
+    step copies its activations in (H2D), quantises, runs the GEMM and reads
+    its bf16 output back (D2H).  Steps are pipelined as a serving loop would
+    run them: the copy-in of step i+1 and the copy-out of step i-1 overlap
+    step i's kernels (three streams, double-buffered device input and output,
+    events order each buffer's reuse); the timed region spans the first
+    copy-in to the last copy-out."""
+    dev = layer.xs[0].device
     xh = torch.from_numpy(layer.x_host.view(np.int16)).view(torch.bfloat16).pin_memory()
-    yh = torch.empty(tuple(layer.ys[0].shape), dtype=torch.bfloat16).pin_memory()
-    xd = torch.empty_like(layer.xs[0])
+    yh = [torch.empty(tuple(layer.ys[0].shape), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    xd = [torch.empty_like(layer.xs[0]) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    in_done, cmp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    for e in cmp_done + out_done:
+        e.record(stream)            # "done" before the first use of each buffer
 
     def one(i):
+        j = i % 2
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(cmp_done[j])            # step i-2's kernels are done with xd[j]
+            xd[j].copy_(xh, non_blocking=True)
+            in_done[j].record(s_in)
         with torch.cuda.stream(stream):
-            xd.copy_(xh, non_blocking=True)
-            layer.quantize(i, stream, x=xd)
+            stream.wait_event(in_done[j])
+            stream.wait_event(out_done[j])          # step i-2's copy-out has read ys[j]
+            layer.quantize(i, stream, x=xd[j])
             layer.gemm(i, stream)
-            yh.copy_(layer.ys[i % 2], non_blocking=True)
+            cmp_done[j].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(cmp_done[j])
+            yh[j].copy_(layer.ys[i % 2], non_blocking=True)
+            out_done[j].record(s_out)
 
     for i in range(warmup):
         one(i)
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for i in range(steps):
+    a.record(s_in)
+    for i in range(warmup, warmup + steps):
         one(i)
-    b.record(stream)
+    s_out.wait_event(cmp_done[(warmup + steps - 1) % 2])
+    b.record(s_out)
     b.synchronize()
     ms = a.elapsed_time(b) / steps
-    return ms, xh.numel() * 2, yh.numel() * 2
+    return ms, xh.numel() * 2, yh[0].numel() * 2
 
 
 def small_m_sweep(device, stream, iters=240, warmup=10):
