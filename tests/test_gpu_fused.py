@@ -145,7 +145,9 @@ def test_gate_up_silu_quantize_equals_the_unfused_chain(M, H, K):
     padding rows of the scale buffer included."""
     ac, as_, wc, ws, a_gs, g_gs, u_gs, _ = _gate_up_operands(M, H, K, seed=M + H + K)
     segs = [nv.SegmentSpec(0, g_gs, a_gs), nv.SegmentSpec(H, u_gs, a_gs)]
+    nv.nvfp4_set_gemm_path(PAIR)        # the fused kernel is a CTA-pair kernel at every M
     gu = nv.nvfp4_fused_linear(ac, as_, wc, ws, M, 2 * H, K, segs)
+    nv.nvfp4_set_gemm_path(AUTO)
     h = nv.nvfp4_silu_mul(gu, H)
     h_gs = float(oracle.global_scale(float(h.float().abs().max().item())))
     ref_c, ref_s = nv.nvfp4_quantize_act(h, h_gs)
