@@ -364,6 +364,43 @@ nvfp4_status noalloc_scratch(float** out) {
   return NVFP4_OK;
 }
 
+// Launch configuration of a CTA-pair kernel (clusters of two CTAs, its
+// dynamic shared memory, `st`); once per device and kernel, also the
+// shared-memory attribute and the number of pairs that fit at once (clusters
+// are placed within one GPC, so an SM count that is odd inside a GPC leaves
+// an SM out).  attr must outlive cfg.
+template <typename Kernel>
+nvfp4_status pair_config(Kernel kernel, DeviceInfo* info, bool* configured, int* max_pairs,
+                         cudaStream_t st, cudaLaunchConfig_t* cfg, cudaLaunchAttribute* attr) {
+  constexpr int smem = nvfp4::tc::Cfg<2>::SMEM_BYTES;
+  *cfg = cudaLaunchConfig_t{};
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg->blockDim = dim3(nvfp4::tc::THREADS, 1, 1);
+  cfg->dynamicSmemBytes = smem;
+  cfg->stream = st;
+  cfg->attrs = attr;
+  cfg->numAttrs = 1;
+  if (!*configured) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return NVFP4_ERR_CUDA;
+    }
+    cfg->gridDim = dim3(2 * (info->sms / 2), 1, 1);
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kernel, cfg) != cudaSuccess || clusters < 1) {
+      cudaGetLastError();
+      return NVFP4_ERR_CUDA;
+    }
+    *max_pairs = clusters;
+    *configured = true;
+  }
+  return NVFP4_OK;
+}
+
 }  // namespace
 
 // =================================================================== C ABI
@@ -636,34 +673,11 @@ nvfp4_status nvfp4_fused_linear_ws(const void* a_codes, const void* a_scales, co
     nvfp4::k_gemm_tc<1><<<grid, nvfp4::tc::THREADS, smem, cs>>>(ta, tb, tsa, tsb, g, table);
     return check_launch();
   }
-  constexpr int smem = nvfp4::tc::Cfg<2>::SMEM_BYTES;
-  cudaLaunchConfig_t cfg = {};
+  cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.blockDim = dim3(nvfp4::tc::THREADS, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = cs;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (!info->attr_tc2) {
-    if (cudaFuncSetAttribute(nvfp4::k_gemm_tc<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
-      return NVFP4_ERR_CUDA;
-    // how many pairs fit at once (clusters are placed within one GPC, so an
-    // SM count that is odd inside a GPC leaves an SM out)
-    cfg.gridDim = dim3(2 * (info->sms / 2), 1, 1);
-    int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, nvfp4::k_gemm_tc<2>, &cfg) != cudaSuccess ||
-        clusters < 1) {
-      cudaGetLastError();
-      return NVFP4_ERR_CUDA;
-    }
-    info->pairs = clusters;
-    info->attr_tc2 = true;
-  }
+  if ((st = pair_config(nvfp4::k_gemm_tc<2>, info, &info->attr_tc2, &info->pairs, cs, &cfg,
+                        attr)) != NVFP4_OK)
+    return st;
   const int64_t tiles = ((M + 2 * nvfp4::tc::BM - 1) / (2 * nvfp4::tc::BM)) * num_n;
   const int pairs = static_cast<int>(tiles < info->pairs ? tiles : info->pairs);
   cfg.gridDim = dim3(2 * pairs, 1, 1);
@@ -752,33 +766,11 @@ nvfp4_status nvfp4_gate_up_silu_quantize(const void* a_codes, const void* a_scal
   if ((st = scale_map(a_scales, M, K, 1, dev, &tsa)) != NVFP4_OK) return st;
   if ((st = scale_map(w_scales, 2 * H, K, 1, dev, &tsb)) != NVFP4_OK) return st;
 
-  constexpr int smem = nvfp4::tc::Cfg<2>::SMEM_BYTES;
-  cudaLaunchConfig_t cfg = {};
+  cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.blockDim = dim3(nvfp4::tc::THREADS, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = cs;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (!info->attr_tc2_swiglu) {
-    if (cudaFuncSetAttribute(nvfp4::k_gemm_tc<2, true>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return NVFP4_ERR_CUDA;
-    cfg.gridDim = dim3(2 * (info->sms / 2), 1, 1);
-    int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, nvfp4::k_gemm_tc<2, true>, &cfg) !=
-            cudaSuccess ||
-        clusters < 1) {
-      cudaGetLastError();
-      return NVFP4_ERR_CUDA;
-    }
-    info->swiglu_pairs = clusters;
-    info->attr_tc2_swiglu = true;
-  }
+  if ((st = pair_config(nvfp4::k_gemm_tc<2, true>, info, &info->attr_tc2_swiglu,
+                        &info->swiglu_pairs, cs, &cfg, attr)) != NVFP4_OK)
+    return st;
   const int64_t tiles = ((M + 2 * nvfp4::tc::BM - 1) / (2 * nvfp4::tc::BM)) * (H / 128);
   const int pairs = static_cast<int>(tiles < info->swiglu_pairs ? tiles : info->swiglu_pairs);
   cfg.gridDim = dim3(2 * pairs, 1, 1);
