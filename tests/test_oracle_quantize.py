@@ -117,3 +117,40 @@ def test_workload_calibration_scales():
     gs = oracle.global_scale(np.abs(xc).max())
     assert np.isfinite(gs) and gs > 0
     assert gs == np.float32(np.float32(np.abs(xc).max()) / np.float32(2688.0))
+
+
+def test_global_scale_by_a_power_of_two_leaves_the_values_unchanged():
+    """A global scale 4x larger quarters every block scale exactly (E4M3 is a
+    binary float format) and leaves the block reciprocal, hence every code and
+    every dequantised value, unchanged -- as long as no block scale leaves the
+    normal E4M3 range.  So the global scale sets only the block scales' range:
+    one shared scale for all modules of a fused weight (the pages' pre-
+    harmonised checkpoint: aimodeling, "What engineers should actually take
+    away") costs no precision beyond where a block scale rounds."""
+    rng = np.random.default_rng(11)
+    x = rng.normal(0, 1, (64, 256)).astype(np.float32)
+    gs = oracle.global_scale(np.abs(x).max())
+    q1, s1 = oracle.quantize(x, gs)
+    q4, s4 = oracle.quantize(x, np.float32(gs * 4))
+    d1, d4 = oracle.e4m3_decode(s1), oracle.e4m3_decode(s4)
+    assert d1.min() / 4 >= 2.0 ** -6                  # quartered scales stay normal E4M3
+    np.testing.assert_array_equal(d4 * 4, d1)
+    np.testing.assert_array_equal(q4, q1)
+    np.testing.assert_array_equal(oracle.dequantize(q4, s4, np.float32(gs * 4)),
+                                  oracle.dequantize(q1, s1, gs))
+
+
+def test_shared_global_scale_across_modules_costs_no_precision():
+    """Modules with the GDN in-projection's spread of weight stds (log-uniform
+    over 0.25..4 of 1/sqrt(K)), each quantised under its own global scale or
+    under the largest one: the relative errors agree within 2%."""
+    rng = np.random.default_rng(12)
+    K = 512
+    stds = np.array([0.25, 0.5, 1.0, 2.0, 4.0]) / np.sqrt(K)
+    mods = [rng.normal(0, s, (64, K)).astype(np.float32) for s in stds]
+    gs_shared = oracle.global_scale(max(np.abs(m).max() for m in mods))
+    for m in mods:
+        gs = oracle.global_scale(np.abs(m).max())
+        own = np.linalg.norm(oracle.dequantize(*oracle.quantize(m, gs), gs) - m)
+        shared = np.linalg.norm(oracle.dequantize(*oracle.quantize(m, gs_shared), gs_shared) - m)
+        assert abs(shared / own - 1.0) < 0.02
