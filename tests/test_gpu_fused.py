@@ -174,3 +174,45 @@ def test_silu_mul_matches_the_oracle_within_one_bf16_step():
     step = np.abs(ref).astype(np.float64) * 2.0 ** -7 + 1e-30
     assert np.all(np.abs(h.astype(np.float64) - ref) <= step)
     assert np.mean(h == ref) > 0.99
+
+
+@pytest.mark.parametrize("path,M,K", [(PAIR, 200, 320), (SMALL, 7, 320), (LARGE, 100, 256)])
+def test_preharmonised_checkpoint(path, M, K):
+    """The pages' other repair: every module of the fused weight quantised under
+    one shared global scale ("pre-harmonised"), served with that scale in every
+    segment; gates still apply per module."""
+    widths, ops, wbits, xbits, a_log, dt = _mini_gdn(M, K, seed=M + 5)
+    N = sum(widths)
+    offs = np.cumsum([0] + widths[:-1]).tolist()
+    xf, wf = H.f32(xbits), H.f32(wbits)
+    a_gs = oracle.global_scale(np.abs(xf).max())
+    ac, as_ = nv.nvfp4_quantize_act(H.bf16_dev(xbits), float(a_gs))
+    wc, ws, (w_gs,) = nv.nvfp4_quantize_weight(H.bf16_dev(wbits))          # one module
+    gs_ref = oracle.global_scale(np.abs(wf).max())
+    assert np.float32(w_gs) == gs_ref
+    a_log_d, dt_d = torch.from_numpy(a_log).cuda(), torch.from_numpy(dt).cuda()
+    specs = [nv.SegmentSpec(o, w_gs, float(a_gs), OPS[ops[i]],
+                            a_log_d if ops[i] == "gdn_decay" else None,
+                            dt_d if ops[i] == "gdn_decay" else None)
+             for i, o in enumerate(offs)]
+    nv.nvfp4_set_gemm_path(path)
+    y32 = nv.nvfp4_fused_linear(ac, as_, wc, ws, M, N, K, specs, out_dtype=nv.OUT_FP32)
+    assert nv.nvfp4_last_device_error()[0] == 0
+    y32 = y32.cpu().numpy()
+    qx, sx = oracle.quantize(xf, a_gs)
+    qw, sw = oracle.quantize(wf, gs_ref)
+    np.testing.assert_array_equal(H.unpack_codes(wc.cpu().numpy()), qw)
+    segs = [dict(n_offset=o, width=wd, w_gs=gs_ref, a_gs=a_gs, op=ops[i], a_log=a_log, dt_bias=dt)
+            for i, (o, wd) in enumerate(zip(offs, widths))]
+    ref = oracle.fused_linear64(qx, sx, qw, sw, segs)
+    pre = oracle.fused_linear64(qx, sx, qw, sw, [dict(s, op="none") for s in segs])
+    for o, wd, op in zip(offs, widths, ops):
+        sl = slice(o, o + wd)
+        e = 1e-3 * np.sqrt(np.mean(pre[:, sl] ** 2))
+        if op == "none":
+            H.check_gemm_fp32(y32[:, sl], ref[:, sl], f"harmonised segment at {o}")
+        elif op == "sigmoid":
+            assert np.all(np.abs(y32[:, sl] - ref[:, sl]) <= 0.25 * e + 2e-6)
+        else:
+            bound = np.exp(a_log)[None, :] * e + 2e-5 * np.abs(ref[:, sl]) + 1e-6
+            assert np.all(np.abs(y32[:, sl] - ref[:, sl]) <= bound)
