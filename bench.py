@@ -473,6 +473,26 @@ def small_m_sweep(device, stream, iters=240, warmup=10):
 
 
 # ------------------------------------------------------------ CPU oracle
+def kv_fp8_rate(device, stream, reps=20):
+    """FP8 KV-cache quantisation of one layer's K (32768 tokens x 8 heads x
+    128 dims, bf16 -> E4M3 under a calibrated scale), rotated over 3 copies
+    (201 MB > L2): graph replay of GRAPH_STEPS launches.  3 bytes per element."""
+    import nvfp4_w4a4_quantized_quantizer_b200 as nv
+    n = 32768 * 8 * 128
+    rng = np.random.default_rng(3)
+    x0 = torch.from_numpy(rng.standard_normal(n).astype(np.float32)).to(device).to(torch.bfloat16)
+    xs = [x0] + [x0.clone() for _ in range(2)]
+    out = torch.empty(n, dtype=torch.uint8, device=device)
+    s = nv.nvfp4_kv_scale(float(x0.float().abs().max().item()))
+
+    def run(i, st):
+        nv.nvfp4_kv_quantize_fp8(xs[i % 3], s, out=out, stream=st)
+
+    t = time_each({"kv": run}, reps, stream)["kv"]
+    gbs = 3.0 * n / (t * 1e-3) / 1e9
+    return {"elements": n, "us": round(t * 1e3, 2), "GBps": round(gbs, 1)}
+
+
 class OracleSample:
     """The oracle, as it stands, on bounded samples of the workload: quantise a
     few activation rows, dequantise, float64 GEMM against the dequantised
@@ -666,6 +686,10 @@ def main():
         for v in sm.values():
             v["hbm_frac"] = round(v["weight_GBps"] / pk["hbm"], 4)
         line["small_m"] = sm
+    if rank == 0 and not args.no_small_m and ws == 1:
+        kv = kv_fp8_rate(device, stream)
+        kv["hbm_frac"] = round(kv["GBps"] / pk["hbm"], 4)
+        line["kv_fp8"] = kv
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     if rank == 0:

@@ -279,6 +279,20 @@ nvfp4_status nvfp4_gate_up_silu_quantize(const void* a_codes, const void* a_scal
 nvfp4_status nvfp4_silu_mul(const void* gu_bf16, int64_t M, int64_t H, int64_t ld_in,
                             void* h_bf16, int64_t ld_out, nvfp4_stream_t stream);
 
+/* FP8 KV cache: the pages' other shipped recipe, calibrated per-tensor FP8
+ * E4M3 KV-cache scales ("quantize everything, ship KV scales": nefut
+ * abstract; aimodeling, "What engineers should actually take away").
+ * nvfp4_kv_scale: fp32(amax) / 448 of a calibration batch (1 when amax <= 0;
+ * amax from nvfp4_amax).  nvfp4_kv_quantize_fp8: out[i] = sign(x[i]) |
+ * E4M3_RNE_satfinite(|fp32(x[i] * fp32(1 / scale))|) for n bf16 values x
+ * (device, 16-byte aligned; n % 8 == 0) into n bytes of out (device,
+ * 16-byte aligned); values past the calibrated range saturate at +-448 and
+ * zeros keep their sign.  Caller-owned buffers; violations return before any
+ * launch; queued on `stream`. */
+float nvfp4_kv_scale(float amax);
+nvfp4_status nvfp4_kv_quantize_fp8(const void* x_bf16, int64_t n, float scale, void* out_e4m3,
+                                   nvfp4_stream_t stream);
+
 /* Human-readable status. */
 const char* nvfp4_status_string(nvfp4_status status);
 

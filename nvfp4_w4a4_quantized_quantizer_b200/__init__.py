@@ -22,7 +22,7 @@ __all__ = [
     "nvfp4_quantize_act", "nvfp4_quantize_weight", "nvfp4_quantize_weight_noalloc",
     "nvfp4_linear", "nvfp4_fused_linear", "nvfp4_gemm_workspace_bytes", "nvfp4_gemm_workspace",
     "nvfp4_gate_up_silu_quantize", "nvfp4_silu_mul", "nvfp4_last_device_error", "nvfp4_set_gemm_path",
-    "nvfp4_set_launch_overlap",
+    "nvfp4_set_launch_overlap", "nvfp4_kv_scale", "nvfp4_kv_quantize_fp8",
     "nvfp4_set_wait_limit_ns", "nvfp4_test_e2m1", "nvfp4_test_e4m3", "nvfp4_test_wait_timeout",
     "SegmentSpec", "NVFP4Error", "OP_NONE", "OP_SIGMOID", "OP_GDN_DECAY",
 ]
@@ -202,6 +202,22 @@ def nvfp4_gate_up_silu_quantize(a_codes, a_scales, w_codes, w_scales, M: int, H:
         ctypes.c_float(h_gs), _ptr(h_codes), _ptr(h_scales), _stream(stream)),
         "nvfp4_gate_up_silu_quantize")
     return h_codes, h_scales
+
+
+def nvfp4_kv_scale(amax: float) -> float:
+    return load().nvfp4_kv_scale(ctypes.c_float(amax))
+
+
+def nvfp4_kv_quantize_fp8(x: torch.Tensor, scale: float, out: Optional[torch.Tensor] = None,
+                          stream=None) -> torch.Tensor:
+    """bf16 tensor (contiguous, numel % 8 == 0) -> E4M3 codes (uint8, same shape)."""
+    if not x.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    check(load().nvfp4_kv_quantize_fp8(_ptr(x), x.numel(), ctypes.c_float(scale), _ptr(out),
+                                       _stream(stream)), "nvfp4_kv_quantize_fp8")
+    return out
 
 
 def nvfp4_silu_mul(gu: torch.Tensor, H: int, h: Optional[torch.Tensor] = None,

@@ -814,6 +814,27 @@ nvfp4_status nvfp4_silu_mul(const void* gu, int64_t M, int64_t H, int64_t ld_in,
   return check_launch();
 }
 
+float nvfp4_kv_scale(float amax) { return amax > 0.0f ? amax / 448.0f : 1.0f; }
+
+nvfp4_status nvfp4_kv_quantize_fp8(const void* x, int64_t n, float scale, void* out,
+                                   nvfp4_stream_t stream) {
+  if (x == nullptr || out == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (n < 0 || n % 8 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(x) || !aligned16(out)) return NVFP4_ERR_ALIGNMENT;
+  if (!good_scale(scale)) return NVFP4_ERR_INVALID_ARG;
+  if (n == 0) return NVFP4_OK;
+  int dev;
+  DeviceInfo* info;
+  nvfp4_status st = current_device(&dev, &info);
+  if (st != NVFP4_OK) return st;
+  volatile float one = 1.0f;
+  const float r = one / scale;   // fp32(1 / scale), IEEE division
+  const int grid = grid_for(n / 8, nvfp4::KV_THREADS, info->sms * 8);
+  nvfp4::k_kv_fp8<<<grid, nvfp4::KV_THREADS, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x), n / 8, r, static_cast<uint2*>(out));
+  return check_launch();
+}
+
 nvfp4_status nvfp4_test_e2m1(const float* in, uint8_t* out, int64_t n, nvfp4_stream_t stream) {
   if (in == nullptr || out == nullptr || n < 0) return NVFP4_ERR_INVALID_ARG;
   if (n == 0) return NVFP4_OK;

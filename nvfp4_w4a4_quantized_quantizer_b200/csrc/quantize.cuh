@@ -370,6 +370,37 @@ __global__ void __launch_bounds__(SILU_THREADS) k_silu_mul(const __nv_bfloat16* 
   }
 }
 
+// ------------------------------------------------------ FP8 (E4M3) KV cache
+// The pages' other shipped recipe: KV-cache tensors in FP8 E4M3 under a
+// calibrated per-tensor scale.  code = sign | E4M3_RNE_satfinite(fp32(x * r))
+// with r = fp32(1 / scale) formed on the host; eight bf16 in (16 bytes),
+// eight codes out (8 bytes) per thread and step.  HBM-bound.
+constexpr int KV_THREADS = 256;
+
+// Two fp32 values -> two E4M3 codes, a in the low byte (the PTX conversion
+// puts its first source in the high byte).
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float a, float b) {
+  uint16_t out;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(b), "f"(a));
+  return static_cast<uint32_t>(out);
+}
+
+__global__ void __launch_bounds__(KV_THREADS) k_kv_fp8(const __nv_bfloat16* __restrict__ x,
+                                                       int64_t n8, float r,
+                                                       uint2* __restrict__ out) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * KV_THREADS + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * KV_THREADS) {
+    float f[8];
+    bf16x8_to_f32(ld_stream_v4(x + i * 8), f);
+    uint32_t w[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      w[h] = cvt_e4m3x2(__fmul_rn(f[4 * h], r), __fmul_rn(f[4 * h + 1], r)) |
+             (cvt_e4m3x2(__fmul_rn(f[4 * h + 2], r), __fmul_rn(f[4 * h + 3], r)) << 16);
+    out[i] = make_uint2(w[0], w[1]);
+  }
+}
+
 // ------------------------------------------------------------ test kernels
 __global__ void k_test_e2m1(const float* in, uint8_t* out, int64_t n) {
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;

@@ -24,6 +24,9 @@ Pinning status (what each function is checked against in ``tests/``):
   sigmoid64 / gdn_decay64    -- Lipschitz bounds, limits, closed values
   silu_mul_bf16              -- ml_dtypes bfloat16 RNE (random and exact ties),
                                 closed values and limits of SiLU
+  kv_quantize / kv_scale /
+  kv_dequantize              -- ml_dtypes.float8_e4m3fn on every finite bf16
+                                value, saturation and signed zeros by hand
 No function is "parity unpinned".
 """
 from .nvfp4 import (  # noqa: F401
@@ -31,3 +34,4 @@ from .nvfp4 import (  # noqa: F401
     global_scale, quantize, dequantize, pack_codes, linear64, fused_linear64,
     fused_linear64_shared_scale, sigmoid64, gdn_decay64, silu_mul_bf16,
 )
+from .kv import kv_scale, kv_quantize, kv_dequantize  # noqa: F401

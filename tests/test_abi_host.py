@@ -154,6 +154,19 @@ def test_gate_up_silu_quantize_validation(lib):
     assert f(*args(M=0)) == 0
 
 
+def test_kv_fp8_validation(lib):
+    assert lib.nvfp4_kv_scale(ctypes.c_float(448.0)) == 1.0
+    assert lib.nvfp4_kv_scale(ctypes.c_float(0.0)) == 1.0
+    q = lib.nvfp4_kv_quantize_fp8
+    assert q(NUL, 8, 1.0, P, NUL) == INVALID
+    assert q(P, 12, 1.0, P, NUL) == SHAPE                     # n % 8
+    assert q(P, -8, 1.0, P, NUL) == SHAPE
+    assert q(P_MIS, 8, 1.0, P, NUL) == ALIGN
+    assert q(P, 8, 1.0, P_MIS, NUL) == ALIGN
+    assert q(P, 8, 0.0, P, NUL) == INVALID
+    assert q(P, 0, 1.0, P, NUL) == 0
+
+
 def test_misc_validation(lib):
     assert lib.nvfp4_set_gemm_path(5) == INVALID
     assert lib.nvfp4_set_gemm_path(0) == 0
