@@ -293,6 +293,23 @@ float nvfp4_kv_scale(float amax);
 nvfp4_status nvfp4_kv_quantize_fp8(const void* x_bf16, int64_t n, float scale, void* out_e4m3,
                                    nvfp4_stream_t stream);
 
+/* Gated DeltaNet state recurrence over T tokens of one sequence (the step
+ * after the GDN in-projection; the pages' third mechanism: each write
+ * overwrites the state along its key direction -- bayesiansapien wiki, "The
+ * four-part mechanism study", part 3; the formula is the published gated
+ * delta rule):  S_t = exp(g_t) S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t
+ * k_t^T,  o_t = S_t q_t, per value head.  Device fp32 arrays, token-major:
+ * q, k [T, Hv/group, 128] (k rows of unit length), v and o [T, Hv, 128],
+ * g (log decay, <= 0) and beta [T, Hv], state [Hv, 128 (value), 128 (key)]
+ * holding the initial state on entry and the final state on return.  Value
+ * head h reads key head h / group.  head_dim must be 128; pointers 16-byte
+ * aligned.  Computed chunk by chunk (64 tokens) in fp32.  Queued on
+ * `stream`. */
+nvfp4_status nvfp4_gdn_recurrence(const float* q, const float* k, const float* v,
+                                  const float* g, const float* beta, int64_t T, int32_t Hv,
+                                  int32_t group, int32_t head_dim, float* o, float* state,
+                                  nvfp4_stream_t stream);
+
 /* Human-readable status. */
 const char* nvfp4_status_string(nvfp4_status status);
 

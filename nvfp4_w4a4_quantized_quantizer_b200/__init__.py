@@ -21,8 +21,8 @@ __all__ = [
     "nvfp4_codes_bytes", "nvfp4_scale_bytes", "nvfp4_global_scale", "nvfp4_amax",
     "nvfp4_quantize_act", "nvfp4_quantize_weight", "nvfp4_quantize_weight_noalloc",
     "nvfp4_linear", "nvfp4_fused_linear", "nvfp4_gemm_workspace_bytes", "nvfp4_gemm_workspace",
-    "nvfp4_gate_up_silu_quantize", "nvfp4_silu_mul", "nvfp4_last_device_error", "nvfp4_set_gemm_path",
-    "nvfp4_set_launch_overlap", "nvfp4_kv_scale", "nvfp4_kv_quantize_fp8",
+    "nvfp4_gate_up_silu_quantize", "nvfp4_gdn_recurrence", "nvfp4_silu_mul", "nvfp4_last_device_error",
+    "nvfp4_set_gemm_path", "nvfp4_set_launch_overlap", "nvfp4_kv_scale", "nvfp4_kv_quantize_fp8",
     "nvfp4_set_wait_limit_ns", "nvfp4_test_e2m1", "nvfp4_test_e4m3", "nvfp4_test_wait_timeout",
     "SegmentSpec", "NVFP4Error", "OP_NONE", "OP_SIGMOID", "OP_GDN_DECAY",
 ]
@@ -218,6 +218,25 @@ def nvfp4_kv_quantize_fp8(x: torch.Tensor, scale: float, out: Optional[torch.Ten
     check(load().nvfp4_kv_quantize_fp8(_ptr(x), x.numel(), ctypes.c_float(scale), _ptr(out),
                                        _stream(stream)), "nvfp4_kv_quantize_fp8")
     return out
+
+
+def nvfp4_gdn_recurrence(q, k, v, g, beta, group: int = 1, state: Optional[torch.Tensor] = None,
+                         o: Optional[torch.Tensor] = None, stream=None):
+    """Gated delta rule over one sequence: q, k [T, Hk, 128], v [T, Hv, 128], g and beta
+    [T, Hv] (fp32, contiguous).  Returns (o [T, Hv, 128], final state [Hv, 128, 128]);
+    `state` (initial state, updated in place) defaults to zeros."""
+    T, Hv, D = v.shape
+    for t in (q, k, v, g, beta):
+        if t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError("expected contiguous float32 tensors")
+    if state is None:
+        state = torch.zeros((Hv, D, D), dtype=torch.float32, device=v.device)
+    if o is None:
+        o = torch.empty((T, Hv, D), dtype=torch.float32, device=v.device)
+    check(load().nvfp4_gdn_recurrence(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), T, Hv, group,
+                                      D, _ptr(o), _ptr(state), _stream(stream)),
+          "nvfp4_gdn_recurrence")
+    return o, state
 
 
 def nvfp4_silu_mul(gu: torch.Tensor, H: int, h: Optional[torch.Tensor] = None,

@@ -51,6 +51,7 @@ SIGNATURES = {
     "nvfp4_silu_mul": (_st, [_vp, _i64, _i64, _i64, _vp, _i64, _vp]),
     "nvfp4_kv_scale": (_f32, [_f32]),
     "nvfp4_kv_quantize_fp8": (_st, [_vp, _i64, _f32, _vp, _vp]),
+    "nvfp4_gdn_recurrence": (_st, [_vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp]),
     "nvfp4_status_string": (ctypes.c_char_p, [_st]),
     "nvfp4_last_device_error": (_st, [_vp, ctypes.POINTER(ctypes.c_uint64)]),
     "nvfp4_set_gemm_path": (_st, [_i32]),

@@ -15,6 +15,7 @@
 #include <unordered_map>
 
 #include "nvfp4.h"
+#include "gdn.cuh"
 #include "gemm.cuh"
 #include "quantize.cuh"
 
@@ -72,6 +73,7 @@ struct DeviceInfo {
   bool attr_tc = false;
   bool attr_tc2 = false;
   bool attr_tc2_swiglu = false;
+  bool attr_gdn = false;
   int quant_blocks = 0;   // resident k_quantize blocks per SM
   int pairs = 0;          // co-resident clusters of two CTAs of k_gemm_tc<2>
   int swiglu_pairs = 0;   // the same for k_gemm_tc<2, true>
@@ -832,6 +834,47 @@ nvfp4_status nvfp4_kv_quantize_fp8(const void* x, int64_t n, float scale, void* 
   const int grid = grid_for(n / 8, nvfp4::KV_THREADS, info->sms * 8);
   nvfp4::k_kv_fp8<<<grid, nvfp4::KV_THREADS, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<const __nv_bfloat16*>(x), n / 8, r, static_cast<uint2*>(out));
+  return check_launch();
+}
+
+nvfp4_status nvfp4_gdn_recurrence(const float* q, const float* k, const float* v, const float* g,
+                                  const float* beta, int64_t T, int32_t Hv, int32_t group,
+                                  int32_t head_dim, float* o, float* state,
+                                  nvfp4_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || g == nullptr || beta == nullptr ||
+      o == nullptr || state == nullptr)
+    return NVFP4_ERR_INVALID_ARG;
+  if (T < 0 || Hv < 1 || group < 1 || Hv % group != 0 || head_dim != nvfp4::gdn::D)
+    return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  for (const void* p : {static_cast<const void*>(q), static_cast<const void*>(k),
+                        static_cast<const void*>(v), static_cast<const void*>(o),
+                        static_cast<const void*>(state)})
+    if (!aligned16(p)) return NVFP4_ERR_ALIGNMENT;
+  int dev;
+  DeviceInfo* info;
+  nvfp4_status st = current_device(&dev, &info);
+  if (st != NVFP4_OK) return st;
+  if (!info->attr_gdn) {
+    if (cudaFuncSetAttribute(nvfp4::k_gdn_chunked, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             nvfp4::gdn::SMEM_BYTES) != cudaSuccess) {
+      cudaGetLastError();
+      return NVFP4_ERR_CUDA;
+    }
+    info->attr_gdn = true;
+  }
+  nvfp4::GdnArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.g = g;
+  a.beta = beta;
+  a.o = o;
+  a.state = state;
+  a.T = T;
+  a.Hv = Hv;
+  a.group = group;
+  nvfp4::k_gdn_chunked<<<Hv, nvfp4::gdn::THREADS, nvfp4::gdn::SMEM_BYTES,
+                         reinterpret_cast<cudaStream_t>(stream)>>>(a);
   return check_launch();
 }
 

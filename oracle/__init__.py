@@ -27,6 +27,12 @@ Pinning status (what each function is checked against in ``tests/``):
   kv_quantize / kv_scale /
   kv_dequantize              -- ml_dtypes.float8_e4m3fn on every finite bf16
                                 value, saturation and signed zeros by hand
+  gdn_recurrence_seq         -- exact overwrite along the key, decay-only action
+                                orthogonal to it, gradient step on the key-value
+                                loss (finite differences)
+  gdn_recurrence_chunked     -- equals gdn_recurrence_seq (ragged chunks)
+  gdn_error_contraction /
+  gdn_noise_plateau          -- simulated impulse decay and noise plateau
 No function is "parity unpinned".
 """
 from .nvfp4 import (  # noqa: F401
@@ -35,3 +41,7 @@ from .nvfp4 import (  # noqa: F401
     fused_linear64_shared_scale, sigmoid64, gdn_decay64, silu_mul_bf16,
 )
 from .kv import kv_scale, kv_quantize, kv_dequantize  # noqa: F401
+from .gdn import (  # noqa: F401
+    gdn_recurrence_seq, gdn_recurrence_chunked, gdn_error_contraction, gdn_noise_plateau,
+    gdn_error_trace,
+)
