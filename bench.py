@@ -493,6 +493,39 @@ def kv_fp8_rate(device, stream, reps=20):
     return {"elements": n, "us": round(t * 1e3, 2), "GBps": round(gbs, 1)}
 
 
+# fp32 FMA peak for ALU-bound kernels: 148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz
+FP32_ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def gdn_rate(device, stream, reps=4):
+    """The gated delta rule over 8192 tokens of the GDN in-projection's heads
+    (48 value heads over 16 key heads, width 128), graph replay.  FLOPs
+    counted as the definition's 6 D^2 per token and value head."""
+    import nvfp4_w4a4_quantized_quantizer_b200 as nv
+    T, Hv, group, D = 8192, 48, 3, 128
+    rng = np.random.default_rng(4)
+    f = lambda a: torch.from_numpy(a.astype(np.float32)).to(device)  # noqa: E731
+    k = rng.standard_normal((T, Hv // group, D))
+    ins = dict(q=f(rng.standard_normal((T, Hv // group, D))),
+               k=f(k / np.linalg.norm(k, axis=2, keepdims=True)),
+               v=f(rng.standard_normal((T, Hv, D))),
+               g=f(-np.log1p(np.exp(rng.normal(-2, 1, (T, Hv))))),
+               beta=f(1 / (1 + np.exp(-rng.normal(0, 1.5, (T, Hv))))))
+    state = torch.zeros((Hv, D, D), dtype=torch.float32, device=device)
+    o = torch.empty((T, Hv, D), dtype=torch.float32, device=device)
+
+    def run(i, st):
+        nv.nvfp4_gdn_recurrence(ins["q"], ins["k"], ins["v"], ins["g"], ins["beta"], group=group,
+                                state=state, o=o, stream=st)
+
+    t = time_each({"gdn": run}, reps, stream)["gdn"]
+    tflops = 6.0 * D * D * T * Hv / (t * 1e-3) / 1e12
+    return {"tokens": T, "value_heads": Hv, "us": round(t * 1e3, 1),
+            "tokens_per_s": round(T / (t * 1e-3), 1), "tflops": round(tflops, 2),
+            "bound": "alu", "peak_tflops": round(FP32_ALU_PEAK_TFLOPS, 1),
+            "frac": round(tflops / FP32_ALU_PEAK_TFLOPS, 4)}
+
+
 class OracleSample:
     """The oracle, as it stands, on bounded samples of the workload: quantise a
     few activation rows, dequantise, float64 GEMM against the dequantised
@@ -690,6 +723,7 @@ def main():
         kv = kv_fp8_rate(device, stream)
         kv["hbm_frac"] = round(kv["GBps"] / pk["hbm"], 4)
         line["kv_fp8"] = kv
+        line["gdn_recurrence"] = gdn_rate(device, stream)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     if rank == 0:
