@@ -873,7 +873,14 @@ nvfp4_status nvfp4_gdn_recurrence(const float* q, const float* k, const float* v
   a.T = T;
   a.Hv = Hv;
   a.group = group;
-  nvfp4::k_gdn_chunked<<<Hv, nvfp4::gdn::THREADS, nvfp4::gdn::SMEM_BYTES,
+  // value rows are independent: split each head over enough CTAs to fill the
+  // SMs in one wave (at most 8 parts of at least 16 rows)
+  int parts = info->sms / Hv;
+  if (parts < 1) parts = 1;
+  if (parts > 8) parts = 8;
+  a.rows = (nvfp4::gdn::D + parts - 1) / parts;
+  a.parts = (nvfp4::gdn::D + a.rows - 1) / a.rows;
+  nvfp4::k_gdn_chunked<<<Hv * a.parts, nvfp4::gdn::THREADS, nvfp4::gdn::SMEM_BYTES,
                          reinterpret_cast<cudaStream_t>(stream)>>>(a);
   return check_launch();
 }

@@ -14,10 +14,15 @@
 //   O_t = e^{G_t} S_0 q_t + sum_{j <= t} e^{G_t - G_j} (q_t . k_j) U_j
 //   S_C = e^{G_C} S_0 + sum_t e^{G_C - G_t} U_t k_t^T
 //
-// k_gdn_chunked: one CTA per (sequence, value head); the fp32 state and one
-// chunk's keys, queries and values stay in shared memory (182 KB); fp32
-// CUDA-core arithmetic.  A first correct form: the products are dense and
-// would belong on the tensor cores.
+// Each value row of S evolves on its own (S_i <- alpha S_i (I - beta k k^T)
+// + beta v_i k^T reads only the keys, beta and g), so a head splits across
+// CTAs by value rows; only the key products (A, and Q K^T) are computed by
+// every CTA of the head.
+//
+// k_gdn_chunked: one CTA per (value head, block of value rows); the fp32
+// state rows and one chunk's keys, queries and value columns stay in shared
+// memory (at most 182 KB); fp32 CUDA-core arithmetic.  A first correct form:
+// the products are dense and would belong on the tensor cores.
 #pragma once
 
 #include <cstdint>
@@ -43,27 +48,31 @@ struct GdnArgs {
   float* state;        // [Hv, D (value), D (key)]: initial state in, final state out
   int64_t T;
   int Hv, group;       // value heads; value heads per key head (Hk = Hv / group)
+  int parts;           // CTAs per head, each with rows [p * rows, min(D, (p + 1) * rows))
+  int rows;
 };
 
 __global__ void __launch_bounds__(gdn::THREADS, 1) k_gdn_chunked(const GdnArgs a) {
   using namespace gdn;
   extern __shared__ __align__(16) float gsm[];
-  float* S = gsm;                   // [D value][LD key]
+  float* S = gsm;                   // [rn value rows][LD key]
   float* Kc = S + D * LD;           // [C][LD]
   float* Qc = Kc + C * LD;          // [C][LD]
-  float* Vc = Qc + C * LD;          // [C][D]: values, then the right-hand side, then U
+  float* Vc = Qc + C * LD;          // [C][rn]: values, then the right-hand side, then U
   float* A = Vc + C * D;            // [C][C]: A, then the masked, scaled Q K^T
   float* G = A + C * C;             // [C] running log decay
   float* B = G + C;                 // [C] beta
   float* E = B + C;                 // [C] e^{G_t}
   float* W = E + C;                 // [C] e^{G_last - G_t}
-  const int h = blockIdx.x;         // value head
+  const int h = blockIdx.x / a.parts;          // value head
+  const int r0 = (blockIdx.x % a.parts) * a.rows;
+  const int rn = min(D, r0 + a.rows) - r0;      // this CTA's value rows [r0, r0 + rn)
   const int hk = h / a.group;
   const int Hk = a.Hv / a.group;
   const int tid = threadIdx.x;
+  float* state = a.state + (static_cast<int64_t>(h) * D + r0) * D;
 
-  for (int x = tid; x < D * D; x += THREADS)
-    S[(x / D) * LD + x % D] = a.state[static_cast<int64_t>(h) * D * D + x];
+  for (int x = tid; x < rn * D; x += THREADS) S[(x / D) * LD + x % D] = state[x];
 
   for (int64_t c0 = 0; c0 < a.T; c0 += C) {
     const int cn = static_cast<int>(a.T - c0 < C ? a.T - c0 : C);
@@ -74,7 +83,10 @@ __global__ void __launch_bounds__(gdn::THREADS, 1) k_gdn_chunked(const GdnArgs a
       const int64_t tok = c0 + t;
       Kc[t * LD + d] = live ? a.k[(tok * Hk + hk) * D + d] : 0.0f;
       Qc[t * LD + d] = live ? a.q[(tok * Hk + hk) * D + d] : 0.0f;
-      Vc[x] = live ? a.v[(tok * a.Hv + h) * D + d] : 0.0f;
+    }
+    for (int x = tid; x < C * rn; x += THREADS) {
+      const int t = x / rn, i = x - t * rn;
+      Vc[x] = t < cn ? a.v[((c0 + t) * a.Hv + h) * D + r0 + i] : 0.0f;
     }
     if (tid < 32) {
       // running sum of g over the chunk: 64 values, two per lane
@@ -108,21 +120,21 @@ __global__ void __launch_bounds__(gdn::THREADS, 1) k_gdn_chunked(const GdnArgs a
       }
       A[x] = acc;
     }
-    // right-hand side: beta_t v_t - beta_t e^{G_t} S_0 k_t
-    for (int x = tid; x < C * D; x += THREADS) {
-      const int t = x / D, i = x - t * D;
+    // right-hand side: beta_t v_t - beta_t e^{G_t} S_0 k_t (this CTA's rows)
+    for (int x = tid; x < C * rn; x += THREADS) {
+      const int t = x / rn, i = x - t * rn;
       float sk = 0.0f;
       for (int d = 0; d < D; ++d) sk = fmaf(S[i * LD + d], Kc[t * LD + d], sk);
       Vc[x] = B[t] * Vc[x] - B[t] * E[t] * sk;
     }
     __syncthreads();
     // (I + A) U = rhs by forward substitution; thread i owns column i
-    if (tid < D) {
+    if (tid < rn) {
       const int i = tid;
       for (int t = 1; t < cn; ++t) {
-        float acc = Vc[t * D + i];
-        for (int j = 0; j < t; ++j) acc = fmaf(-A[t * C + j], Vc[j * D + i], acc);
-        Vc[t * D + i] = acc;
+        float acc = Vc[t * rn + i];
+        for (int j = 0; j < t; ++j) acc = fmaf(-A[t * C + j], Vc[j * rn + i], acc);
+        Vc[t * rn + i] = acc;
       }
     }
     __syncthreads();
@@ -138,29 +150,28 @@ __global__ void __launch_bounds__(gdn::THREADS, 1) k_gdn_chunked(const GdnArgs a
     }
     __syncthreads();
     // o_t = e^{G_t} S_0 q_t + sum_j P_tj U_j
-    for (int x = tid; x < cn * D; x += THREADS) {
-      const int t = x / D, i = x - t * D;
+    for (int x = tid; x < cn * rn; x += THREADS) {
+      const int t = x / rn, i = x - t * rn;
       float sq = 0.0f;
       for (int d = 0; d < D; ++d) sq = fmaf(S[i * LD + d], Qc[t * LD + d], sq);
       float pu = 0.0f;
-      for (int j = 0; j <= t; ++j) pu = fmaf(A[t * C + j], Vc[j * D + i], pu);
-      a.o[((c0 + t) * a.Hv + h) * D + i] = E[t] * sq + pu;
+      for (int j = 0; j <= t; ++j) pu = fmaf(A[t * C + j], Vc[j * rn + i], pu);
+      a.o[((c0 + t) * a.Hv + h) * D + r0 + i] = E[t] * sq + pu;
     }
     const float gc = G[cn - 1];
     if (tid < C) W[tid] = tid < cn ? expf(gc - G[tid]) : 0.0f;
     __syncthreads();   // every output of the chunk read the old state; W is ready
     // S = e^{G_C} S_0 + sum_t e^{G_C - G_t} U_t k_t^T
     const float ec = expf(gc);
-    for (int x = tid; x < D * D; x += THREADS) {
+    for (int x = tid; x < rn * D; x += THREADS) {
       const int i = x / D, j = x - i * D;
       float acc = ec * S[i * LD + j];
-      for (int t = 0; t < cn; ++t) acc = fmaf(Vc[t * D + i] * W[t], Kc[t * LD + j], acc);
+      for (int t = 0; t < cn; ++t) acc = fmaf(Vc[t * rn + i] * W[t], Kc[t * LD + j], acc);
       S[i * LD + j] = acc;
     }
   }
   __syncthreads();
-  for (int x = tid; x < D * D; x += THREADS)
-    a.state[static_cast<int64_t>(h) * D * D + x] = S[(x / D) * LD + x % D];
+  for (int x = tid; x < rn * D; x += THREADS) state[x] = S[(x / D) * LD + x % D];
 }
 
 }  // namespace nvfp4
