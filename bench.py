@@ -222,6 +222,8 @@ class Layer:
         self.scales = [torch.empty(nv.nvfp4_scale_bytes(M, self.K), dtype=torch.uint8, device=device)
                        for _ in range(2)]
         self.ys = [torch.empty((M, self.N), dtype=torch.bfloat16, device=device) for _ in range(2)]
+        # lets the CTA-pair GEMM split its last partial wave of tiles along K
+        self.work = nv.nvfp4_gemm_workspace(device)
         self.segs = []
         gate_dev = {}
         if any(s.op == "gdn_decay" for s in wl.segments):
@@ -241,7 +243,8 @@ class Layer:
     def gemm(self, i, stream):
         wc, ws = self.ws[i % len(self.ws)]
         self.nv.nvfp4_fused_linear(self.codes[i % 2], self.scales[i % 2], wc, ws, self.M, self.N,
-                                   self.K, self.segs, y=self.ys[i % 2], stream=stream)
+                                   self.K, self.segs, y=self.ys[i % 2], stream=stream,
+                                   workspace=self.work)
 
     @property
     def flops(self):
@@ -253,10 +256,10 @@ class Layer:
 
 
 class MlpChain:
-    """The MLP pair as one step: quantise x, gate_up (two modules, one fused
-    GEMM), h = bf16(SiLU(gate) * up), requantise h under its calibrated global
-    scale, down GEMM.  Activation copies rotate over 3, weight sets over 2
-    (working set > L2)."""
+    """The MLP pair as one step: quantise x; gate_up (two modules) with
+    h = bf16(SiLU(gate) * up) requantised under its calibrated global scale in
+    the same kernel; down GEMM.  Activation copies rotate over 3, weight sets
+    over 2 (working set > L2)."""
 
     def __init__(self, device, rotate_act=3, rotate_w=2):
         import nvfp4_w4a4_quantized_quantizer_b200 as nv
@@ -277,51 +280,46 @@ class MlpChain:
         w2c, w2s, (self.w2_gs,) = nv.nvfp4_quantize_weight(w2bits)
         del w2bits
         self.segs = [nv.SegmentSpec(off, g, self.a_gs) for off, g in zip(wl.seg_offsets, self.w_gs)]
+        self.work = nv.nvfp4_gemm_workspace(device)
         # the down input's static global scale: the chain on the calibration batch
         cc, cs = nv.nvfp4_quantize_act(calib, self.a_gs)
         gu_cal = nv.nvfp4_fused_linear(cc, cs, wc, ws, calib.shape[0], self.N, self.K, self.segs)
         h_cal = nv.nvfp4_silu_mul(gu_cal, self.H)
         self.a2_gs = nv.nvfp4_global_scale(nv.nvfp4_amax(h_cal).item())
+        self.segs2 = [nv.SegmentSpec(0, self.w2_gs, self.a2_gs)]
         del calib, cc, cs, gu_cal, h_cal
         self.ws = [(wc, ws, w2c, w2s)] + [tuple(t.clone() for t in (wc, ws, w2c, w2s))
                                           for _ in range(rotate_w - 1)]
         self.xc = torch.empty((self.M, self.K // 2), dtype=torch.uint8, device=device)
         self.xsc = torch.empty(nv.nvfp4_scale_bytes(self.M, self.K), dtype=torch.uint8, device=device)
-        self.gu = torch.empty((self.M, self.N), dtype=torch.bfloat16, device=device)
-        self.h = torch.empty((self.M, self.H), dtype=torch.bfloat16, device=device)
         self.hc = torch.empty((self.M, self.H // 2), dtype=torch.uint8, device=device)
         self.hsc = torch.empty(nv.nvfp4_scale_bytes(self.M, self.H), dtype=torch.uint8, device=device)
-        self.y = torch.empty((self.M, self.N2), dtype=torch.bfloat16, device=device)
-        self.ys = [self.y, self.y]
+        # two output buffers: a step's read-back may overlap the next step's kernels
+        self.ys = [torch.empty((self.M, self.N2), dtype=torch.bfloat16, device=device)
+                   for _ in range(2)]
 
     def quantize(self, i, stream, x=None):
         xx = self.xs[i % len(self.xs)] if x is None else x
         self.nv.nvfp4_quantize_act(xx, self.a_gs, codes=self.xc, scales=self.xsc, stream=stream)
 
     def gate_up(self, i, stream):
+        """gate_up GEMM + SiLU(gate) * up + requantisation of h, one kernel."""
         wc, ws, _, _ = self.ws[i % len(self.ws)]
-        self.nv.nvfp4_fused_linear(self.xc, self.xsc, wc, ws, self.M, self.N, self.K, self.segs,
-                                   y=self.gu, stream=stream)
-
-    def silu(self, i, stream):
-        self.nv.nvfp4_silu_mul(self.gu, self.H, h=self.h, stream=stream)
-
-    def requantize(self, i, stream):
-        self.nv.nvfp4_quantize_act(self.h, self.a2_gs, codes=self.hc, scales=self.hsc, stream=stream)
+        self.nv.nvfp4_gate_up_silu_quantize(self.xc, self.xsc, wc, ws, self.M, self.H, self.K,
+                                            self.a_gs, self.w_gs[0], self.w_gs[1], self.a2_gs,
+                                            h_codes=self.hc, h_scales=self.hsc, stream=stream)
 
     def down(self, i, stream):
         _, _, w2c, w2s = self.ws[i % len(self.ws)]
-        self.nv.nvfp4_linear(self.hc, self.hsc, self.a2_gs, w2c, w2s, self.w2_gs, self.M, self.N2,
-                             self.H, y=self.y, stream=stream)
+        self.nv.nvfp4_fused_linear(self.hc, self.hsc, w2c, w2s, self.M, self.N2, self.H, self.segs2,
+                                   y=self.ys[i % 2], stream=stream, workspace=self.work)
 
     def gemm(self, i, stream):
         """Everything after the first quantisation."""
         self.gate_up(i, stream)
-        self.silu(i, stream)
-        self.requantize(i, stream)
         self.down(i, stream)
 
-    launches_per_step = 5
+    launches_per_step = 3
 
     @property
     def flops(self):
@@ -392,30 +390,52 @@ def time_kernels(layer: Layer, reps: int, stream):
 
 
 def e2e(layer: Layer, steps: int, warmup: int, stream):
-    """Same metric through the public API from pinned host buffers: H2D of the
-    step's activations, quantise, GEMM, D2H of the bf16 output, every step."""
+    """Same metric through the public API from pinned host buffers: every
+    step copies its activations in (H2D), quantises, runs the GEMM and reads
+    its bf16 output back (D2H).  Steps are pipelined as a serving loop would
+    run them: the copy-in of step i+1 and the copy-out of step i-1 overlap
+    step i's kernels (three streams, double-buffered device input and output,
+    events order each buffer's reuse); the timed region spans the first
+    copy-in to the last copy-out."""
+    dev = layer.xs[0].device
     xh = torch.from_numpy(layer.x_host.view(np.int16)).view(torch.bfloat16).pin_memory()
-    yh = torch.empty(tuple(layer.ys[0].shape), dtype=torch.bfloat16).pin_memory()
-    xd = torch.empty_like(layer.xs[0])
+    yh = [torch.empty(tuple(layer.ys[0].shape), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    xd = [torch.empty_like(layer.xs[0]) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    in_done, cmp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    for e in cmp_done + out_done:
+        e.record(stream)            # "done" before the first use of each buffer
 
     def one(i):
+        j = i % 2
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(cmp_done[j])            # step i-2's kernels are done with xd[j]
+            xd[j].copy_(xh, non_blocking=True)
+            in_done[j].record(s_in)
         with torch.cuda.stream(stream):
-            xd.copy_(xh, non_blocking=True)
-            layer.quantize(i, stream, x=xd)
+            stream.wait_event(in_done[j])
+            stream.wait_event(out_done[j])          # step i-2's copy-out has read ys[j]
+            layer.quantize(i, stream, x=xd[j])
             layer.gemm(i, stream)
-            yh.copy_(layer.ys[i % 2], non_blocking=True)
+            cmp_done[j].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(cmp_done[j])
+            yh[j].copy_(layer.ys[i % 2], non_blocking=True)
+            out_done[j].record(s_out)
 
     for i in range(warmup):
         one(i)
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for i in range(steps):
+    a.record(s_in)
+    for i in range(warmup, warmup + steps):
         one(i)
-    b.record(stream)
+    s_out.wait_event(cmp_done[(warmup + steps - 1) % 2])
+    b.record(s_out)
     b.synchronize()
     ms = a.elapsed_time(b) / steps
-    return ms, xh.numel() * 2, yh.numel() * 2
+    return ms, xh.numel() * 2, yh[0].numel() * 2
 
 
 def small_m_sweep(device, stream, iters=240, warmup=10):
@@ -453,6 +473,59 @@ def small_m_sweep(device, stream, iters=240, warmup=10):
 
 
 # ------------------------------------------------------------ CPU oracle
+def kv_fp8_rate(device, stream, reps=20):
+    """FP8 KV-cache quantisation of one layer's K (32768 tokens x 8 heads x
+    128 dims, bf16 -> E4M3 under a calibrated scale), rotated over 3 copies
+    (201 MB > L2): graph replay of GRAPH_STEPS launches.  3 bytes per element."""
+    import nvfp4_w4a4_quantized_quantizer_b200 as nv
+    n = 32768 * 8 * 128
+    rng = np.random.default_rng(3)
+    x0 = torch.from_numpy(rng.standard_normal(n).astype(np.float32)).to(device).to(torch.bfloat16)
+    xs = [x0] + [x0.clone() for _ in range(2)]
+    out = torch.empty(n, dtype=torch.uint8, device=device)
+    s = nv.nvfp4_kv_scale(float(x0.float().abs().max().item()))
+
+    def run(i, st):
+        nv.nvfp4_kv_quantize_fp8(xs[i % 3], s, out=out, stream=st)
+
+    t = time_each({"kv": run}, reps, stream)["kv"]
+    gbs = 3.0 * n / (t * 1e-3) / 1e9
+    return {"elements": n, "us": round(t * 1e3, 2), "GBps": round(gbs, 1)}
+
+
+# fp32 FMA peak for ALU-bound kernels: 148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz
+FP32_ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def gdn_rate(device, stream, reps=4):
+    """The gated delta rule over 8192 tokens of the GDN in-projection's heads
+    (48 value heads over 16 key heads, width 128), graph replay.  FLOPs
+    counted as the definition's 6 D^2 per token and value head."""
+    import nvfp4_w4a4_quantized_quantizer_b200 as nv
+    T, Hv, group, D = 8192, 48, 3, 128
+    rng = np.random.default_rng(4)
+    f = lambda a: torch.from_numpy(a.astype(np.float32)).to(device)  # noqa: E731
+    k = rng.standard_normal((T, Hv // group, D))
+    ins = dict(q=f(rng.standard_normal((T, Hv // group, D))),
+               k=f(k / np.linalg.norm(k, axis=2, keepdims=True)),
+               v=f(rng.standard_normal((T, Hv, D))),
+               g=f(-np.log1p(np.exp(rng.normal(-2, 1, (T, Hv))))),
+               beta=f(1 / (1 + np.exp(-rng.normal(0, 1.5, (T, Hv))))))
+    state = torch.zeros((Hv, D, D), dtype=torch.float32, device=device)
+    o = torch.empty((T, Hv, D), dtype=torch.float32, device=device)
+
+    def run(i, st):
+        nv.nvfp4_gdn_recurrence(ins["q"], ins["k"], ins["v"], ins["g"], ins["beta"], group=group,
+                                state=state, o=o, stream=st)
+
+    t = time_each({"gdn": run}, reps, stream)["gdn"]
+    tflops = 6.0 * D * D * T * Hv / (t * 1e-3) / 1e12
+    return {"tokens": T, "value_heads": Hv, "us": round(t * 1e3, 1),
+            "tokens_per_s": round(T / (t * 1e-3), 1), "tflops": round(tflops, 2),
+            "bound": "alu", "peak_tflops": round(FP32_ALU_PEAK_TFLOPS, 1),
+            "frac": round(tflops / FP32_ALU_PEAK_TFLOPS, 4)}
+
+
 class OracleSample:
     """The oracle, as it stands, on bounded samples of the workload: quantise a
     few activation rows, dequantise, float64 GEMM against the dequantised
@@ -523,6 +596,8 @@ def main():
     ap.add_argument("--workload", default="prefill", choices=sorted(WORKLOAD_BY_NAME))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-small-m", action="store_true")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="launch the quantiser and the small-M GEMM without launch overlap")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -556,6 +631,9 @@ def main():
 
     import nvfp4_w4a4_quantized_quantizer_b200 as nv
     nv.load()
+    # the weights are quantised before any timed launch, so no kernel just
+    # ahead of a GEMM writes its weights (the contract of launch overlap)
+    nv.nvfp4_set_launch_overlap(not args.no_overlap)
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     pg = None
@@ -584,19 +662,15 @@ def main():
     pk = peaks()
     fp4_peak = pk["bf16"] * FP4_PER_BF16
     if mlp:
-        t = time_each({"quantize": layer.quantize, "gate_up": layer.gate_up, "silu_mul": layer.silu,
-                       "requantize": layer.requantize, "down": layer.down}, max(2, reps // 4), stream)
+        t = time_each({"quantize": layer.quantize, "gate_up": layer.gate_up, "down": layer.down},
+                      max(2, reps // 4), stream)
         q_ms, g_ms = t["quantize"], t["gate_up"]
         g_flops = 2.0 * layer.M * layer.K * layer.N           # the dominant kernel: gate_up
         d_tflops = 2.0 * layer.M * layer.H * layer.N2 / (t["down"] * 1e-3) / 1e12
-        rq_bytes = layer.M * layer.H * 2 + layer.M * layer.H // 2 + nv.nvfp4_scale_bytes(layer.M, layer.H)
         extra = {"down_us": round(t["down"] * 1e3, 2), "down_tflops": round(d_tflops, 1),
-                 "down_frac": round(d_tflops / fp4_peak, 4),
-                 "silu_mul_us": round(t["silu_mul"] * 1e3, 2),
-                 "requantize_us": round(t["requantize"] * 1e3, 2),
-                 "requantize_GBps": round(rq_bytes / (t["requantize"] * 1e-3) / 1e9, 1)}
-        step_desc = ("quantize_act + gate_up (2 modules) + silu_mul + quantize_act + down GEMM "
-                     "(bf16 out)")
+                 "down_frac": round(d_tflops / fp4_peak, 4)}
+        step_desc = ("quantize_act + gate_up (2 modules) with SiLU(gate)*up and its requantisation "
+                     "in the epilogue + down GEMM (bf16 out)")
         cfg_shape = {"M": layer.M, "K": layer.K, "N_gate_up": layer.N, "N_down": layer.N2,
                      "K_down": layer.H}
         profile = f"gemm_tc_{wl.name}.md"
@@ -622,7 +696,8 @@ def main():
                    "step": step_desc,
                    "l2": f"inputs rotated over {len(layer.xs)} activation / {len(layer.ws)} weight copies "
                          "(working set > L2)", "parallelism": f"replicas x{ws}",
-                   "launch": f"steps replayed from CUDA graphs of {GRAPH_STEPS} steps"},
+                   "launch": f"steps replayed from CUDA graphs of {GRAPH_STEPS} steps; launch overlap "
+                             + ("off" if args.no_overlap else "on (quantiser, small-M GEMM)")},
         "roofline": {"bound": "tensor", "achieved": round(g_tflops, 1), "peak": round(fp4_peak, 1),
                      "unit": "TFLOP/s", "frac": round(g_tflops / fp4_peak, 4),
                      "traffic": traffic,
@@ -644,6 +719,11 @@ def main():
         for v in sm.values():
             v["hbm_frac"] = round(v["weight_GBps"] / pk["hbm"], 4)
         line["small_m"] = sm
+    if rank == 0 and not args.no_small_m and ws == 1:
+        kv = kv_fp8_rate(device, stream)
+        kv["hbm_frac"] = round(kv["GBps"] / pk["hbm"], 4)
+        line["kv_fp8"] = kv
+        line["gdn_recurrence"] = gdn_rate(device, stream)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     if rank == 0:

@@ -146,7 +146,8 @@ nvfp4_status nvfp4_quantize_act(const void* x_bf16, int64_t M, int64_t K, int64_
  * nseg floats), and is quantised with it into the shared codes / scales
  * buffers (padding rows zeroed).  `workspace` is caller-owned DEVICE scratch
  * of nvfp4_quantize_weight_workspace_bytes(nseg) bytes (the per-module amax
- * reduction); its contents on entry do not matter.  Synchronises `stream`. */
+ * reduction); its contents on entry do not matter.  Synchronises `stream`
+ * and returns once the codes and scales are written. */
 size_t nvfp4_quantize_weight_workspace_bytes(int32_t nseg);
 nvfp4_status nvfp4_quantize_weight(const void* w_bf16, int64_t N, int64_t K, int64_t ldw,
                                    const int64_t* seg_offsets, int32_t nseg,
@@ -214,12 +215,100 @@ nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales,
                                 void* y, int64_t ldy, nvfp4_out_dtype out_dtype,
                                 nvfp4_stream_t stream);
 
+/* Workspace of nvfp4_fused_linear_ws: NVFP4_GEMM_WS_COUNTER_BYTES of
+ * arrival counters followed by one 256 KB fp32 partial tile per K-part. */
+#define NVFP4_GEMM_WS_COUNTER_BYTES 4096
+#define NVFP4_GEMM_WS_MAX_UNITS 128
+
+/* Bytes of a workspace that never limits the split of
+ * nvfp4_fused_linear_ws (NVFP4_GEMM_WS_COUNTER_BYTES + 128 partial tiles,
+ * about 32 MB).  Any device. */
+size_t nvfp4_gemm_workspace_bytes(void);
+
+/* nvfp4_fused_linear with a caller-owned device workspace that lets the
+ * CTA-pair kernel balance its last, partial wave of tiles: each tile of that
+ * wave is computed as up to 4 K-parts by pairs that would otherwise idle;
+ * each part writes an fp32 partial tile to the workspace and the last part
+ * to arrive sums the parts in part order (the same order whichever arrives
+ * last, so results do not depend on timing) and applies the epilogue.  The
+ * sum differs from the unsplit kernel's by fp32 rounding only.
+ * workspace: 16-byte aligned; its first NVFP4_GEMM_WS_COUNTER_BYTES must be
+ * zero before its first use (every call leaves them zero, also after a
+ * bounded wait ran out); it must not be in use by another call that may run
+ * at the same time.  workspace_bytes below nvfp4_gemm_workspace_bytes()
+ * limits the number of parts; NULL (or too small for two parts) runs the
+ * last wave as whole tiles, exactly like nvfp4_fused_linear.  Other
+ * arguments, layouts and errors as for nvfp4_fused_linear; an unaligned
+ * workspace returns NVFP4_ERR_ALIGNMENT. */
+nvfp4_status nvfp4_fused_linear_ws(const void* a_codes, const void* a_scales,
+                                   const void* w_codes, const void* w_scales,
+                                   int64_t M, int64_t N, int64_t K,
+                                   const nvfp4_segment* segs, int32_t nseg,
+                                   void* y, int64_t ldy, nvfp4_out_dtype out_dtype,
+                                   void* workspace, size_t workspace_bytes,
+                                   nvfp4_stream_t stream);
+
+/* The MLP pair's first half in one kernel (gate_up GEMM, SiLU(gate) * up
+ * and the NVFP4 quantisation of the product that the down projection
+ * consumes; the all-linear-layers W4A4 recipe: nefut abstract).  The weight
+ * [2H, K] holds the gate module's H rows, then the up module's H rows, each
+ * quantised with its own global scale (w_gs_gate, w_gs_up).  For every
+ * activation row m and h < H:
+ *   g = bf16(fp32(a_gs * w_gs_gate) * acc_gate[m, h]),
+ *   u = bf16(fp32(a_gs * w_gs_up) * acc_up[m, h]),
+ *   h = bf16(g / (1 + exp(-g)) * u)        (fp32 steps, as nvfp4_silu_mul),
+ * and h [M, H] is quantised under the static global scale h_gs exactly as
+ * nvfp4_quantize_act quantises it: h_codes [M, H/2], h_scales
+ * nvfp4_scale_bytes(M, H) bytes in the atom layout (padding rows zero).
+ * The result equals nvfp4_fused_linear (bf16 out, segments gate | up) ->
+ * nvfp4_silu_mul -> nvfp4_quantize_act bit for bit, without the bf16
+ * [M, 2H] and [M, H] intermediates.  Requires H % 128 == 0, K % 64 == 0,
+ * 16-byte aligned caller-owned device pointers, finite positive scales;
+ * violations return before any launch.  Queued on `stream`. */
+nvfp4_status nvfp4_gate_up_silu_quantize(const void* a_codes, const void* a_scales,
+                                          const void* w_codes, const void* w_scales,
+                                          int64_t M, int64_t H, int64_t K,
+                                          float a_gs, float w_gs_gate, float w_gs_up,
+                                          float h_gs, void* h_codes, void* h_scales,
+                                          nvfp4_stream_t stream);
+
 /* MLP glue between the two projections of the MLP pair (not an NVFP4 step):
  * h[m, j] = bf16(silu(gu[m, j]) * gu[m, H + j]) for j < H, computed in fp32.
  * gu: bf16 [M, ld_in] with ld_in >= 2H; h: bf16 [M, ld_out], ld_out >= H.
  * H % 8 == 0. */
 nvfp4_status nvfp4_silu_mul(const void* gu_bf16, int64_t M, int64_t H, int64_t ld_in,
                             void* h_bf16, int64_t ld_out, nvfp4_stream_t stream);
+
+/* FP8 KV cache: the pages' other shipped recipe, calibrated per-tensor FP8
+ * E4M3 KV-cache scales ("quantize everything, ship KV scales": nefut
+ * abstract; aimodeling, "What engineers should actually take away").
+ * nvfp4_kv_scale: fp32(amax) / 448 of a calibration batch (1 when amax <= 0;
+ * amax from nvfp4_amax).  nvfp4_kv_quantize_fp8: out[i] = sign(x[i]) |
+ * E4M3_RNE_satfinite(|fp32(x[i] * fp32(1 / scale))|) for n bf16 values x
+ * (device, 16-byte aligned; n % 8 == 0) into n bytes of out (device,
+ * 16-byte aligned); values past the calibrated range saturate at +-448 and
+ * zeros keep their sign.  Caller-owned buffers; violations return before any
+ * launch; queued on `stream`. */
+float nvfp4_kv_scale(float amax);
+nvfp4_status nvfp4_kv_quantize_fp8(const void* x_bf16, int64_t n, float scale, void* out_e4m3,
+                                   nvfp4_stream_t stream);
+
+/* Gated DeltaNet state recurrence over T tokens of one sequence (the step
+ * after the GDN in-projection; the pages' third mechanism: each write
+ * overwrites the state along its key direction -- bayesiansapien wiki, "The
+ * four-part mechanism study", part 3; the formula is the published gated
+ * delta rule):  S_t = exp(g_t) S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t
+ * k_t^T,  o_t = S_t q_t, per value head.  Device fp32 arrays, token-major:
+ * q, k [T, Hv/group, 128] (k rows of unit length), v and o [T, Hv, 128],
+ * g (log decay, <= 0) and beta [T, Hv], state [Hv, 128 (value), 128 (key)]
+ * holding the initial state on entry and the final state on return.  Value
+ * head h reads key head h / group.  head_dim must be 128; pointers 16-byte
+ * aligned.  Computed chunk by chunk (64 tokens) in fp32.  Queued on
+ * `stream`. */
+nvfp4_status nvfp4_gdn_recurrence(const float* q, const float* k, const float* v,
+                                  const float* g, const float* beta, int64_t T, int32_t Hv,
+                                  int32_t group, int32_t head_dim, float* o, float* state,
+                                  nvfp4_stream_t stream);
 
 /* Human-readable status. */
 const char* nvfp4_status_string(nvfp4_status status);
@@ -239,6 +328,21 @@ nvfp4_status nvfp4_last_device_error(nvfp4_stream_t stream, uint64_t* info);
  * automatically when the activation codes exceed 64 MB and the weight codes
  * are smaller).  Process-wide. */
 nvfp4_status nvfp4_set_gemm_path(int32_t path);
+
+/* Launch overlap (process-wide, off by default; on = 1, off = 0): the
+ * activation quantiser and the small-M GEMM (M <= 64) are launched with
+ * programmatic stream serialization, so that each may start while the
+ * kernel ahead of it on the stream is still running and the next call's
+ * weight stream overlaps this call's tail (the decode loop of consecutive
+ * layers).  The quantiser waits for the kernel ahead before it reads x or
+ * writes codes and scales.  The GEMM waits for it before it reads the
+ * activation codes and scales and before it writes y, but streams the
+ * weight codes and scales from its start: with overlap on, the kernel
+ * launched just ahead of a small-M GEMM on the same stream must not write
+ * that GEMM's weight codes or scales (weights quantised offline, or any
+ * other kernel in between, satisfy this).  Results are identical with
+ * overlap on or off. */
+nvfp4_status nvfp4_set_launch_overlap(int32_t on);
 
 /* Time limit of every bounded in-kernel wait, in nanoseconds (default 2e9;
  * also read once from the environment variable NVFP4_SPIN_LIMIT_NS). */

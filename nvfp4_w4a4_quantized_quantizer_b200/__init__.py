@@ -20,8 +20,9 @@ from ._lib import (NVFP4Error, OP_GDN_DECAY, OP_NONE, OP_SIGMOID, OUT_BF16, OUT_
 __all__ = [
     "nvfp4_codes_bytes", "nvfp4_scale_bytes", "nvfp4_global_scale", "nvfp4_amax",
     "nvfp4_quantize_act", "nvfp4_quantize_weight", "nvfp4_quantize_weight_noalloc",
-    "nvfp4_linear", "nvfp4_fused_linear",
-    "nvfp4_silu_mul", "nvfp4_last_device_error", "nvfp4_set_gemm_path",
+    "nvfp4_linear", "nvfp4_fused_linear", "nvfp4_gemm_workspace_bytes", "nvfp4_gemm_workspace",
+    "nvfp4_gate_up_silu_quantize", "nvfp4_gdn_recurrence", "nvfp4_silu_mul", "nvfp4_last_device_error",
+    "nvfp4_set_gemm_path", "nvfp4_set_launch_overlap", "nvfp4_kv_scale", "nvfp4_kv_quantize_fp8",
     "nvfp4_set_wait_limit_ns", "nvfp4_test_e2m1", "nvfp4_test_e4m3", "nvfp4_test_wait_timeout",
     "SegmentSpec", "NVFP4Error", "OP_NONE", "OP_SIGMOID", "OP_GDN_DECAY",
 ]
@@ -155,15 +156,87 @@ def nvfp4_linear(a_codes, a_scales, a_gs: float, w_codes, w_scales, w_gs: float,
     return y
 
 
+def nvfp4_gemm_workspace_bytes() -> int:
+    return load().nvfp4_gemm_workspace_bytes()
+
+
+def nvfp4_gemm_workspace(device=None) -> torch.Tensor:
+    """A zeroed workspace of nvfp4_gemm_workspace_bytes() for nvfp4_fused_linear."""
+    return torch.zeros(nvfp4_gemm_workspace_bytes(), dtype=torch.uint8, device=device)
+
+
 def nvfp4_fused_linear(a_codes, a_scales, w_codes, w_scales, M: int, N: int, K: int,
                        segments: Sequence[SegmentSpec], y: Optional[torch.Tensor] = None,
-                       out_dtype: int = OUT_BF16, stream=None) -> torch.Tensor:
+                       out_dtype: int = OUT_BF16, stream=None,
+                       workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """With `workspace` (see nvfp4_gemm_workspace) the call is
+    nvfp4_fused_linear_ws, which splits the last partial wave along K."""
     y = _out(y, M, N, out_dtype, a_codes.device)
     segs = (Segment * len(segments))(*[s.c() for s in segments])
-    check(load().nvfp4_fused_linear(_ptr(a_codes), _ptr(a_scales), _ptr(w_codes), _ptr(w_scales),
-                                    M, N, K, segs, len(segments), _ptr(y), _ld(y), out_dtype,
-                                    _stream(stream)), "nvfp4_fused_linear")
+    if workspace is None:
+        check(load().nvfp4_fused_linear(_ptr(a_codes), _ptr(a_scales), _ptr(w_codes),
+                                        _ptr(w_scales), M, N, K, segs, len(segments), _ptr(y),
+                                        _ld(y), out_dtype, _stream(stream)), "nvfp4_fused_linear")
+    else:
+        check(load().nvfp4_fused_linear_ws(_ptr(a_codes), _ptr(a_scales), _ptr(w_codes),
+                                           _ptr(w_scales), M, N, K, segs, len(segments), _ptr(y),
+                                           _ld(y), out_dtype, _ptr(workspace),
+                                           workspace.numel() * workspace.element_size(),
+                                           _stream(stream)), "nvfp4_fused_linear_ws")
     return y
+
+
+def nvfp4_gate_up_silu_quantize(a_codes, a_scales, w_codes, w_scales, M: int, H: int, K: int,
+                                a_gs: float, w_gs_gate: float, w_gs_up: float, h_gs: float,
+                                h_codes: Optional[torch.Tensor] = None,
+                                h_scales: Optional[torch.Tensor] = None,
+                                stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    dev = a_codes.device
+    if h_codes is None:
+        h_codes = torch.empty((M, H // 2), dtype=torch.uint8, device=dev)
+    if h_scales is None:
+        h_scales = torch.empty(nvfp4_scale_bytes(M, H), dtype=torch.uint8, device=dev)
+    check(load().nvfp4_gate_up_silu_quantize(
+        _ptr(a_codes), _ptr(a_scales), _ptr(w_codes), _ptr(w_scales), M, H, K,
+        ctypes.c_float(a_gs), ctypes.c_float(w_gs_gate), ctypes.c_float(w_gs_up),
+        ctypes.c_float(h_gs), _ptr(h_codes), _ptr(h_scales), _stream(stream)),
+        "nvfp4_gate_up_silu_quantize")
+    return h_codes, h_scales
+
+
+def nvfp4_kv_scale(amax: float) -> float:
+    return load().nvfp4_kv_scale(ctypes.c_float(amax))
+
+
+def nvfp4_kv_quantize_fp8(x: torch.Tensor, scale: float, out: Optional[torch.Tensor] = None,
+                          stream=None) -> torch.Tensor:
+    """bf16 tensor (contiguous, numel % 8 == 0) -> E4M3 codes (uint8, same shape)."""
+    if not x.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    check(load().nvfp4_kv_quantize_fp8(_ptr(x), x.numel(), ctypes.c_float(scale), _ptr(out),
+                                       _stream(stream)), "nvfp4_kv_quantize_fp8")
+    return out
+
+
+def nvfp4_gdn_recurrence(q, k, v, g, beta, group: int = 1, state: Optional[torch.Tensor] = None,
+                         o: Optional[torch.Tensor] = None, stream=None):
+    """Gated delta rule over one sequence: q, k [T, Hk, 128], v [T, Hv, 128], g and beta
+    [T, Hv] (fp32, contiguous).  Returns (o [T, Hv, 128], final state [Hv, 128, 128]);
+    `state` (initial state, updated in place) defaults to zeros."""
+    T, Hv, D = v.shape
+    for t in (q, k, v, g, beta):
+        if t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError("expected contiguous float32 tensors")
+    if state is None:
+        state = torch.zeros((Hv, D, D), dtype=torch.float32, device=v.device)
+    if o is None:
+        o = torch.empty((T, Hv, D), dtype=torch.float32, device=v.device)
+    check(load().nvfp4_gdn_recurrence(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), T, Hv, group,
+                                      D, _ptr(o), _ptr(state), _stream(stream)),
+          "nvfp4_gdn_recurrence")
+    return o, state
 
 
 def nvfp4_silu_mul(gu: torch.Tensor, H: int, h: Optional[torch.Tensor] = None,
@@ -184,6 +257,10 @@ def nvfp4_last_device_error(stream=None) -> Tuple[int, int]:
 
 def nvfp4_set_gemm_path(path: int) -> None:
     check(load().nvfp4_set_gemm_path(path), "nvfp4_set_gemm_path")
+
+
+def nvfp4_set_launch_overlap(on: bool) -> None:
+    check(load().nvfp4_set_launch_overlap(1 if on else 0), "nvfp4_set_launch_overlap")
 
 
 def nvfp4_set_wait_limit_ns(limit_ns: int) -> None:

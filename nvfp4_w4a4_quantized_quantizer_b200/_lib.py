@@ -43,10 +43,19 @@ SIGNATURES = {
     "nvfp4_linear": (_st, [_vp, _vp, _f32, _vp, _vp, _f32, _i64, _i64, _i64, _vp, _i64, _st, _vp]),
     "nvfp4_fused_linear": (_st, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.POINTER(Segment), _i32,
                                  _vp, _i64, _st, _vp]),
+    "nvfp4_gemm_workspace_bytes": (_sz, []),
+    "nvfp4_fused_linear_ws": (_st, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.POINTER(Segment),
+                                    _i32, _vp, _i64, _st, _vp, _sz, _vp]),
+    "nvfp4_gate_up_silu_quantize": (_st, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _f32, _f32, _f32,
+                                          _f32, _vp, _vp, _vp]),
     "nvfp4_silu_mul": (_st, [_vp, _i64, _i64, _i64, _vp, _i64, _vp]),
+    "nvfp4_kv_scale": (_f32, [_f32]),
+    "nvfp4_kv_quantize_fp8": (_st, [_vp, _i64, _f32, _vp, _vp]),
+    "nvfp4_gdn_recurrence": (_st, [_vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp]),
     "nvfp4_status_string": (ctypes.c_char_p, [_st]),
     "nvfp4_last_device_error": (_st, [_vp, ctypes.POINTER(ctypes.c_uint64)]),
     "nvfp4_set_gemm_path": (_st, [_i32]),
+    "nvfp4_set_launch_overlap": (_st, [_i32]),
     "nvfp4_set_wait_limit_ns": (_st, [_u64]),
     "nvfp4_test_e2m1": (_st, [_vp, _vp, _i64, _vp]),
     "nvfp4_test_e4m3": (_st, [_vp, _vp, _i64, _vp]),

@@ -15,6 +15,7 @@
 #include <unordered_map>
 
 #include "nvfp4.h"
+#include "gdn.cuh"
 #include "gemm.cuh"
 #include "quantize.cuh"
 
@@ -34,6 +35,34 @@ uint64_t read_env_wait_ns() {
 
 uint64_t g_wait_ns = read_env_wait_ns();
 int g_gemm_path = 0;
+bool g_overlap = false;
+
+// Launch with programmatic stream serialization when launch overlap is on:
+// the kernel may then start before the kernel ahead of it on the stream has
+// finished (it waits for it with griddepcontrol.wait where it must).
+template <typename Kernel, typename... Args>
+nvfp4_status launch_maybe_overlapped(Kernel kernel, dim3 grid, dim3 block, int smem,
+                                     cudaStream_t st, Args... args) {
+  if (!g_overlap) {
+    kernel<<<grid, block, smem, st>>>(args...);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, args...) != cudaSuccess) {
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+  }
+  return NVFP4_OK;
+}
 
 // ----------------------------------------------------------- device info
 constexpr int MAX_DEVICES = 64;
@@ -43,8 +72,11 @@ struct DeviceInfo {
   int sms = 0;
   bool attr_tc = false;
   bool attr_tc2 = false;
+  bool attr_tc2_swiglu = false;
+  bool attr_gdn = false;
   int quant_blocks = 0;   // resident k_quantize blocks per SM
   int pairs = 0;          // co-resident clusters of two CTAs of k_gemm_tc<2>
+  int swiglu_pairs = 0;   // the same for k_gemm_tc<2, true>
   bool attr_small[3] = {false, false, false};
 };
 DeviceInfo g_dev[MAX_DEVICES];
@@ -199,6 +231,10 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 constexpr int64_t kMaxDim = (1ll << 31) - 1;
 
+// One K-part's fp32 partial tile: 2 CTAs x 128 rows x 256 columns.
+constexpr size_t kPartialBytes = 2ull * nvfp4::tc::BM * nvfp4::tc::BN * 4;
+constexpr int64_t kMaxSplit = 4;
+
 nvfp4_status check_bf16_matrix(const void* x, int64_t R, int64_t K, int64_t ld) {
   if (x == nullptr) return NVFP4_ERR_INVALID_ARG;
   if (R < 0 || K < 64 || K % 64 != 0 || R > kMaxDim || K > kMaxDim) return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -259,8 +295,8 @@ nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t K, int64_t ld,
   }
   // persistent: one wave of resident blocks, each warp striding over the units
   const int grid = grid_for(units, nvfp4::QUANT_WARPS, info->sms * info->quant_blocks);
-  nvfp4::k_quantize<<<grid, nvfp4::QUANT_THREADS, smem, st>>>(a);
-  return check_launch();
+  return launch_maybe_overlapped(nvfp4::k_quantize, dim3(grid), dim3(nvfp4::QUANT_THREADS), smem,
+                                 st, a);
 }
 
 nvfp4_status launch_amax(const void* x, int64_t rows, int64_t K, int64_t ld, float* out, int sms,
@@ -330,6 +366,43 @@ nvfp4_status noalloc_scratch(float** out) {
   return NVFP4_OK;
 }
 
+// Launch configuration of a CTA-pair kernel (clusters of two CTAs, its
+// dynamic shared memory, `st`); once per device and kernel, also the
+// shared-memory attribute and the number of pairs that fit at once (clusters
+// are placed within one GPC, so an SM count that is odd inside a GPC leaves
+// an SM out).  attr must outlive cfg.
+template <typename Kernel>
+nvfp4_status pair_config(Kernel kernel, DeviceInfo* info, bool* configured, int* max_pairs,
+                         cudaStream_t st, cudaLaunchConfig_t* cfg, cudaLaunchAttribute* attr) {
+  constexpr int smem = nvfp4::tc::Cfg<2>::SMEM_BYTES;
+  *cfg = cudaLaunchConfig_t{};
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg->blockDim = dim3(nvfp4::tc::THREADS, 1, 1);
+  cfg->dynamicSmemBytes = smem;
+  cfg->stream = st;
+  cfg->attrs = attr;
+  cfg->numAttrs = 1;
+  if (!*configured) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return NVFP4_ERR_CUDA;
+    }
+    cfg->gridDim = dim3(2 * (info->sms / 2), 1, 1);
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kernel, cfg) != cudaSuccess || clusters < 1) {
+      cudaGetLastError();
+      return NVFP4_ERR_CUDA;
+    }
+    *max_pairs = clusters;
+    *configured = true;
+  }
+  return NVFP4_OK;
+}
+
 }  // namespace
 
 // =================================================================== C ABI
@@ -363,6 +436,12 @@ const char* nvfp4_status_string(nvfp4_status s) {
 nvfp4_status nvfp4_set_gemm_path(int32_t path) {
   if (path < 0 || path > 4) return NVFP4_ERR_INVALID_ARG;
   g_gemm_path = path;
+  return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_set_launch_overlap(int32_t on) {
+  if (on != 0 && on != 1) return NVFP4_ERR_INVALID_ARG;
+  g_overlap = (on == 1);
   return NVFP4_OK;
 }
 
@@ -466,6 +545,12 @@ nvfp4_status nvfp4_quantize_weight(const void* w, int64_t N, int64_t K, int64_t 
                          scales, last ? N : 0, last ? pad128(N) : 0, info, cs);
     if (st != NVFP4_OK) return st;
   }
+  // the codes and scales are complete on return, so that a GEMM launched
+  // with launch overlap may stream them from its start
+  if (cudaStreamSynchronize(cs) != cudaSuccess) {
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+  }
   return NVFP4_OK;
 }
 
@@ -487,13 +572,20 @@ nvfp4_status nvfp4_quantize_weight_noalloc(const void* w, int64_t N, int64_t K, 
                                stream);
 }
 
-nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales, const void* w_codes,
-                                const void* w_scales, int64_t M, int64_t N, int64_t K,
-                                const nvfp4_segment* segs, int32_t nseg, void* y, int64_t ldy,
-                                nvfp4_out_dtype out_dtype, nvfp4_stream_t stream) {
+size_t nvfp4_gemm_workspace_bytes(void) {
+  return static_cast<size_t>(NVFP4_GEMM_WS_COUNTER_BYTES) +
+         static_cast<size_t>(NVFP4_GEMM_WS_MAX_UNITS) * kPartialBytes;
+}
+
+nvfp4_status nvfp4_fused_linear_ws(const void* a_codes, const void* a_scales, const void* w_codes,
+                                   const void* w_scales, int64_t M, int64_t N, int64_t K,
+                                   const nvfp4_segment* segs, int32_t nseg, void* y, int64_t ldy,
+                                   nvfp4_out_dtype out_dtype, void* workspace,
+                                   size_t workspace_bytes, nvfp4_stream_t stream) {
   if (a_codes == nullptr || a_scales == nullptr || w_codes == nullptr || w_scales == nullptr ||
       y == nullptr)
     return NVFP4_ERR_INVALID_ARG;
+  if (workspace != nullptr && !aligned16(workspace)) return NVFP4_ERR_ALIGNMENT;
   if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_FP32) return NVFP4_ERR_INVALID_ARG;
   if (M < 0 || M > kMaxDim || N < 16 || N % 16 != 0 || N > kMaxDim || K < 64 || K % 64 != 0 ||
       K > kMaxDim || ldy < N)
@@ -524,6 +616,11 @@ nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales, const
   g.sector_stores = ((reinterpret_cast<uintptr_t>(y) & 31u) == 0) &&
                     ((ldy * (g.out_fp32 ? 4 : 2)) % 32 == 0);
   g.wait_ns = g_wait_ns;
+  g.full_tiles = 0;
+  g.split = 1;
+  g.split_units = 0;
+  g.partial = nullptr;
+  g.counters = nullptr;
   // Tile raster.  Consecutive CTAs (pairs) run tiles that share one operand
   // tile, and the rest of that operand is re-read from L2 for each of the
   // other operand's tiles.  By default they share weight tiles (M fastest),
@@ -549,8 +646,8 @@ nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales, const
           return NVFP4_ERR_CUDA;
         info->attr_small[which] = true;
       }
-      kernel<<<grid, nvfp4::sm::THREADS, smem, cs>>>(tw, tx, g, table);
-      return check_launch();
+      return launch_maybe_overlapped(kernel, dim3(grid), dim3(nvfp4::sm::THREADS), smem, cs, tw,
+                                     tx, g, table);
     };
     if (nt == 16) return launch(nvfp4::k_gemm_small<16>, nvfp4::sm::Cfg<16>::SMEM_BYTES);
     if (nt == 32) return launch(nvfp4::k_gemm_small<32>, nvfp4::sm::Cfg<32>::SMEM_BYTES);
@@ -563,7 +660,7 @@ nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales, const
   if ((st = code_map(w_codes, N, K / 2, nvfp4::tc::BN / (pair ? 2 : 1), dev, &tb)) != NVFP4_OK)
     return st;
   if ((st = scale_map(a_scales, M, K, 1, dev, &tsa)) != NVFP4_OK) return st;
-  if ((st = scale_map(w_scales, N, K, 2, dev, &tsb)) != NVFP4_OK) return st;
+  if ((st = scale_map(w_scales, N, K, pair ? 1 : 2, dev, &tsb)) != NVFP4_OK) return st;
   const int64_t num_n = (N + nvfp4::tc::BN - 1) / nvfp4::tc::BN;
   if (!pair) {
     constexpr int smem = nvfp4::tc::Cfg<1>::SMEM_BYTES;
@@ -578,38 +675,109 @@ nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales, const
     nvfp4::k_gemm_tc<1><<<grid, nvfp4::tc::THREADS, smem, cs>>>(ta, tb, tsa, tsb, g, table);
     return check_launch();
   }
-  constexpr int smem = nvfp4::tc::Cfg<2>::SMEM_BYTES;
-  cudaLaunchConfig_t cfg = {};
+  cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.blockDim = dim3(nvfp4::tc::THREADS, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = cs;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (!info->attr_tc2) {
-    if (cudaFuncSetAttribute(nvfp4::k_gemm_tc<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
-      return NVFP4_ERR_CUDA;
-    // how many pairs fit at once (clusters are placed within one GPC, so an
-    // SM count that is odd inside a GPC leaves an SM out)
-    cfg.gridDim = dim3(2 * (info->sms / 2), 1, 1);
-    int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, nvfp4::k_gemm_tc<2>, &cfg) != cudaSuccess ||
-        clusters < 1) {
-      cudaGetLastError();
-      return NVFP4_ERR_CUDA;
-    }
-    info->pairs = clusters;
-    info->attr_tc2 = true;
-  }
+  if ((st = pair_config(nvfp4::k_gemm_tc<2>, info, &info->attr_tc2, &info->pairs, cs, &cfg,
+                        attr)) != NVFP4_OK)
+    return st;
   const int64_t tiles = ((M + 2 * nvfp4::tc::BM - 1) / (2 * nvfp4::tc::BM)) * num_n;
   const int pairs = static_cast<int>(tiles < info->pairs ? tiles : info->pairs);
   cfg.gridDim = dim3(2 * pairs, 1, 1);
+  // Last partial wave: when the tiles are not a multiple of the pairs, each
+  // tile of the last wave is split into S K-parts run by otherwise idle
+  // pairs (S = pairs / leftover tiles, at most 4, at most the k-tiles and
+  // within the workspace); the parts meet in the caller's workspace.
+  if (workspace != nullptr && tiles > pairs) {
+    const int64_t num_kt = (K + nvfp4::tc::BK - 1) / nvfp4::tc::BK;
+    const int64_t left = tiles % pairs;
+    const int64_t max_units =
+        workspace_bytes > NVFP4_GEMM_WS_COUNTER_BYTES
+            ? static_cast<int64_t>((workspace_bytes - NVFP4_GEMM_WS_COUNTER_BYTES) / kPartialBytes)
+            : 0;
+    int64_t S = left > 0 ? pairs / left : 0;
+    if (S > kMaxSplit) S = kMaxSplit;
+    if (S > num_kt) S = num_kt;
+    while (S >= 2 && left * S > max_units) --S;
+    if (S >= 2 && left * 2 * 4 <= NVFP4_GEMM_WS_COUNTER_BYTES) {
+      g.full_tiles = static_cast<int>(tiles - left);
+      g.split = static_cast<int>(S);
+      g.split_units = static_cast<int>(left * S);
+      g.counters = static_cast<unsigned*>(workspace);
+      g.partial = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                           NVFP4_GEMM_WS_COUNTER_BYTES);
+    }
+  }
   if (cudaLaunchKernelEx(&cfg, nvfp4::k_gemm_tc<2>, ta, tb, tsa, tsb, g, table) != cudaSuccess) {
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+  }
+  return check_launch();
+}
+
+nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales, const void* w_codes,
+                                const void* w_scales, int64_t M, int64_t N, int64_t K,
+                                const nvfp4_segment* segs, int32_t nseg, void* y, int64_t ldy,
+                                nvfp4_out_dtype out_dtype, nvfp4_stream_t stream) {
+  return nvfp4_fused_linear_ws(a_codes, a_scales, w_codes, w_scales, M, N, K, segs, nseg, y, ldy,
+                               out_dtype, nullptr, 0, stream);
+}
+
+nvfp4_status nvfp4_gate_up_silu_quantize(const void* a_codes, const void* a_scales,
+                                          const void* w_codes, const void* w_scales, int64_t M,
+                                          int64_t H, int64_t K, float a_gs, float w_gs_gate,
+                                          float w_gs_up, float h_gs, void* h_codes, void* h_scales,
+                                          nvfp4_stream_t stream) {
+  if (a_codes == nullptr || a_scales == nullptr || w_codes == nullptr || w_scales == nullptr ||
+      h_codes == nullptr || h_scales == nullptr)
+    return NVFP4_ERR_INVALID_ARG;
+  if (M < 0 || M > kMaxDim || H < 128 || H % 128 != 0 || 2 * H > kMaxDim || K < 64 ||
+      K % 64 != 0 || K > kMaxDim)
+    return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(w_codes) ||
+      !aligned16(w_scales) || !aligned16(h_codes) || !aligned16(h_scales))
+    return NVFP4_ERR_ALIGNMENT;
+  if (!good_scale(a_gs) || !good_scale(w_gs_gate) || !good_scale(w_gs_up) || !good_scale(h_gs))
+    return NVFP4_ERR_INVALID_ARG;
+  if (M == 0) return NVFP4_OK;
+  int dev;
+  DeviceInfo* info;
+  nvfp4_status st = current_device(&dev, &info);
+  if (st != NVFP4_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+
+  nvfp4::GemmArgs g = {};
+  g.M = static_cast<int>(M);
+  g.N = static_cast<int>(2 * H);
+  g.K = static_cast<int>(K);
+  g.wait_ns = g_wait_ns;
+  g.H = static_cast<int>(H);
+  g.alpha_gate = a_gs * w_gs_gate;   // fp32 products, as the segment table forms them
+  g.alpha_up = a_gs * w_gs_up;
+  g.h_gs = h_gs;
+  g.h_codes = static_cast<uint8_t*>(h_codes);
+  g.h_scales = static_cast<uint8_t*>(h_scales);
+  const int64_t a_bytes = M * (K / 2), w_bytes = 2 * H * (K / 2);
+  g.n_fastest = a_bytes > (64ll << 20) && w_bytes < a_bytes;
+  nvfp4_segment one = {0, w_gs_gate, a_gs, NVFP4_OP_NONE, nullptr, nullptr};
+  SegTable table;
+  if ((st = build_segments(&one, 1, 2 * H, &table)) != NVFP4_OK) return st;
+
+  CUtensorMap ta, tb, tsa, tsb;
+  if ((st = code_map(a_codes, M, K / 2, nvfp4::tc::BM, dev, &ta)) != NVFP4_OK) return st;
+  if ((st = code_map(w_codes, 2 * H, K / 2, nvfp4::tc::BN / 2, dev, &tb)) != NVFP4_OK) return st;
+  if ((st = scale_map(a_scales, M, K, 1, dev, &tsa)) != NVFP4_OK) return st;
+  if ((st = scale_map(w_scales, 2 * H, K, 1, dev, &tsb)) != NVFP4_OK) return st;
+
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  if ((st = pair_config(nvfp4::k_gemm_tc<2, true>, info, &info->attr_tc2_swiglu,
+                        &info->swiglu_pairs, cs, &cfg, attr)) != NVFP4_OK)
+    return st;
+  const int64_t tiles = ((M + 2 * nvfp4::tc::BM - 1) / (2 * nvfp4::tc::BM)) * (H / 128);
+  const int pairs = static_cast<int>(tiles < info->swiglu_pairs ? tiles : info->swiglu_pairs);
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  if (cudaLaunchKernelEx(&cfg, nvfp4::k_gemm_tc<2, true>, ta, tb, tsa, tsb, g, table) !=
+      cudaSuccess) {
     cudaGetLastError();
     return NVFP4_ERR_CUDA;
   }
@@ -645,6 +813,75 @@ nvfp4_status nvfp4_silu_mul(const void* gu, int64_t M, int64_t H, int64_t ld_in,
   const int grid = grid_for(M * (H / 8), nvfp4::SILU_THREADS, info->sms * 8);
   nvfp4::k_silu_mul<<<grid, nvfp4::SILU_THREADS, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<const __nv_bfloat16*>(gu), M, H, ld_in, static_cast<__nv_bfloat16*>(h), ld_out);
+  return check_launch();
+}
+
+float nvfp4_kv_scale(float amax) { return amax > 0.0f ? amax / 448.0f : 1.0f; }
+
+nvfp4_status nvfp4_kv_quantize_fp8(const void* x, int64_t n, float scale, void* out,
+                                   nvfp4_stream_t stream) {
+  if (x == nullptr || out == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (n < 0 || n % 8 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(x) || !aligned16(out)) return NVFP4_ERR_ALIGNMENT;
+  if (!good_scale(scale)) return NVFP4_ERR_INVALID_ARG;
+  if (n == 0) return NVFP4_OK;
+  int dev;
+  DeviceInfo* info;
+  nvfp4_status st = current_device(&dev, &info);
+  if (st != NVFP4_OK) return st;
+  volatile float one = 1.0f;
+  const float r = one / scale;   // fp32(1 / scale), IEEE division
+  const int grid = grid_for(n / 8, nvfp4::KV_THREADS, info->sms * 8);
+  nvfp4::k_kv_fp8<<<grid, nvfp4::KV_THREADS, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x), n / 8, r, static_cast<uint2*>(out));
+  return check_launch();
+}
+
+nvfp4_status nvfp4_gdn_recurrence(const float* q, const float* k, const float* v, const float* g,
+                                  const float* beta, int64_t T, int32_t Hv, int32_t group,
+                                  int32_t head_dim, float* o, float* state,
+                                  nvfp4_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || g == nullptr || beta == nullptr ||
+      o == nullptr || state == nullptr)
+    return NVFP4_ERR_INVALID_ARG;
+  if (T < 0 || Hv < 1 || group < 1 || Hv % group != 0 || head_dim != nvfp4::gdn::D)
+    return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  for (const void* p : {static_cast<const void*>(q), static_cast<const void*>(k),
+                        static_cast<const void*>(v), static_cast<const void*>(o),
+                        static_cast<const void*>(state)})
+    if (!aligned16(p)) return NVFP4_ERR_ALIGNMENT;
+  int dev;
+  DeviceInfo* info;
+  nvfp4_status st = current_device(&dev, &info);
+  if (st != NVFP4_OK) return st;
+  if (!info->attr_gdn) {
+    if (cudaFuncSetAttribute(nvfp4::k_gdn_chunked, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             nvfp4::gdn::SMEM_BYTES) != cudaSuccess) {
+      cudaGetLastError();
+      return NVFP4_ERR_CUDA;
+    }
+    info->attr_gdn = true;
+  }
+  nvfp4::GdnArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.g = g;
+  a.beta = beta;
+  a.o = o;
+  a.state = state;
+  a.T = T;
+  a.Hv = Hv;
+  a.group = group;
+  // value rows are independent: split each head over enough CTAs to fill the
+  // SMs in one wave (at most 8 parts of at least 16 rows)
+  int parts = info->sms / Hv;
+  if (parts < 1) parts = 1;
+  if (parts > 8) parts = 8;
+  a.rows = (nvfp4::gdn::D + parts - 1) / parts;
+  a.parts = (nvfp4::gdn::D + a.rows - 1) / a.rows;
+  nvfp4::k_gdn_chunked<<<Hv * a.parts, nvfp4::gdn::THREADS, nvfp4::gdn::SMEM_BYTES,
+                         reinterpret_cast<cudaStream_t>(stream)>>>(a);
   return check_launch();
 }
 

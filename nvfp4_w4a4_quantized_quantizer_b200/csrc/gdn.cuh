@@ -1,0 +1,177 @@
+// gdn.cuh -- the Gated DeltaNet state recurrence (the step after the GDN
+// in-projection), chunk by chunk.
+//
+// The recurrent half of the hybrid model keeps, per value head, a state
+// S in R^{dv x dk} that every token overwrites along its key direction
+// (bayesiansapien wiki, "The four-part mechanism study", part 3; the
+// formula is the published gated delta rule):
+//   S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,   o_t = S_t q_t,
+// with alpha_t = exp(g_t) (g and beta from the in-projection's gate
+// epilogue) and unit keys.  Per chunk of C tokens starting from S_0, with
+// G_t the running sum of g inside the chunk:
+//   A_tj = beta_t e^{G_t - G_j} (k_t . k_j)               (j < t)
+//   (I + A) U = diag(beta) V - diag(beta e^G) K S_0^T      (forward substitution)
+//   O_t = e^{G_t} S_0 q_t + sum_{j <= t} e^{G_t - G_j} (q_t . k_j) U_j
+//   S_C = e^{G_C} S_0 + sum_t e^{G_C - G_t} U_t k_t^T
+//
+// Each value row of S evolves on its own (S_i <- alpha S_i (I - beta k k^T)
+// + beta v_i k^T reads only the keys, beta and g), so a head splits across
+// CTAs by value rows; only the key products (A, and Q K^T) are computed by
+// every CTA of the head.
+//
+// k_gdn_chunked: one CTA per (value head, block of value rows); the fp32
+// state rows and one chunk's keys, queries and value columns stay in shared
+// memory (at most 182 KB); fp32 CUDA-core arithmetic.  A first correct form:
+// the products are dense and would belong on the tensor cores.
+#pragma once
+
+#include <cstdint>
+
+namespace nvfp4 {
+namespace gdn {
+constexpr int C = 64;          // tokens per chunk
+constexpr int D = 128;         // key and value head width
+constexpr int LD = D + 1;      // padded rows of S, K, Q: a warp reading a column is bank-conflict free
+constexpr int THREADS = 256;
+constexpr int SMEM_FLOATS = D * LD + 2 * C * LD + C * D + C * C + 4 * C;
+constexpr int SMEM_BYTES = SMEM_FLOATS * 4;
+static_assert(SMEM_BYTES <= 232448, "shared memory");
+}  // namespace gdn
+
+struct GdnArgs {
+  const float* q;      // [T, Hk, D] (unit rows expected for k; q as is)
+  const float* k;      // [T, Hk, D]
+  const float* v;      // [T, Hv, D]
+  const float* g;      // [T, Hv] log decay (<= 0)
+  const float* beta;   // [T, Hv]
+  float* o;            // [T, Hv, D]
+  float* state;        // [Hv, D (value), D (key)]: initial state in, final state out
+  int64_t T;
+  int Hv, group;       // value heads; value heads per key head (Hk = Hv / group)
+  int parts;           // CTAs per head, each with rows [p * rows, min(D, (p + 1) * rows))
+  int rows;
+};
+
+__global__ void __launch_bounds__(gdn::THREADS, 1) k_gdn_chunked(const GdnArgs a) {
+  using namespace gdn;
+  extern __shared__ __align__(16) float gsm[];
+  float* S = gsm;                   // [rn value rows][LD key]
+  float* Kc = S + D * LD;           // [C][LD]
+  float* Qc = Kc + C * LD;          // [C][LD]
+  float* Vc = Qc + C * LD;          // [C][rn]: values, then the right-hand side, then U
+  float* A = Vc + C * D;            // [C][C]: A, then the masked, scaled Q K^T
+  float* G = A + C * C;             // [C] running log decay
+  float* B = G + C;                 // [C] beta
+  float* E = B + C;                 // [C] e^{G_t}
+  float* W = E + C;                 // [C] e^{G_last - G_t}
+  const int h = blockIdx.x / a.parts;          // value head
+  const int r0 = (blockIdx.x % a.parts) * a.rows;
+  const int rn = min(D, r0 + a.rows) - r0;      // this CTA's value rows [r0, r0 + rn)
+  const int hk = h / a.group;
+  const int Hk = a.Hv / a.group;
+  const int tid = threadIdx.x;
+  float* state = a.state + (static_cast<int64_t>(h) * D + r0) * D;
+
+  for (int x = tid; x < rn * D; x += THREADS) S[(x / D) * LD + x % D] = state[x];
+
+  for (int64_t c0 = 0; c0 < a.T; c0 += C) {
+    const int cn = static_cast<int>(a.T - c0 < C ? a.T - c0 : C);
+    __syncthreads();   // the previous chunk is done with Kc, Qc, Vc, A and S
+    for (int x = tid; x < C * D; x += THREADS) {
+      const int t = x / D, d = x - t * D;
+      const bool live = t < cn;
+      const int64_t tok = c0 + t;
+      Kc[t * LD + d] = live ? a.k[(tok * Hk + hk) * D + d] : 0.0f;
+      Qc[t * LD + d] = live ? a.q[(tok * Hk + hk) * D + d] : 0.0f;
+    }
+    for (int x = tid; x < C * rn; x += THREADS) {
+      const int t = x / rn, i = x - t * rn;
+      Vc[x] = t < cn ? a.v[((c0 + t) * a.Hv + h) * D + r0 + i] : 0.0f;
+    }
+    if (tid < 32) {
+      // running sum of g over the chunk: 64 values, two per lane
+      float g0 = 0.0f, g1 = 0.0f;
+      const int t0 = 2 * tid, t1 = 2 * tid + 1;
+      if (t0 < cn) g0 = a.g[(c0 + t0) * a.Hv + h];
+      if (t1 < cn) g1 = a.g[(c0 + t1) * a.Hv + h];
+      float run = g0 + g1;
+      for (int off = 1; off < 32; off <<= 1) {
+        const float up = __shfl_up_sync(0xffffffffu, run, off);
+        if (tid >= off) run += up;
+      }
+      float before = __shfl_up_sync(0xffffffffu, run, 1);   // sum over earlier pairs
+      if (tid == 0) before = 0.0f;
+      G[t0] = before + g0;
+      G[t1] = G[t0] + g1;
+      B[t0] = t0 < cn ? a.beta[(c0 + t0) * a.Hv + h] : 0.0f;
+      B[t1] = t1 < cn ? a.beta[(c0 + t1) * a.Hv + h] : 0.0f;
+      E[t0] = expf(G[t0]);
+      E[t1] = expf(G[t1]);
+    }
+    __syncthreads();
+
+    // A_tj = beta_t e^{G_t - G_j} (k_t . k_j), j < t
+    for (int x = tid; x < C * C; x += THREADS) {
+      const int t = x / C, j = x - t * C;
+      float acc = 0.0f;
+      if (j < t && t < cn) {
+        for (int d = 0; d < D; ++d) acc = fmaf(Kc[t * LD + d], Kc[j * LD + d], acc);
+        acc *= B[t] * expf(G[t] - G[j]);
+      }
+      A[x] = acc;
+    }
+    // right-hand side: beta_t v_t - beta_t e^{G_t} S_0 k_t (this CTA's rows)
+    for (int x = tid; x < C * rn; x += THREADS) {
+      const int t = x / rn, i = x - t * rn;
+      float sk = 0.0f;
+      for (int d = 0; d < D; ++d) sk = fmaf(S[i * LD + d], Kc[t * LD + d], sk);
+      Vc[x] = B[t] * Vc[x] - B[t] * E[t] * sk;
+    }
+    __syncthreads();
+    // (I + A) U = rhs by forward substitution; thread i owns column i
+    if (tid < rn) {
+      const int i = tid;
+      for (int t = 1; t < cn; ++t) {
+        float acc = Vc[t * rn + i];
+        for (int j = 0; j < t; ++j) acc = fmaf(-A[t * C + j], Vc[j * rn + i], acc);
+        Vc[t * rn + i] = acc;
+      }
+    }
+    __syncthreads();
+    // P_tj = e^{G_t - G_j} (q_t . k_j), j <= t (into A)
+    for (int x = tid; x < C * C; x += THREADS) {
+      const int t = x / C, j = x - t * C;
+      float acc = 0.0f;
+      if (j <= t && t < cn) {
+        for (int d = 0; d < D; ++d) acc = fmaf(Qc[t * LD + d], Kc[j * LD + d], acc);
+        acc *= expf(G[t] - G[j]);
+      }
+      A[x] = acc;
+    }
+    __syncthreads();
+    // o_t = e^{G_t} S_0 q_t + sum_j P_tj U_j
+    for (int x = tid; x < cn * rn; x += THREADS) {
+      const int t = x / rn, i = x - t * rn;
+      float sq = 0.0f;
+      for (int d = 0; d < D; ++d) sq = fmaf(S[i * LD + d], Qc[t * LD + d], sq);
+      float pu = 0.0f;
+      for (int j = 0; j <= t; ++j) pu = fmaf(A[t * C + j], Vc[j * rn + i], pu);
+      a.o[((c0 + t) * a.Hv + h) * D + r0 + i] = E[t] * sq + pu;
+    }
+    const float gc = G[cn - 1];
+    if (tid < C) W[tid] = tid < cn ? expf(gc - G[tid]) : 0.0f;
+    __syncthreads();   // every output of the chunk read the old state; W is ready
+    // S = e^{G_C} S_0 + sum_t e^{G_C - G_t} U_t k_t^T
+    const float ec = expf(gc);
+    for (int x = tid; x < rn * D; x += THREADS) {
+      const int i = x / D, j = x - i * D;
+      float acc = ec * S[i * LD + j];
+      for (int t = 0; t < cn; ++t) acc = fmaf(Vc[t * rn + i] * W[t], Kc[t * LD + j], acc);
+      S[i * LD + j] = acc;
+    }
+  }
+  __syncthreads();
+  for (int x = tid; x < rn * D; x += THREADS) state[x] = S[(x / D) * LD + x % D];
+}
+
+}  // namespace nvfp4

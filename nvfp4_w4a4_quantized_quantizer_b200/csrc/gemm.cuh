@@ -35,6 +35,7 @@
 #include <cstdint>
 
 #include "ptx.cuh"
+#include "quantize.cuh"
 
 namespace nvfp4 {
 
@@ -59,7 +60,29 @@ struct GemmArgs {
   int sector_stores;   // y base 32-byte aligned and rows a multiple of 32 bytes
   int n_fastest;       // tile raster: 0 = M fastest (consecutive CTAs share a weight tile),
                        // 1 = N fastest (they share an activation tile)
+  // Last-wave K split (CTA-pair kernel): tiles [full_tiles, num_tiles) are each
+  // computed as `split` K-parts by split_units = (num_tiles - full_tiles) * split
+  // units; unit u (u < split_units) takes part u % split of tile
+  // full_tiles + u / split after its whole tiles.  split <= 1: no split.
+  // The parts meet in a caller-owned workspace: one arrival counter per
+  // (split tile, CTA of the pair), all zero between launches (the last part
+  // wraps its counter back to 0), and one fp32 partial tile per unit.
+  int full_tiles;
+  int split;
+  int split_units;
+  float* partial;      // [split_units][2 CTAs][2 halves][32 chunks][128 rows] float4
+  unsigned* counters;  // [num_tiles - full_tiles][2 CTAs]
   uint64_t wait_ns;
+  // SwiGLU epilogue (k_gemm_tc<2, true>): the weight is [gate; up], H rows
+  // each; tile column nb covers h columns [128 nb, 128 nb + 128) -- the even
+  // CTA loads those gate rows, the odd CTA the matching up rows -- and the
+  // epilogue writes h = bf16(silu(g) * u), g = bf16(alpha_gate * acc_gate),
+  // u = bf16(alpha_up * acc_up), quantised under h_gs: codes [M, H/2] and
+  // scales in the atom layout (the down projection's activation operand).
+  int H;
+  float alpha_gate, alpha_up, h_gs;
+  uint8_t* h_codes;
+  uint8_t* h_scales;
 };
 
 // ------------------------------------------------------------- epilogue op
@@ -137,6 +160,89 @@ __device__ __forceinline__ int seg_advance(const SegTable& t, int seg, int n) {
 // Tiles are walked M fastest (consecutive CTAs share a weight tile and the
 // activations stay in L2) or, when GemmArgs::n_fastest is set, N fastest
 // (they share an activation tile: for activations too large for the L2).
+// One unit of work of a CTA (pair): a whole tile (part < 0) or one K-part of
+// a tile of the last partial wave.
+struct WorkItem {
+  int tile;
+  int kt0, kt1;   // k-tiles [kt0, kt1)
+  int part;
+};
+
+__device__ __forceinline__ int work_full(const GemmArgs& g, int num_tiles) {
+  return g.split > 1 ? g.full_tiles : num_tiles;
+}
+
+__device__ __forceinline__ int work_count(const GemmArgs& g, int unit, int units, int num_tiles) {
+  const int full = work_full(g, num_tiles);
+  int n = unit < full ? (full - 1 - unit) / units + 1 : 0;
+  if (g.split > 1 && unit < g.split_units) ++n;
+  return n;
+}
+
+__device__ __forceinline__ WorkItem work_item(const GemmArgs& g, int unit, int units,
+                                              int num_tiles, int num_kt, int i) {
+  const int full = work_full(g, num_tiles);
+  const int nfull = unit < full ? (full - 1 - unit) / units + 1 : 0;
+  WorkItem w;
+  if (i < nfull) {
+    w.tile = unit + i * units;
+    w.kt0 = 0;
+    w.kt1 = num_kt;
+    w.part = -1;
+  } else {
+    w.tile = full + unit / g.split;
+    w.part = unit % g.split;
+    w.kt0 = w.part * num_kt / g.split;
+    w.kt1 = (w.part + 1) * num_kt / g.split;
+  }
+  return w;
+}
+
+// SwiGLU epilogue of one output row: g = bf16(alpha_gate * acc) for the 64
+// gate columns in v[0..63], u = bf16(alpha_up * acc) for the up columns in
+// v[64..127], h = bf16(silu(g) * u) (silu_mul_f32, as the standalone MLP
+// glue kernel computes it), then NVFP4 quantisation of h's four 16-blocks
+// under g.h_gs with exactly k_quantize's arithmetic: 32 code bytes at
+// h_codes[gm, h0 / 2] and the four scale bytes (one 32-bit word) at the
+// atom-layout position of blocks h0/16 .. h0/16 + 3.  Rows gm >= M store
+// only their scale word (zero).
+__device__ __forceinline__ void swiglu_store_row(const GemmArgs& g, int64_t gm, int h0,
+                                                 const uint32_t (&v)[128]) {
+  const float c = __fmul_rn(6.0f, g.h_gs);
+  uint32_t codes[8];
+  uint32_t word = 0;
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    float h[16];
+    uint32_t amax_bits = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float gv = __bfloat162float(__float2bfloat16_rn(__fmul_rn(g.alpha_gate, __uint_as_float(v[16 * b + i]))));
+      const float uv = __bfloat162float(__float2bfloat16_rn(__fmul_rn(g.alpha_up, __uint_as_float(v[64 + 16 * b + i]))));
+      h[i] = __bfloat162float(__float2bfloat16_rn(silu_mul_f32(gv, uv)));
+      // |h| max on the bit patterns (h is bf16-valued: exact)
+      const uint32_t mag = __float_as_uint(h[i]) & 0x7FFFFFFFu;
+      amax_bits = mag > amax_bits ? mag : amax_bits;
+    }
+    const uint32_t sc = cvt_e4m3(__fdiv_rn(__uint_as_float(amax_bits), c));
+    const float r = block_reciprocal(sc, g.h_gs);
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      float f[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) f[k] = __fmul_rn(h[8 * hh + k], r);
+      codes[2 * b + hh] = sc == 0 ? 0u : cvt_e2m1x8(f);
+    }
+    word |= sc << (8 * b);
+  }
+  if (gm < g.M) {
+    uint4* dst = reinterpret_cast<uint4*>(g.h_codes + gm * (g.H / 2) + h0 / 2);
+    dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+    dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+  }
+  *reinterpret_cast<uint32_t*>(g.h_scales + sf_offset(gm, h0 / 16, g.H)) = word;
+}
+
 namespace tc {
 constexpr int BM = 128;                 // rows of A per CTA
 constexpr int BN = 256;                 // tile columns (MMA N)
@@ -151,8 +257,7 @@ constexpr uint32_t REGS_EPI = 184;      // WG2 and WG3 after setmaxnreg
 static_assert(2 * 128 * REGS_SMALL + 2 * 128 * REGS_EPI <= 65536, "register split");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
-constexpr uint32_t SF_COL = 256;        // + 48 * stage
-constexpr uint32_t SF_STRIDE = 48;
+constexpr uint32_t SF_COL = 256;        // + SF_STRIDE * stage
 constexpr int BAR_BYTES = 256;
 
 template <int CG>
@@ -161,9 +266,16 @@ struct Cfg {
   static constexpr int A_BYTES = BM * BKB;                 // 16 KB
   static constexpr int B_BYTES = B_ROWS * BKB;             // 32 / 16 KB
   static constexpr int SFA_BYTES = 4 * 512;                // 4 atoms (K = 64 each) x 128 rows
-  static constexpr int SFB_BYTES = 2 * 4 * 512;            // both row blocks of the tile
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 54 / 38 KB
-  static constexpr int STAGES = CG == 1 ? 4 : 5;
+  // Weight scales: a one-CTA tile needs both 128-row blocks of its 256 rows;
+  // in a pair each CTA's MMA half reads the scales of the weight rows that
+  // CTA loaded, from its own TMEM, so each CTA loads only its own block.
+  static constexpr int SFB_BYTES = (CG == 1 ? 2 : 1) * 4 * 512;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 54 / 36 KB
+  static constexpr int STAGES = CG == 1 ? 4 : 6;
+  // TMEM scale region per stage: SFA 16 columns, then SFB 8 (CG 1) or 4
+  // (CG 2) columns per MMA
+  static constexpr uint32_t SFB_PER_MMA = CG == 1 ? 8 : 4;
+  static constexpr uint32_t SF_STRIDE = 16 + 4 * SFB_PER_MMA;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
   static_assert(SF_COL + STAGES * SF_STRIDE <= TMEM_COLS, "TMEM budget");
@@ -174,12 +286,14 @@ struct Cfg {
 // tmA / tmB: code matrices [rows, K/2] (box 128 bytes x 128 / (256 / CG)
 // rows, 128-byte swizzle).  tmSA / tmSB: scale buffers viewed as [row blocks]
 // [K/64 atoms][64 u64] (box 64 x 4 x 1 / 2, i.e. one stage's atoms of 1 / 2
-// row blocks).  CG = 2 must be launched with clusters of 2 CTAs.
-template <int CG>
+// row blocks).  CG = 2 must be launched with clusters of 2 CTAs.  SWIGLU
+// (CG = 2 only): the epilogue is the SwiGLU one described at GemmArgs::H.
+template <int CG, bool SWIGLU = false>
 __global__ void __launch_bounds__(tc::THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
               const GemmArgs g, const __grid_constant__ SegTable seg) {
+  static_assert(!SWIGLU || CG == 2, "the SwiGLU epilogue pairs gate and up rows across a CTA pair");
   using namespace tc;
   using C = Cfg<CG>;
   constexpr int STAGES = C::STAGES;
@@ -188,6 +302,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
   constexpr int B_BYTES = C::B_BYTES;
   constexpr int SFA_BYTES = C::SFA_BYTES;
   constexpr int SFB_BYTES = C::SFB_BYTES;
+  constexpr uint32_t SF_STRIDE = C::SF_STRIDE;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -202,9 +317,10 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
   const int unit = static_cast<int>(blockIdx.x) / CG;     // CTA (pair) index
   const int units = static_cast<int>(gridDim.x) / CG;
   const int num_m = (g.M + BM * CG - 1) / (BM * CG);
-  const int num_n = (g.N + BN - 1) / BN;
+  const int num_n = SWIGLU ? g.H / 128 : (g.N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
   const int num_kt = (g.K + BK - 1) / BK;
+  const int n_items = work_count(g, unit, units, num_tiles);
 
   auto full_bar = [&](int s) { return smem_addr(bars + s); };
   auto empty_bar = [&](int s) { return smem_addr(bars + STAGES + s); };
@@ -273,12 +389,16 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       uint32_t phase = 0;
       int64_t issued = 0;
       bool ok = true;
-      for (int tile = unit; tile < num_tiles && ok; tile += units) {
+      for (int it = 0; it < n_items && ok; ++it) {
+        const WorkItem w = work_item(g, unit, units, num_tiles, num_kt, it);
+        const int tile = w.tile;
         const int mb = g.n_fastest ? tile / num_n : tile % num_m;
         const int nb = g.n_fastest ? tile % num_n : tile / num_m;
         const int arow = (mb * CG + static_cast<int>(rank)) * BM;
-        const int brow = nb * BN + static_cast<int>(rank) * C::B_ROWS;
-        for (int kt = 0; kt < num_kt; ++kt) {
+        // SwiGLU: the even CTA's half of the tile is gate rows, the odd CTA's the up rows
+        const int brow = SWIGLU ? nb * 128 + (rank ? g.H : 0)
+                                : nb * BN + static_cast<int>(rank) * C::B_ROWS;
+        for (int kt = w.kt0; kt < w.kt1; ++kt) {
           if (!wait_pair(empty_bar(stage), phase ^ 1u)) {
             raise_abort(SITE_PRODUCER_EMPTY, warp);
             ok = false;
@@ -296,8 +416,12 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             mbar_arrive_expect_tx_warp(sfull_bar(stage), SFA_BYTES + SFB_BYTES);
             tma_load_3d_warp(smem_addr(st + A_BYTES + B_BYTES), &tmSA, 0, kt * 4,
                         mb * CG + static_cast<int>(rank), sfull_bar(stage), pol);
-            tma_load_3d_warp(smem_addr(st + A_BYTES + B_BYTES + SFA_BYTES), &tmSB, 0, kt * 4, nb * 2,
-                        sfull_bar(stage), pol);
+            // CG 2: this CTA's own weight-row block (tmSB has 1-block boxes);
+            // SwiGLU: the gate block nb (even CTA) or the up block H/128 + nb
+            const int sfb_block = SWIGLU ? nb + (rank ? g.H / 128 : 0)
+                                         : nb * 2 + (CG == 2 ? static_cast<int>(rank) : 0);
+            tma_load_3d_warp(smem_addr(st + A_BYTES + B_BYTES + SFA_BYTES), &tmSB, 0, kt * 4,
+                             sfb_block, sfull_bar(stage), pol);
           }
           ++issued;
           if (++stage == STAGES) {
@@ -323,9 +447,10 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     int stage = 0;
     uint32_t phase = 0;
-    for (int tile = unit; tile < num_tiles; tile += units) {
+    for (int it = 0; it < n_items; ++it) {
+      const WorkItem w = work_item(g, unit, units, num_tiles, num_kt, it);
       bool ok = true;
-      for (int kt = 0; kt < num_kt; ++kt) {
+      for (int kt = w.kt0; kt < w.kt1; ++kt) {
         if (!mbar_wait(sfull_bar(stage), phase, g.wait_ns, abort_flag)) {
           raise_abort(SITE_MMA_FULL, warp);
           ok = false;
@@ -343,18 +468,19 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
           r[4 * kk + 2] = a;
           r[4 * kk + 3] = a;
 #pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            // weight rows 128 j + 32 c + lane, c = 0..3 -> columns 8 kk + 4 j + c
+          for (int j = 0; j < (CG == 1 ? 2 : 1); ++j) {
+            // weight rows 128 j + 32 c + lane of the stage's blocks, c = 0..3
+            // -> columns SFB_PER_MMA kk + 4 j + c
             const uint4 b = ld_shared_v4(sfb_s + j * 2048 + kk * 512 + lane * 16);
-            r[16 + 8 * kk + 4 * j + 0] = b.x;
-            r[16 + 8 * kk + 4 * j + 1] = b.y;
-            r[16 + 8 * kk + 4 * j + 2] = b.z;
-            r[16 + 8 * kk + 4 * j + 3] = b.w;
+            r[16 + C::SFB_PER_MMA * kk + 4 * j + 0] = b.x;
+            r[16 + C::SFB_PER_MMA * kk + 4 * j + 1] = b.y;
+            r[16 + C::SFB_PER_MMA * kk + 4 * j + 2] = b.z;
+            r[16 + C::SFB_PER_MMA * kk + 4 * j + 3] = b.w;
           }
         }
         const uint32_t col = tmem_base + lane_off + SF_COL + SF_STRIDE * stage;
         tmem_st_x32(col, r);
-        tmem_st_x16(col + 32, r + 32);
+        if constexpr (CG == 1) tmem_st_x16(col + 32, r + 32);
         tmem_wait_st();
         tc_fence_before();
         // the MMA warp waits on this barrier alone: arrive only once the
@@ -391,14 +517,15 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
-      for (int tile = unit; tile < num_tiles && ok; tile += units, ++local) {
+      for (int it = 0; it < n_items && ok; ++it, ++local) {
+        const WorkItem w = work_item(g, unit, units, num_tiles, num_kt, it);
         if (!wait_pair(tmem_empty, static_cast<uint32_t>((local & 1) ^ 1))) {
           raise_abort(SITE_MMA_TMEM_EMPTY, 1);
           break;
         }
         tc_fence_after();
         int prev = -1;
-        for (int kt = 0; kt < num_kt; ++kt) {
+        for (int kt = w.kt0; kt < w.kt1; ++kt) {
           if (!wait_pair(sf_bar(stage), phase)) {
             raise_abort(SITE_MMA_FULL, 1);
             ok = false;
@@ -410,11 +537,11 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
           const uint64_t ad = adesc0 + soff, bd = bdesc0 + soff;
           const uint32_t col = tmem_base + SF_COL + SF_STRIDE * stage;
           // K = 64 fp4 = 32 bytes per MMA: advance the start address inside the swizzle atom
-          mma_mxf4nvf4_warp<CG>(tmem_base + ACC_COL, ad, bd, idesc, col, col + 16, kt != 0);
+          mma_mxf4nvf4_warp<CG>(tmem_base + ACC_COL, ad, bd, idesc, col, col + 16, kt != w.kt0);
           if (prev >= 0) tc_commit_all_warp<CG>(empty_bar(prev));
           for (int kk = 1; kk < nk; ++kk)
             mma_mxf4nvf4_warp<CG>(tmem_base + ACC_COL, ad + 2 * kk, bd + 2 * kk, idesc,
-                                col + 4 * kk, col + 16 + 8 * kk, 1u);
+                                col + 4 * kk, col + 16 + C::SFB_PER_MMA * kk, 1u);
           prev = stage;
           if (++stage == STAGES) {
             stage = 0;
@@ -436,69 +563,170 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     const int q = warp & 3;                       // TMEM lane quarter this warp may access
     const int half = (warp - EPI_WARP0) >> 2;     // columns [128*half, 128*half + 128)
     const int row_in_tile = q * 32 + lane;
-    int local = 0;
-    for (int tile = unit; tile < num_tiles; tile += units, ++local) {
-      const int mb = g.n_fastest ? tile / num_n : tile % num_m;
-      const int nb = g.n_fastest ? tile % num_n : tile / num_m;
-      if (!wait_pair(tmem_full, static_cast<uint32_t>(local & 1))) {
-        raise_abort(SITE_EPI_TMEM_FULL, warp);
-        break;
-      }
-      tc_fence_after();
-      uint32_t v[128];
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ACC_COL + half * 128;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld_x32(taddr + c * 32, v + c * 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) arrive_leader(tmem_empty);
-
+    // The output of one tile row: alpha / op, bf16 RNE (or fp32), store.
+    // fetch(grp, a) yields the fp32 accumulator bits of columns
+    // 16 grp .. 16 grp + 15 of this thread's 128.
+    // Rows past M skip only the stores: fetch may issue warp-collective
+    // TMEM loads, so every lane of the warp runs it.
+    auto store_row = [&](int mb, int nb, auto&& fetch) {
       const int64_t gm = static_cast<int64_t>(mb * CG + static_cast<int>(rank)) * BM + row_in_tile;
-      if (gm < g.M) {
-        const int n0 = nb * BN + half * 128;
-        int s = seg_advance(seg, 0, n0);
+      const bool row_live = gm < g.M;
+      const int n0 = nb * BN + half * 128;
+      int s = seg_advance(seg, 0, n0);
 #pragma unroll
-        for (int grp = 0; grp < 8; ++grp) {
-          const int n = n0 + grp * 16;
-          if (n < g.N) {
-            s = seg_advance(seg, s, n);
-            const float alpha = seg.alpha[s];
-            const int op = seg.op[s];
-            const int h0 = n - seg.n_off[s];
-            float o[16];
+      for (int grp = 0; grp < 8; ++grp) {
+        const int n = n0 + grp * 16;
+        if (n < g.N) {
+          s = seg_advance(seg, s, n);
+          const float alpha = seg.alpha[s];
+          const int op = seg.op[s];
+          const int h0 = n - seg.n_off[s];
+          uint32_t a[16];
+          fetch(grp, a);
+          float o[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) o[i] = __fmul_rn(alpha, __uint_as_float(v[grp * 16 + i]));
-            if (op != 0) {
-              float t[16];
+          for (int i = 0; i < 16; ++i) o[i] = __fmul_rn(alpha, __uint_as_float(a[i]));
+          if (op != 0) {
+            float t[16];
 #pragma unroll
-              for (int i = 0; i < 16; ++i) t[i] = o[i];
-              apply_op_16(t, op, seg.a_log[s], seg.dt_bias[s], h0);
+            for (int i = 0; i < 16; ++i) t[i] = o[i];
+            apply_op_16(t, op, seg.a_log[s], seg.dt_bias[s], h0);
 #pragma unroll
-              for (int i = 0; i < 16; ++i) o[i] = t[i];
+            for (int i = 0; i < 16; ++i) o[i] = t[i];
+          }
+          if (row_live && g.out_fp32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.y) + gm * g.ldy + n);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+          } else if (row_live) {
+            uint32_t w[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const __nv_bfloat162 p = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);
+              w[i] = *reinterpret_cast<const uint32_t*>(&p);
             }
-            if (g.out_fp32) {
-              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.y) + gm * g.ldy + n);
-#pragma unroll
-              for (int i = 0; i < 4; ++i)
-                dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.y) + gm * g.ldy + n;
+            if (g.sector_stores) {
+              st_global_v8(dst, w);   // the row's 16 columns = one full 32-byte sector
             } else {
-              uint32_t w[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const __nv_bfloat162 p = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);
-                w[i] = *reinterpret_cast<const uint32_t*>(&p);
-              }
-              __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.y) + gm * g.ldy + n;
-              if (g.sector_stores) {
-                st_global_v8(dst, w);   // the row's 16 columns = one full 32-byte sector
-              } else {
-                reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
-              }
+              reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+              reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
             }
           }
         }
+      }
+    };
+    // K-parts: chunk c (columns 4c..4c+3 of this thread's 128) of unit u's
+    // partial tile; for one chunk a warp's 32 rows are 512 contiguous bytes
+    auto part_chunk = [&](int u, int c) {
+      return reinterpret_cast<float4*>(g.partial) +
+             ((((static_cast<size_t>(u) * 2 + rank) * 2 + half) * 32 + c) * BM + row_in_tile);
+    };
+    volatile int* last_flag = abort_flag + 1;
+    int local = 0;
+    bool dead = false;   // a wait ran out: skip the work, keep every barrier
+    for (int it = 0; it < n_items; ++it, ++local) {
+      const WorkItem wi = work_item(g, unit, units, num_tiles, num_kt, it);
+      const int mb = g.n_fastest ? wi.tile / num_n : wi.tile % num_m;
+      const int nb = g.n_fastest ? wi.tile % num_n : wi.tile / num_m;
+      bool ok = !dead;
+      if (ok && !wait_pair(tmem_full, static_cast<uint32_t>(local & 1))) {
+        raise_abort(SITE_EPI_TMEM_FULL, warp);
+        dead = true;
+        ok = false;
+      }
+      uint32_t v[128];
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ACC_COL + half * 128;
+      if (ok) {
+        tc_fence_after();
+        if constexpr (SWIGLU) {
+          // this warp's 64 h columns: gate accumulator columns [64 half, +64)
+          // into v[0..63], the matching up columns [128 + 64 half, +64) into v[64..127]
+          const uint32_t lane_base = taddr - half * 128;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            tmem_ld_x32(lane_base + half * 64 + c * 32, v + c * 32);
+            tmem_ld_x32(lane_base + 128 + half * 64 + c * 32, v + 64 + c * 32);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld_x32(taddr + c * 32, v + c * 32);
+        }
+        tmem_wait_ld();
+        // A K-part is always a CTA's last item: no MMA waits for its
+        // accumulator, which stays in TMEM for the sum below.
+        if (wi.part < 0) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) arrive_leader(tmem_empty);
+        }
+      }
+      if constexpr (SWIGLU) {
+        // whole tiles only (the host never splits this launch); rows past M
+        // inside the last 128-row block still write their (zero) scale
+        // bytes: the scale buffer's padding rows must hold zeros
+        const int64_t gm = static_cast<int64_t>(mb * CG + static_cast<int>(rank)) * BM + row_in_tile;
+        const int64_t rows_padded = (static_cast<int64_t>(g.M) + 127) / 128 * 128;
+        if (ok && gm < rows_padded) swiglu_store_row(g, gm, nb * 128 + half * 64, v);
+        continue;
+      } else if (wi.part < 0) {
+        if (ok)
+          store_row(mb, nb, [&](int grp, uint32_t (&a)[16]) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) a[i] = v[grp * 16 + i];
+          });
+        continue;
+      }
+      // one K-part of a last-wave tile: publish it; the CTA that publishes
+      // the tile's last part sums all parts in part order and stores
+      if (ok) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          __stcg(part_chunk(unit, c),
+                 make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]),
+                             __uint_as_float(v[4 * c + 2]), __uint_as_float(v[4 * c + 3])));
+        __threadfence();
+      }
+      // Every epilogue warp passes both barriers once per part and every part
+      // counts itself, whatever its waits returned, so that each counter
+      // wraps back to zero (atomicInc with limit split - 1) in every launch.
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (warp == EPI_WARP0 && lane == 0) {
+        const unsigned idx = static_cast<unsigned>((wi.tile - g.full_tiles) * 2) + rank;
+        const unsigned lim = static_cast<unsigned>(g.split - 1);
+        *last_flag = atomicInc(g.counters + idx, lim) == lim;
+      }
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (ok && *last_flag && !*abort_flag) {
+        __threadfence();
+        // sum the parts in part order, whichever CTA is last, 16 columns at
+        // a time: this CTA's own part is re-read from TMEM (a K-part is a
+        // CTA's last item, so its accumulator was not released), the others
+        // come from the workspace
+        const int u0 = (wi.tile - g.full_tiles) * g.split;
+        const int mine = wi.part;
+        store_row(mb, nb, [&](int grp, uint32_t (&a)[16]) {
+          for (int p = 0; p < g.split; ++p) {
+            uint32_t t[16];
+            if (p == mine) {
+              tmem_ld_x16(taddr + grp * 16, t);
+              tmem_wait_ld();
+            } else {
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const float4 x = __ldcg(part_chunk(u0 + p, grp * 4 + c));
+                t[4 * c] = __float_as_uint(x.x);
+                t[4 * c + 1] = __float_as_uint(x.y);
+                t[4 * c + 2] = __float_as_uint(x.z);
+                t[4 * c + 3] = __float_as_uint(x.w);
+              }
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              a[i] = p == 0 ? t[i] : __float_as_uint(__uint_as_float(a[i]) + __uint_as_float(t[i]));
+          }
+        });
       }
     }
   }
@@ -527,7 +755,6 @@ constexpr int BW = 128;                 // weight rows per CTA (MMA M)
 constexpr int DIRECT_M = 8;             // up to this many tokens the epilogue stores directly
 constexpr int BK = 256;
 constexpr int BKB = BK / 2;
-constexpr int STAGES = 6;
 constexpr int W_BYTES = BW * BKB;       // 16 KB
 constexpr int SFW_BYTES = 4 * 512;
 constexpr int SFX_BYTES = 4 * 512;
@@ -540,24 +767,33 @@ constexpr uint32_t ACC_COL = 0;         // NT columns
 constexpr uint32_t SF_COL = 64;         // + 32 * stage
 constexpr uint32_t SF_STRIDE = 32;
 constexpr int BAR_BYTES = 256;
-static_assert(SF_COL + STAGES * SF_STRIDE <= TMEM_COLS, "TMEM budget");
+// Two CTAs fit on one SM (shared memory, 256 TMEM columns and <= 80
+// registers per thread each), so that with launch overlap the next call's
+// CTAs start streaming their weights beside this call's.
+constexpr int SMEM_PER_SM = 233472;     // 228 KB
+constexpr int SMEM_RESERVED = 1024;     // per CTA
 template <int NT>
 struct Cfg {
   static constexpr int X_BYTES = NT * BKB;   // NT rows x 128 bytes
   static constexpr int STAGE_BYTES = W_BYTES + X_BYTES + SFW_BYTES + SFX_BYTES;
+  static constexpr int STAGES = NT <= 16 ? 5 : (NT <= 32 ? 4 : 3);   // 22 / 24 / 28 KB stages
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
+  static_assert(SF_COL + STAGES * SF_STRIDE <= TMEM_COLS, "TMEM budget");
+  static_assert(2 * (SMEM_BYTES + SMEM_RESERVED) <= SMEM_PER_SM, "two CTAs per SM");
+  static_assert(NT * BW * 4 <= STAGES * STAGE_BYTES, "the epilogue's transpose fits the ring");
 };
 }  // namespace sm
 
 // tmW: weight codes [N, K/2]; tmX: token codes [M, K/2].  D (TMEM) is
 // [128 weight rows] x [NT tokens]; y[token, n] is written transposed back.
 template <int NT>
-__global__ void __launch_bounds__(sm::THREADS, 1)
+__global__ void __launch_bounds__(sm::THREADS, 2)
     k_gemm_small(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                  const GemmArgs g, const __grid_constant__ SegTable seg) {
   using namespace sm;
   using C = Cfg<NT>;
+  constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -599,11 +835,17 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // With launch overlap the next kernel may now be scheduled beside this one.
+  // Only the weight stream starts before the kernel ahead has finished: the
+  // token producer and the epilogue wait for it (griddep_wait) before they
+  // read the token operands or write y.
+  griddep_launch_dependents();
 
   if (warp == 0 || warp == 2) {
     // warp-wide loop; one elected lane issues each copy
     {
       const bool is_w = (warp == 0);
+      if (!is_w) griddep_wait();   // the token operands may come from the kernel ahead
       // weights stream through once; tokens are re-read by every CTA
       const uint64_t pol = is_w ? policy_evict_first() : policy_evict_last();
       int stage = 0;
@@ -723,6 +965,7 @@ __global__ void __launch_bounds__(sm::THREADS, 1)
     // every MMA has completed) so that each token's 128 columns leave as
     // 16-byte stores of one contiguous segment instead of M strided 2-byte
     // stores per thread.
+    griddep_wait();   // y may still be read or written by the kernel ahead
     const bool ok = mbar_wait(acc_full, 0, g.wait_ns, abort_flag);
     if (ok) {
       tc_fence_after();

@@ -100,6 +100,21 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
   }
 }
 
+// ------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start before
+// the kernel ahead of it on the stream has finished.  griddep_wait() returns
+// once that kernel has completed and its memory writes are visible (at once
+// when the launch had no such dependency); griddep_launch_dependents() lets
+// the kernel behind this one start once every CTA of this grid has issued it
+// or exited.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- clusters
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;

@@ -116,33 +116,48 @@ constexpr int QUANT_SMEM = QUANT_WARPS * QUANT_SLOTS * QUANT_UNIT * 2;   // 64 K
 constexpr int QUANT_BAR_BYTES = QUANT_WARPS * QUANT_SLOTS * 8;
 
 // |x| max of sixteen bf16 values (eight packed words), exact: the magnitude
-// bits of non-negative bf16 values order like unsigned integers.
+// bits of non-negative bf16 values order like unsigned integers, so one
+// 16-bit-lane unsigned max per word pair does it.
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 __device__ __forceinline__ float bf16x16_absmax(const uint32_t (&w)[8]) {
-  uint32_t m = __vmaxu2(w[0] & 0x7FFF7FFFu, w[1] & 0x7FFF7FFFu);
-  m = __vmaxu2(m, w[2] & 0x7FFF7FFFu);
-  m = __vmaxu2(m, w[3] & 0x7FFF7FFFu);
-  m = __vmaxu2(m, w[4] & 0x7FFF7FFFu);
-  m = __vmaxu2(m, w[5] & 0x7FFF7FFFu);
-  m = __vmaxu2(m, w[6] & 0x7FFF7FFFu);
-  m = __vmaxu2(m, w[7] & 0x7FFF7FFFu);
+  const uint32_t m01 = max_u16x2(w[0] & 0x7FFF7FFFu, w[1] & 0x7FFF7FFFu);
+  const uint32_t m23 = max_u16x2(w[2] & 0x7FFF7FFFu, w[3] & 0x7FFF7FFFu);
+  const uint32_t m45 = max_u16x2(w[4] & 0x7FFF7FFFu, w[5] & 0x7FFF7FFFu);
+  const uint32_t m67 = max_u16x2(w[6] & 0x7FFF7FFFu, w[7] & 0x7FFF7FFFu);
+  const uint32_t m = max_u16x2(max_u16x2(m01, m23), max_u16x2(m45, m67));
   const uint32_t hi = m >> 16, lo = m & 0xFFFFu;
   return __uint_as_float((hi > lo ? hi : lo) << 16);
 }
 
-// Elements of work unit u: row u / per_row, columns [c * QUANT_UNIT, +n).
-struct QuantUnit {
-  int64_t row;
-  int col;
-  int n;
-};
-
-__device__ __forceinline__ QuantUnit quant_unit(int64_t u, int per_row, int K) {
-  QuantUnit q;
-  q.row = u / per_row;
-  q.col = static_cast<int>(u - q.row * per_row) * QUANT_UNIT;
-  q.n = min(QUANT_UNIT, K - q.col);
-  return q;
+// The two bf16 values of a packed word times r, as two fp32 products each
+// rounded to nearest (one packed fp32 multiply; no flush of subnormals).
+__device__ __forceinline__ void bf16x2_times(uint32_t w, uint64_t rr, float& lo, float& hi) {
+  uint64_t x, d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "r"(w << 16), "r"(w & 0xFFFF0000u));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(x), "l"(rr));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(d));
 }
+
+// Position of a warp's current work unit (row, unit within the row).  A warp
+// visits units gwarp, gwarp + nwarps, ...; the cursor advances by nwarps
+// without a division (nwarps = step_rows * per_row + step_cols).
+struct UnitCursor {
+  int64_t row;
+  int col;       // unit index within the row
+  __device__ __forceinline__ void advance(int64_t step_rows, int step_cols, int per_row) {
+    row += step_rows;
+    col += step_cols;
+    if (col >= per_row) {
+      col -= per_row;
+      ++row;
+    }
+  }
+};
 
 __global__ void __launch_bounds__(QUANT_THREADS) k_quantize(const __grid_constant__ QuantArgs a) {
   extern __shared__ __align__(128) uint8_t qsmem[];
@@ -157,30 +172,41 @@ __global__ void __launch_bounds__(QUANT_THREADS) k_quantize(const __grid_constan
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * QUANT_WARPS;
   const float c = __fmul_rn(6.0f, a.gs);
   const int64_t code_ld = a.K / 2;
+  const int64_t kb4 = a.K / 64;                  // scale atoms per 128-row block along K
   const uint64_t pol = policy_evict_first();
+  const int64_t step_rows = nwarps / per_row;
+  const int step_cols = static_cast<int>(nwarps - step_rows * per_row);
+
+  // With launch overlap this grid may start before the kernel ahead of it
+  // has finished: let the kernel behind it be scheduled, then wait before
+  // reading x or writing codes and scales.
+  griddep_launch_dependents();
+  griddep_wait();
 
   if (lane == 0) {
     for (int s = 0; s < QUANT_SLOTS; ++s) mbar_init(smem_addr(bars + s), 1);
     fence_mbar_init();
   }
   __syncwarp();
-  // lane 0 starts the copy of the warp's i-th unit into slot i % QUANT_SLOTS
+  // lane 0 starts the copy of unit `at` (the warp's i-th) into slot i % QUANT_SLOTS
+  UnitCursor at{gwarp / per_row, static_cast<int>(gwarp % per_row)};
   auto issue = [&](int64_t i) {
-    const int64_t u = gwarp + i * nwarps;
-    if (u >= units) return;
-    const QuantUnit q = quant_unit(u, per_row, K);
+    if (at.row >= a.rows) return;
+    const int col = at.col * QUANT_UNIT;
+    const uint32_t bytes = static_cast<uint32_t>(min(QUANT_UNIT, K - col)) * 2u;
     const int s = static_cast<int>(i % QUANT_SLOTS);
-    const uint32_t bytes = static_cast<uint32_t>(q.n) * 2u;
     mbar_arrive_expect_tx(smem_addr(bars + s), bytes);
-    bulk_load(smem_addr(ring + s * (QUANT_UNIT * 2)), a.x + q.row * a.ldx + q.col, bytes,
+    bulk_load(smem_addr(ring + s * (QUANT_UNIT * 2)), a.x + at.row * a.ldx + col, bytes,
               smem_addr(bars + s), pol);
+    at.advance(step_rows, step_cols, per_row);
   };
   if (lane == 0)
     for (int i = 0; i < QUANT_SLOTS; ++i) issue(i);
 
+  UnitCursor cur{gwarp / per_row, static_cast<int>(gwarp % per_row)};
   int64_t i = 0;
   bool ok = true;
-  for (int64_t u = gwarp; u < units; u += nwarps, ++i) {
+  for (; cur.row < a.rows; cur.advance(step_rows, step_cols, per_row), ++i) {
     const int s = static_cast<int>(i % QUANT_SLOTS);
     if (!mbar_wait(smem_addr(bars + s), static_cast<uint32_t>((i / QUANT_SLOTS) & 1), a.wait_ns,
                    nullptr)) {
@@ -188,15 +214,20 @@ __global__ void __launch_bounds__(QUANT_THREADS) k_quantize(const __grid_constan
       ok = false;
       break;
     }
-    const QuantUnit q = quant_unit(u, per_row, K);
-    const int64_t grow = a.row0 + q.row;
+    const int col = cur.col * QUANT_UNIT;
+    const int n = min(QUANT_UNIT, K - col);
+    const int64_t grow = a.row0 + cur.row;
     const uint32_t slot = smem_addr(ring + s * (QUANT_UNIT * 2));
+    // this unit's code row and the scale bytes of its first 4-block group
+    uint8_t* code_row = a.codes + grow * code_ld + col / 2;
+    uint8_t* sf_unit = a.scales + ((grow >> 7) * kb4 + col / 64) * 512 + (grow & 31) * 16 +
+                       ((grow >> 5) & 3) * 4;
 #pragma unroll
     for (int p = 0; p < QUANT_UNIT / 512; ++p) {
       const int e0 = p * 512;
-      if (e0 >= q.n) break;                               // warp-uniform
+      if (e0 >= n) break;                                 // warp-uniform
       const int e = e0 + lane * 16;                       // this lane's block
-      const bool live = e < q.n;                          // uniform per 4 lanes (n % 64 == 0)
+      const bool live = e < n;                            // uniform per 4 lanes (n % 64 == 0)
       uint32_t w[8];
       // lanes 4..7 of each group of 8 read their halves in the other order,
       // so a quarter-warp's 16-byte reads cover all 32 banks once
@@ -209,15 +240,14 @@ __global__ void __launch_bounds__(QUANT_THREADS) k_quantize(const __grid_constan
       const float amax = bf16x16_absmax(w);
       const uint32_t sc = cvt_e4m3(__fdiv_rn(amax, c));
       const float rr = a.rtab[sc];
+      uint64_t rr2;
+      asm("mov.b64 %0, {%1, %1};" : "=l"(rr2) : "f"(rr));
       float f[8];
       uint32_t qv[2];
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          f[2 * k] = __fmul_rn(__uint_as_float(w[4 * hh + k] << 16), rr);
-          f[2 * k + 1] = __fmul_rn(__uint_as_float(w[4 * hh + k] & 0xFFFF0000u), rr);
-        }
+        for (int k = 0; k < 4; ++k) bf16x2_times(w[4 * hh + k], rr2, f[2 * k], f[2 * k + 1]);
         qv[hh] = cvt_e2m1x8(f);
       }
       if (sc == 0) qv[0] = qv[1] = 0u;
@@ -226,11 +256,11 @@ __global__ void __launch_bounds__(QUANT_THREADS) k_quantize(const __grid_constan
       const uint32_t s2 = __shfl_down_sync(0xffffffffu, sc, 2);
       const uint32_t s3 = __shfl_down_sync(0xffffffffu, sc, 3);
       if (live) {
-        const int k = q.col + e;
-        *reinterpret_cast<uint2*>(a.codes + grow * code_ld + k / 2) = make_uint2(qv[0], qv[1]);
+        *reinterpret_cast<uint2*>(code_row + e / 2) = make_uint2(qv[0], qv[1]);
         if ((lane & 3) == 0) {
+          // blocks e/16 .. e/16 + 3 of the unit: atom (e / 64) after the unit's first
           const uint32_t word = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
-          *reinterpret_cast<uint32_t*>(a.scales + sf_offset(grow, k / 16, a.K)) = word;
+          *reinterpret_cast<uint32_t*>(sf_unit + (e / 64) * 512) = word;
         }
       }
     }
@@ -298,6 +328,21 @@ __global__ void __launch_bounds__(AMAX_THREADS) k_amax(const __nv_bfloat16* __re
 }
 
 // ------------------------------------------------------- MLP glue (SiLU*up)
+// h = fp32(silu(g) * u) for bf16-valued g and u: g / (1 + e^-g) with an
+// IEEE divide, then the product, each step rounded to nearest and none
+// contracted (the fused gate_up epilogue computes the same function, so
+// both paths give identical h).
+__device__ __forceinline__ float silu_mul_f32(float g, float u) {
+  return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+}
+
+// Block reciprocal of scale code `code` under global scale gs:
+// fp32(1 / fp32(e4m3(code) * gs)), 0 for code 0 -- the entry of k_quantize's
+// host-built table, computed on the device with the same two roundings.
+__device__ __forceinline__ float block_reciprocal(uint32_t code, float gs) {
+  return code == 0 ? 0.0f : __frcp_rn(__fmul_rn(e4m3_value(code), gs));
+}
+
 constexpr int SILU_THREADS = 256;
 
 __global__ void __launch_bounds__(SILU_THREADS) k_silu_mul(const __nv_bfloat16* __restrict__ gu,
@@ -316,12 +361,43 @@ __global__ void __launch_bounds__(SILU_THREADS) k_silu_mul(const __nv_bfloat16* 
     uint32_t w[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float a0 = __fmul_rn(__fdiv_rn(g[2 * e], 1.0f + expf(-g[2 * e])), u[2 * e]);
-      const float a1 = __fmul_rn(__fdiv_rn(g[2 * e + 1], 1.0f + expf(-g[2 * e + 1])), u[2 * e + 1]);
+      const float a0 = silu_mul_f32(g[2 * e], u[2 * e]);
+      const float a1 = silu_mul_f32(g[2 * e + 1], u[2 * e + 1]);
       const __nv_bfloat162 p = __floats2bfloat162_rn(a0, a1);
       w[e] = *reinterpret_cast<const uint32_t*>(&p);
     }
     *reinterpret_cast<uint4*>(h + m * ld_out + j) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// ------------------------------------------------------ FP8 (E4M3) KV cache
+// The pages' other shipped recipe: KV-cache tensors in FP8 E4M3 under a
+// calibrated per-tensor scale.  code = sign | E4M3_RNE_satfinite(fp32(x * r))
+// with r = fp32(1 / scale) formed on the host; eight bf16 in (16 bytes),
+// eight codes out (8 bytes) per thread and step.  HBM-bound.
+constexpr int KV_THREADS = 256;
+
+// Two fp32 values -> two E4M3 codes, a in the low byte (the PTX conversion
+// puts its first source in the high byte).
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float a, float b) {
+  uint16_t out;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(b), "f"(a));
+  return static_cast<uint32_t>(out);
+}
+
+__global__ void __launch_bounds__(KV_THREADS) k_kv_fp8(const __nv_bfloat16* __restrict__ x,
+                                                       int64_t n8, float r,
+                                                       uint2* __restrict__ out) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * KV_THREADS + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * KV_THREADS) {
+    float f[8];
+    bf16x8_to_f32(ld_stream_v4(x + i * 8), f);
+    uint32_t w[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      w[h] = cvt_e4m3x2(__fmul_rn(f[4 * h], r), __fmul_rn(f[4 * h + 1], r)) |
+             (cvt_e4m3x2(__fmul_rn(f[4 * h + 2], r), __fmul_rn(f[4 * h + 3], r)) << 16);
+    out[i] = make_uint2(w[0], w[1]);
   }
 }
 

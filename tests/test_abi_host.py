@@ -113,6 +113,19 @@ def test_fused_linear_validation(lib):
     assert f(*args(ok, 2, M=0)) == 0                          # no-op
 
 
+def test_gemm_workspace(lib):
+    # arrival counters + 128 fp32 partial tiles of 2 x 128 x 256
+    assert lib.nvfp4_gemm_workspace_bytes() == 4096 + 128 * 2 * 128 * 256 * 4
+    f = lib.nvfp4_fused_linear_ws
+    ok = _segs((0, 0), (32, 1))
+    args = lambda work, M=8, K=128: (P, P, P, P, M, 64, K, ok, 2, P, 64, 0, work,  # noqa: E731
+                                     lib.nvfp4_gemm_workspace_bytes(), NUL)
+    assert f(*args(P_MIS)) == ALIGN                           # workspace not 16-byte aligned
+    assert f(*args(P, K=96)) == SHAPE                         # the fused_linear checks apply
+    assert f(*args(P, M=0)) == 0
+    assert f(*args(NUL, M=0)) == 0                            # no workspace: plain fused_linear
+
+
 def test_linear_and_weight_validation(lib):
     assert lib.nvfp4_linear(P, P, 1.0, P, P, 1.0, 4, 64, 64, NUL, 64, 0, NUL) == INVALID
     assert lib.nvfp4_linear(P, P, -1.0, P, P, 1.0, 4, 64, 64, P, 64, 0, NUL) == INVALID
@@ -127,10 +140,40 @@ def test_linear_and_weight_validation(lib):
     assert w(P, 64, 64, 64, None, 1, gs, P, P, NUL, NUL) == INVALID  # workspace required
 
 
+def test_gate_up_silu_quantize_validation(lib):
+    f = lib.nvfp4_gate_up_silu_quantize
+    args = lambda M=8, H=128, K=128, hc=P, gs=1.0: (P, P, P, P, M, H, K, 1.0, 1.0, 1.0, gs, hc, P,  # noqa: E731
+                                                   NUL)
+    assert f(*args(H=192)) == SHAPE                           # H % 128
+    assert f(*args(H=0)) == SHAPE
+    assert f(*args(K=96)) == SHAPE                            # K % 64
+    assert f(*args(hc=NUL)) == INVALID
+    assert f(*args(hc=P_MIS)) == ALIGN
+    assert f(*args(gs=0.0)) == INVALID
+    assert f(*args(gs=float("nan"))) == INVALID
+    assert f(*args(M=0)) == 0
+
+
+def test_kv_fp8_validation(lib):
+    assert lib.nvfp4_kv_scale(ctypes.c_float(448.0)) == 1.0
+    assert lib.nvfp4_kv_scale(ctypes.c_float(0.0)) == 1.0
+    q = lib.nvfp4_kv_quantize_fp8
+    assert q(NUL, 8, 1.0, P, NUL) == INVALID
+    assert q(P, 12, 1.0, P, NUL) == SHAPE                     # n % 8
+    assert q(P, -8, 1.0, P, NUL) == SHAPE
+    assert q(P_MIS, 8, 1.0, P, NUL) == ALIGN
+    assert q(P, 8, 1.0, P_MIS, NUL) == ALIGN
+    assert q(P, 8, 0.0, P, NUL) == INVALID
+    assert q(P, 0, 1.0, P, NUL) == 0
+
+
 def test_misc_validation(lib):
     assert lib.nvfp4_set_gemm_path(5) == INVALID
     assert lib.nvfp4_set_gemm_path(0) == 0
     assert lib.nvfp4_set_wait_limit_ns(0) == INVALID
+    assert lib.nvfp4_set_launch_overlap(2) == INVALID
+    assert lib.nvfp4_set_launch_overlap(1) == 0
+    assert lib.nvfp4_set_launch_overlap(0) == 0
     assert lib.nvfp4_silu_mul(P, 4, 12, 24, P, 12, NUL) == SHAPE       # H % 8
     assert lib.nvfp4_amax(P, 4, 64, 64, NUL, NUL) == INVALID
     assert lib.nvfp4_test_e2m1(NUL, P, 4, NUL) == INVALID

@@ -18,6 +18,8 @@ import workloads
 import nvfp4_w4a4_quantized_quantizer_b200 as nv
 from tests import _helpers as H
 
+_H = H  # the helpers, where a parameter named H (the MLP hidden size) shadows them
+
 pytestmark = pytest.mark.gpu
 
 LARGE, SMALL, AUTO, PAIR, PAIR_NFAST = 1, 2, 0, 3, 4
@@ -120,3 +122,97 @@ def test_repair_vs_shared_scale():
                                    atol=1e-6 * np.abs(yb[:, sl]).max())
         if i > 0:
             assert abs(ratio - 1) > 1e-3        # the modules really do differ
+
+
+# ------------------------------------------ MLP first half in one kernel
+def _gate_up_operands(M, H, K, seed):
+    rng = np.random.default_rng(seed)
+    xb = workloads.random_bf16((M, K), seed=seed, std=1.0)
+    std_g, std_u = 1 / np.sqrt(K), 3 / np.sqrt(K)          # up weights 3x the gate's scale
+    wb = np.concatenate([workloads.random_bf16((H, K), seed=seed + 1, std=std_g),
+                         workloads.random_bf16((H, K), seed=seed + 2, std=std_u)])
+    a_gs = float(oracle.global_scale(np.abs(_H.f32(xb)).max()))
+    ac, as_ = nv.nvfp4_quantize_act(_H.bf16_dev(xb), a_gs)
+    wc, ws, (g_gs, u_gs) = nv.nvfp4_quantize_weight(_H.bf16_dev(wb), seg_offsets=[0, H])
+    return ac, as_, wc, ws, a_gs, g_gs, u_gs, rng
+
+
+
+@pytest.mark.parametrize("M,H,K", [(100, 128, 256), (256, 384, 512), (300, 256, 1280),
+                                   (600, 640, 320), (2304, 1024, 256)])
+def test_gate_up_silu_quantize_equals_the_unfused_chain(M, H, K):
+    """One kernel = fused_linear (bf16, gate | up) -> silu_mul -> quantize_act, bit for bit,
+    padding rows of the scale buffer included."""
+    ac, as_, wc, ws, a_gs, g_gs, u_gs, _ = _gate_up_operands(M, H, K, seed=M + H + K)
+    segs = [nv.SegmentSpec(0, g_gs, a_gs), nv.SegmentSpec(H, u_gs, a_gs)]
+    nv.nvfp4_set_gemm_path(PAIR)        # the fused kernel is a CTA-pair kernel at every M
+    gu = nv.nvfp4_fused_linear(ac, as_, wc, ws, M, 2 * H, K, segs)
+    nv.nvfp4_set_gemm_path(AUTO)
+    h = nv.nvfp4_silu_mul(gu, H)
+    h_gs = float(oracle.global_scale(float(h.float().abs().max().item())))
+    ref_c, ref_s = nv.nvfp4_quantize_act(h, h_gs)
+    hc = torch.full((M, H // 2), 0xAB, dtype=torch.uint8, device="cuda")
+    hs = torch.full((nv.nvfp4_scale_bytes(M, H),), 0xCD, dtype=torch.uint8, device="cuda")
+    nv.nvfp4_gate_up_silu_quantize(ac, as_, wc, ws, M, H, K, a_gs, g_gs, u_gs, h_gs,
+                                   h_codes=hc, h_scales=hs)
+    st, info = nv.nvfp4_last_device_error()
+    assert st == 0, f"device error word {info:#x}"
+    assert torch.equal(hc, ref_c)
+    assert torch.equal(hs, ref_s)
+
+
+def test_silu_mul_matches_the_oracle_within_one_bf16_step():
+    """nvfp4_silu_mul (fp32 steps) against the float64 oracle on the same bf16 gate / up."""
+    M, Hd = 64, 4096
+    rng = np.random.default_rng(3)
+    g = workloads.f32_to_bf16_bits(rng.normal(0, 3, (M, Hd)).astype(np.float32))
+    u = workloads.f32_to_bf16_bits(rng.normal(0, 2, (M, Hd)).astype(np.float32))
+    gu = np.concatenate([g, u], axis=1)
+    h = nv.nvfp4_silu_mul(H.bf16_dev(gu), Hd).float().cpu().numpy()
+    ref = oracle.silu_mul_bf16(H.f32(g), H.f32(u))
+    # both are bf16-rounded: at most one bf16 step apart (fp32 vs float64 inner steps)
+    step = np.abs(ref).astype(np.float64) * 2.0 ** -7 + 1e-30
+    assert np.all(np.abs(h.astype(np.float64) - ref) <= step)
+    assert np.mean(h == ref) > 0.99
+
+
+@pytest.mark.parametrize("path,M,K", [(PAIR, 200, 320), (SMALL, 7, 320), (LARGE, 100, 256)])
+def test_preharmonised_checkpoint(path, M, K):
+    """The pages' other repair: every module of the fused weight quantised under
+    one shared global scale ("pre-harmonised"), served with that scale in every
+    segment; gates still apply per module."""
+    widths, ops, wbits, xbits, a_log, dt = _mini_gdn(M, K, seed=M + 5)
+    N = sum(widths)
+    offs = np.cumsum([0] + widths[:-1]).tolist()
+    xf, wf = H.f32(xbits), H.f32(wbits)
+    a_gs = oracle.global_scale(np.abs(xf).max())
+    ac, as_ = nv.nvfp4_quantize_act(H.bf16_dev(xbits), float(a_gs))
+    wc, ws, (w_gs,) = nv.nvfp4_quantize_weight(H.bf16_dev(wbits))          # one module
+    gs_ref = oracle.global_scale(np.abs(wf).max())
+    assert np.float32(w_gs) == gs_ref
+    a_log_d, dt_d = torch.from_numpy(a_log).cuda(), torch.from_numpy(dt).cuda()
+    specs = [nv.SegmentSpec(o, w_gs, float(a_gs), OPS[ops[i]],
+                            a_log_d if ops[i] == "gdn_decay" else None,
+                            dt_d if ops[i] == "gdn_decay" else None)
+             for i, o in enumerate(offs)]
+    nv.nvfp4_set_gemm_path(path)
+    y32 = nv.nvfp4_fused_linear(ac, as_, wc, ws, M, N, K, specs, out_dtype=nv.OUT_FP32)
+    assert nv.nvfp4_last_device_error()[0] == 0
+    y32 = y32.cpu().numpy()
+    qx, sx = oracle.quantize(xf, a_gs)
+    qw, sw = oracle.quantize(wf, gs_ref)
+    np.testing.assert_array_equal(H.unpack_codes(wc.cpu().numpy()), qw)
+    segs = [dict(n_offset=o, width=wd, w_gs=gs_ref, a_gs=a_gs, op=ops[i], a_log=a_log, dt_bias=dt)
+            for i, (o, wd) in enumerate(zip(offs, widths))]
+    ref = oracle.fused_linear64(qx, sx, qw, sw, segs)
+    pre = oracle.fused_linear64(qx, sx, qw, sw, [dict(s, op="none") for s in segs])
+    for o, wd, op in zip(offs, widths, ops):
+        sl = slice(o, o + wd)
+        e = 1e-3 * np.sqrt(np.mean(pre[:, sl] ** 2))
+        if op == "none":
+            H.check_gemm_fp32(y32[:, sl], ref[:, sl], f"harmonised segment at {o}")
+        elif op == "sigmoid":
+            assert np.all(np.abs(y32[:, sl] - ref[:, sl]) <= 0.25 * e + 2e-6)
+        else:
+            bound = np.exp(a_log)[None, :] * e + 2e-5 * np.abs(ref[:, sl]) + 1e-6
+            assert np.all(np.abs(y32[:, sl] - ref[:, sl]) <= bound)

@@ -201,3 +201,150 @@ def test_bf16_row_stride_both_store_widths(ldy, path):
     out = y.float().cpu().numpy()
     assert np.all(out[:, N:] == 3.0)
     np.testing.assert_array_equal(out[:, :N], H.bf16_round(y32.cpu().numpy()))
+
+
+# ------------------------------------------------------------ launch overlap
+@pytest.fixture
+def overlap():
+    nv.nvfp4_set_launch_overlap(True)
+    yield
+    nv.nvfp4_set_launch_overlap(False)
+
+
+def _decode_layer(M, N, K, seed):
+    xb = workloads.random_bf16((M, K), seed=seed, std=1.0)
+    wb = workloads.random_bf16((N, K), seed=seed + 1, std=1 / np.sqrt(K))
+    a_gs = float(oracle.global_scale(np.abs(H.f32(xb)).max()))
+    wc, ws, (w_gs,) = nv.nvfp4_quantize_weight(H.bf16_dev(wb))
+    return xb, wb, a_gs, wc, ws, w_gs
+
+
+@pytest.mark.parametrize("M", [1, 8, 17, 40, 64])
+def test_overlap_gives_identical_results(M, overlap):
+    """quantise + small-M GEMM chains with launch overlap on equal the plain launches bit for bit."""
+    N, K = 1040, 2048
+    xb, _, a_gs, wc, ws, w_gs = _decode_layer(M, N, K, seed=M)
+    nv.nvfp4_set_launch_overlap(False)
+    ac, as_ = nv.nvfp4_quantize_act(H.bf16_dev(xb), a_gs)
+    ref = nv.nvfp4_linear(ac, as_, a_gs, wc, ws, w_gs, M, N, K, out_dtype=nv.OUT_FP32).cpu()
+    nv.nvfp4_set_launch_overlap(True)
+    x = H.bf16_dev(xb)
+    for _ in range(3):
+        ac2, as2 = nv.nvfp4_quantize_act(x, a_gs)
+        y = nv.nvfp4_linear(ac2, as2, a_gs, wc, ws, w_gs, M, N, K, out_dtype=nv.OUT_FP32)
+        assert torch.equal(y.cpu(), ref)
+        assert torch.equal(ac2.cpu(), ac.cpu()) and torch.equal(as2.cpu(), as_.cpu())
+    assert nv.nvfp4_last_device_error()[0] == 0
+
+
+def test_overlap_keeps_stream_order_of_shared_buffers(overlap):
+    """Consecutive layers sharing one code buffer and one output buffer: the
+    quantiser of layer i+1 must not overwrite the codes layer i's GEMM still
+    reads, and each GEMM must read the codes just written (read-after-write,
+    write-after-read and write-after-write through the same buffers)."""
+    M, N, K = 16, 2064, 1024
+    layers = [_decode_layer(M, N, K, seed=100 + 7 * i) for i in range(4)]
+    nv.nvfp4_set_launch_overlap(False)
+    expect = []
+    for xb, _, a_gs, wc, ws, w_gs in layers:
+        ac, as_ = nv.nvfp4_quantize_act(H.bf16_dev(xb), a_gs)
+        expect.append(nv.nvfp4_linear(ac, as_, a_gs, wc, ws, w_gs, M, N, K, out_dtype=nv.OUT_FP32).cpu())
+    nv.nvfp4_set_launch_overlap(True)
+    xs = [H.bf16_dev(l[0]) for l in layers]
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+    scales = torch.empty(nv.nvfp4_scale_bytes(M, K), dtype=torch.uint8, device="cuda")
+    outs = [torch.empty((M, N), dtype=torch.float32, device="cuda") for _ in layers]
+    y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    for rep in range(5):
+        # one code buffer, back-to-back quantise / GEMM launches
+        for i, (_, _, a_gs, wc, ws, w_gs) in enumerate(layers):
+            nv.nvfp4_quantize_act(xs[i], a_gs, codes=codes, scales=scales)
+            nv.nvfp4_linear(codes, scales, a_gs, wc, ws, w_gs, M, N, K, y=outs[i],
+                            out_dtype=nv.OUT_FP32)
+        for i in range(len(layers)):
+            assert torch.equal(outs[i].cpu(), expect[i]), (rep, i)
+        # one output buffer: the last GEMM's result stays
+        for i, (_, _, a_gs, wc, ws, w_gs) in enumerate(layers):
+            nv.nvfp4_quantize_act(xs[i], a_gs, codes=codes, scales=scales)
+            nv.nvfp4_linear(codes, scales, a_gs, wc, ws, w_gs, M, N, K, y=y, out_dtype=nv.OUT_FP32)
+        assert torch.equal(y.cpu(), expect[-1]), rep
+    assert nv.nvfp4_last_device_error()[0] == 0
+
+
+# ------------------------------------------------- last-wave K split (workspace)
+# Shapes with more 256 x 256 tiles than a B200's 74 CTA pairs and a partial
+# last wave: 180 tiles (32 left, 2 parts of 1 k-tile), 320 tiles (24 left,
+# 3 parts of 1-2 k-tiles), ragged M and N inside the split tiles.
+@pytest.mark.parametrize("path,M,N,K", [
+    (PAIR, 2304, 5120, 512), (PAIR, 4096, 5120, 1280), (PAIR, 2200, 5104, 512),
+    (PAIR_NFAST, 2304, 5120, 512), (AUTO, 4096, 5120, 1280)])
+def test_split_last_wave(path, M, N, K):
+    rng = np.random.default_rng(M * 17 + N + K)
+    ac = rng.integers(0, 16, size=(M, K)).astype(np.uint8)
+    wc = rng.integers(0, 16, size=(N, K)).astype(np.uint8)
+    as_ = rng.integers(0x28, 0x58, size=(M, K // 16)).astype(np.uint8)
+    ws = rng.integers(0x28, 0x58, size=(N, K // 16)).astype(np.uint8)
+    a_gs, w_gs = np.float32(0.0173), np.float32(0.00291)
+    A, W = dev_operands(ac, as_, M, K), dev_operands(wc, ws, N, K)
+    seg = [nv.SegmentSpec(0, float(w_gs), float(a_gs))]
+    work = nv.nvfp4_gemm_workspace("cuda")
+    nv.nvfp4_set_gemm_path(path)
+    y32 = nv.nvfp4_fused_linear(A[0], A[1], W[0], W[1], M, N, K, seg, out_dtype=nv.OUT_FP32,
+                                workspace=work)
+    y32b = nv.nvfp4_fused_linear(A[0], A[1], W[0], W[1], M, N, K, seg, out_dtype=nv.OUT_FP32,
+                                 workspace=work)
+    yb = nv.nvfp4_fused_linear(A[0], A[1], W[0], W[1], M, N, K, seg, workspace=work)
+    st, info = nv.nvfp4_last_device_error()
+    assert st == 0, f"device error word {info:#x}"
+    # every call leaves the arrival counters at zero
+    assert int(work[:4096].count_nonzero()) == 0
+    y32, y32b = y32.cpu().numpy(), y32b.cpu().numpy()
+    # the parts are summed in a fixed order: no run-to-run variation
+    np.testing.assert_array_equal(y32, y32b)
+    ref = oracle.linear64(oracle.dequantize(ac, as_, a_gs), oracle.dequantize(wc, ws, w_gs))
+    H.check_gemm_fp32(y32, ref, f"split {M}x{N}x{K}")
+    H.check_bf16_out(yb.float().cpu().numpy(), y32, ref, f"split {M}x{N}x{K}")
+
+
+def test_split_with_gates_and_small_workspace():
+    """GDN gate segments inside split tiles; a workspace too small for two
+    parts per leftover tile gives exactly the unsplit result."""
+    M, N, K = 2304, 5120, 512
+    rng = np.random.default_rng(5)
+    ac = rng.integers(0, 16, size=(M, K)).astype(np.uint8)
+    wc = rng.integers(0, 16, size=(N, K)).astype(np.uint8)
+    as_ = rng.integers(0x28, 0x58, size=(M, K // 16)).astype(np.uint8)
+    ws = rng.integers(0x28, 0x58, size=(N, K // 16)).astype(np.uint8)
+    A, W = dev_operands(ac, as_, M, K), dev_operands(wc, ws, N, K)
+    width = 128
+    a_log = torch.from_numpy(rng.uniform(-1, 1.5, width).astype(np.float32)).cuda()
+    dt_bias = torch.from_numpy(rng.normal(0, 0.5, width).astype(np.float32)).cuda()
+    seg = [nv.SegmentSpec(0, 0.002, 0.02), nv.SegmentSpec(N - 2 * width, 0.003, 0.02, nv.OP_SIGMOID),
+           nv.SegmentSpec(N - width, 0.004, 0.02, nv.OP_GDN_DECAY, a_log, dt_bias)]
+    nv.nvfp4_set_gemm_path(PAIR)
+    plain = nv.nvfp4_fused_linear(A[0], A[1], W[0], W[1], M, N, K, seg, out_dtype=nv.OUT_FP32)
+    work = nv.nvfp4_gemm_workspace("cuda")
+    split = nv.nvfp4_fused_linear(A[0], A[1], W[0], W[1], M, N, K, seg, out_dtype=nv.OUT_FP32,
+                                  workspace=work)
+    tiny = torch.zeros(4096 + 262144, dtype=torch.uint8, device="cuda")
+    unsplit = nv.nvfp4_fused_linear(A[0], A[1], W[0], W[1], M, N, K, seg, out_dtype=nv.OUT_FP32,
+                                    workspace=tiny)
+    st, info = nv.nvfp4_last_device_error()
+    assert st == 0, f"device error word {info:#x}"
+    np.testing.assert_array_equal(unsplit.cpu().numpy(), plain.cpu().numpy())
+    xa = oracle.dequantize(ac, as_, np.float32(0.02))
+    pre = np.concatenate([oracle.linear64(xa, oracle.dequantize(wc[:N - 2 * width], ws[:N - 2 * width], np.float32(0.002))),
+                          oracle.linear64(xa, oracle.dequantize(wc[N - 2 * width:N - width], ws[N - 2 * width:N - width], np.float32(0.003))),
+                          oracle.linear64(xa, oracle.dequantize(wc[N - width:], ws[N - width:], np.float32(0.004)))], axis=1)
+    out = split.cpu().numpy()
+    # gate bars: e = 1e-3 rms of the module's pre-activation through the
+    # gates' Lipschitz constants, as in the fused-projection tests
+    b_sl, g_sl = slice(N - 2 * width, N - width), slice(N - width, N)
+    H.check_gemm_fp32(out[:, :N - 2 * width], pre[:, :N - 2 * width], "split none")
+    e_b = 1e-3 * np.sqrt(np.mean(pre[:, b_sl] ** 2))
+    assert np.all(np.abs(out[:, b_sl] - oracle.sigmoid64(pre[:, b_sl])) <= 0.25 * e_b + 2e-6)
+    e_g = 1e-3 * np.sqrt(np.mean(pre[:, g_sl] ** 2))
+    a_log64 = a_log.cpu().numpy().astype(np.float64)
+    g_ref = oracle.gdn_decay64(pre[:, g_sl], a_log64, dt_bias.cpu().numpy().astype(np.float64))
+    bound = np.exp(a_log64)[None, :] * e_g + 2e-5 * np.abs(g_ref) + 1e-6
+    assert np.all(np.abs(out[:, g_sl] - g_ref) <= bound)
