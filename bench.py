@@ -370,23 +370,20 @@ def time_steps(layer: Layer, steps: int, warmup: int, stream):
     return replay_ms(seq, stream)
 
 
-def time_each(fns, reps: int, stream):
+MIN_KERNEL_S = 0.2          # every per-kernel figure is averaged over at least this much device time
+
+
+def time_each(fns, stream, min_s: float = MIN_KERNEL_S):
     """Mean device time (ms) of each named launch alone: a graph of
-    GRAPH_STEPS launches of it, replayed `reps` times."""
+    GRAPH_STEPS launches of it, replayed until at least `min_s` seconds of
+    device time are covered (the replay count is sized from a first replay)."""
     graphs = {name: capture(fn, 0, GRAPH_STEPS, stream) for name, fn in fns.items()}
-    replay_ms(list(graphs.values()), stream)
-    return {name: replay_ms([g] * reps, stream) / (reps * GRAPH_STEPS) for name, g in graphs.items()}
-
-
-def time_kernels(layer: Layer, reps: int, stream):
-    """Mean device time of each kernel alone: graphs of GRAPH_STEPS quantiser
-    launches and of GRAPH_STEPS GEMM launches, each replayed `reps` times."""
-    gq = capture(lambda i, st: layer.quantize(i, st), 0, GRAPH_STEPS, stream)
-    gg = capture(lambda i, st: layer.gemm(i, st), 0, GRAPH_STEPS, stream)
-    replay_ms([gq, gg], stream)
-    q_ms = replay_ms([gq] * reps, stream) / (reps * GRAPH_STEPS)
-    g_ms = replay_ms([gg] * reps, stream) / (reps * GRAPH_STEPS)
-    return q_ms, g_ms
+    out = {}
+    for name, g in graphs.items():
+        first = replay_ms([g], stream)                      # uploads the graph
+        reps = max(2, int(np.ceil(min_s * 1e3 / max(first, 1e-3))))
+        out[name] = replay_ms([g] * reps, stream) / (reps * GRAPH_STEPS)
+    return out
 
 
 def e2e(layer: Layer, steps: int, warmup: int, stream):
@@ -438,7 +435,7 @@ def e2e(layer: Layer, steps: int, warmup: int, stream):
     return ms, xh.numel() * 2, yh[0].numel() * 2
 
 
-def small_m_sweep(device, stream, iters=240, warmup=10):
+def small_m_sweep(device, stream, warmup=10):
     """Decode-shaped sweep on the fused GDN in-projection weights: weight-stream
     GB/s of the GEMM alone (graph replays over the rotated weight copies)."""
     import nvfp4_w4a4_quantized_quantizer_b200 as nv
@@ -462,10 +459,7 @@ def small_m_sweep(device, stream, iters=240, warmup=10):
         def gemm(i, st):
             wc, ws = base.ws[i % len(base.ws)]
             nv.nvfp4_fused_linear(c, s, wc, ws, M, base.N, base.K, base.segs, y=y, stream=st)
-        g = capture(gemm, 0, GRAPH_STEPS, stream)
-        replay_ms([g], stream)
-        reps = max(1, iters // GRAPH_STEPS)
-        g_ms = replay_ms([g] * reps, stream) / (reps * GRAPH_STEPS)
+        g_ms = time_each({"gemm": gemm}, stream)["gemm"]
         out[f"M={M}"] = {"gemm_us": round(g_ms * 1e3, 2),
                          "weight_GBps": round(base.weight_bytes / (g_ms * 1e-3) / 1e9, 1),
                          "tokens_per_s": round(M / (g_ms * 1e-3), 1)}
@@ -473,7 +467,7 @@ def small_m_sweep(device, stream, iters=240, warmup=10):
 
 
 # ------------------------------------------------------------ CPU oracle
-def kv_fp8_rate(device, stream, reps=20):
+def kv_fp8_rate(device, stream):
     """FP8 KV-cache quantisation of one layer's K (32768 tokens x 8 heads x
     128 dims, bf16 -> E4M3 under a calibrated scale), rotated over 3 copies
     (201 MB > L2): graph replay of GRAPH_STEPS launches.  3 bytes per element."""
@@ -488,7 +482,7 @@ def kv_fp8_rate(device, stream, reps=20):
     def run(i, st):
         nv.nvfp4_kv_quantize_fp8(xs[i % 3], s, out=out, stream=st)
 
-    t = time_each({"kv": run}, reps, stream)["kv"]
+    t = time_each({"kv": run}, stream)["kv"]
     gbs = 3.0 * n / (t * 1e-3) / 1e9
     return {"elements": n, "us": round(t * 1e3, 2), "GBps": round(gbs, 1)}
 
@@ -497,7 +491,7 @@ def kv_fp8_rate(device, stream, reps=20):
 FP32_ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
-def gdn_rate(device, stream, reps=4):
+def gdn_rate(device, stream):
     """The gated delta rule over 8192 tokens of the GDN in-projection's heads
     (48 value heads over 16 key heads, width 128), graph replay.  FLOPs
     counted as the definition's 6 D^2 per token and value head."""
@@ -518,7 +512,7 @@ def gdn_rate(device, stream, reps=4):
         nv.nvfp4_gdn_recurrence(ins["q"], ins["k"], ins["v"], ins["g"], ins["beta"], group=group,
                                 state=state, o=o, stream=st)
 
-    t = time_each({"gdn": run}, reps, stream)["gdn"]
+    t = time_each({"gdn": run}, stream)["gdn"]
     tflops = 6.0 * D * D * T * Hv / (t * 1e-3) / 1e12
     return {"tokens": T, "value_heads": Hv, "us": round(t * 1e3, 1),
             "tokens_per_s": round(T / (t * 1e-3), 1), "tflops": round(tflops, 2),
@@ -526,76 +520,192 @@ def gdn_rate(device, stream, reps=4):
             "frac": round(tflops / FP32_ALU_PEAK_TFLOPS, 4)}
 
 
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        return os.cpu_count()
+
+
 class OracleSample:
-    """The oracle, as it stands, on bounded samples of the workload: quantise a
-    few activation rows, dequantise, float64 GEMM against the dequantised
-    weights (static: quantised and dequantised once, outside the timing)."""
+    """The oracle, as it stands, on bounded row samples of a workload.  One
+    step = the layer's path for `rows` activation rows: the oracle quantiser,
+    then dequantisation and the float64 GEMM against the weights (quantised
+    and dequantised once, outside the timing).  For the MLP pair the step is
+    quantise x -> gate_up -> SiLU(gate) * up -> quantise h -> down.  The
+    quantiser phases and the GEMM phases (dequantise + float64 product) are
+    timed separately."""
 
     def __init__(self, wl: workloads.Workload):
         import oracle
         self.oracle, self.wl = oracle, wl
+        self.mlp = wl.name.startswith("mlp")
         f32 = workloads.bf16_bits_to_f32
         calib = f32(workloads.activations(wl, calib=True))
         self.a_gs = oracle.global_scale(np.abs(calib).max())
-        wf = f32(workloads.weights(wl))
-        self.what = np.empty(wf.shape, np.float64)
-        for s, off in zip(wl.segments, wl.seg_offsets):
-            sl = slice(off, off + s.width)
-            gs = oracle.global_scale(np.abs(wf[sl]).max())
-            q, sc = oracle.quantize(wf[sl], gs)
-            self.what[sl] = oracle.dequantize(q, sc, gs)
+        self.what = self._dequantized_weights(f32(workloads.weights(wl)), wl.seg_offsets, wl.N)
+        if self.mlp:
+            self.H, self.N2 = wl.N // 2, workloads.MLP_DOWN_N
+            w2 = f32(workloads.down_weights())
+            self.w2hat = self._dequantized_weights(w2, [0], self.N2)
+            del w2
+            # the down input's static scale: the oracle chain on the calibration batch
+            h = self._silu(self._gemm(calib, self.a_gs, self.what))
+            self.a2_gs = oracle.global_scale(np.abs(h).max())
         self.x = f32(workloads.activations(wl, rows=(0, min(256, wl.M))))
-        try:
-            from threadpoolctl import threadpool_info
-            self.threads = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
-        except Exception:  # pragma: no cover
-            self.threads = os.cpu_count()
+        self.threads = _threads()
+
+    def _dequantized_weights(self, wf, offs, N):
+        out = np.empty(wf.shape, np.float64)
+        ends = list(offs[1:]) + [N]
+        for o, e in zip(offs, ends):
+            gs = self.oracle.global_scale(np.abs(wf[o:e]).max())
+            q, sc = self.oracle.quantize(wf[o:e], gs)
+            out[o:e] = self.oracle.dequantize(q, sc, gs)
+        return out
+
+    def _gemm(self, x, gs, what):
+        q, sc = self.oracle.quantize(x, gs)
+        return self.oracle.linear64(self.oracle.dequantize(q, sc, gs), what)
+
+    def _silu(self, gu):
+        return self.oracle.silu_mul_bf16(gu[:, :self.H], gu[:, self.H:])
 
     def run(self, rows: int):
-        q, sc = self.oracle.quantize(self.x[:rows], self.a_gs)
-        return self.oracle.linear64(self.oracle.dequantize(q, sc, self.a_gs), self.what)
+        """One step; returns (quantiser seconds, GEMM seconds)."""
+        o, tq, tg = self.oracle, 0.0, 0.0
+        t0 = time.perf_counter()
+        q, sc = o.quantize(self.x[:rows], self.a_gs)
+        t1 = time.perf_counter()
+        y = o.linear64(o.dequantize(q, sc, self.a_gs), self.what)
+        t2 = time.perf_counter()
+        tq, tg = t1 - t0, t2 - t1
+        if self.mlp:
+            h = self._silu(y)
+            t3 = time.perf_counter()
+            q2, s2 = o.quantize(h, self.a2_gs)
+            t4 = time.perf_counter()
+            o.linear64(o.dequantize(q2, s2, self.a2_gs), self.w2hat)
+            t5 = time.perf_counter()
+            tq += t4 - t2            # SiLU * up + requantisation: the MLP glue
+            tg += t5 - t4
+        return tq, tg
 
     def flops(self, rows: int) -> float:
-        return 2.0 * rows * self.wl.N * self.wl.K
+        f = 2.0 * rows * self.wl.N * self.wl.K
+        return f + (2.0 * rows * self.H * self.N2 if self.mlp else 0.0)
+
+    def quant_bytes(self, rows: int) -> float:
+        """Algorithmic bytes of the step's quantiser phases (2.5625 B per element)."""
+        return 2.5625 * rows * (self.wl.K + (self.H if self.mlp else 0))
 
     def describe(self, rows: int, reps: int, el: float) -> str:
-        return (f"{rows} activation rows x K={self.wl.K} x N={self.wl.N} per step: oracle quantise + "
-                f"dequantise + float64 GEMM vs pre-dequantised weights; {reps} steps in {el:.1f} s")
+        what = ("quantise x, dequantise + float64 gate_up GEMM, SiLU(gate)*up, quantise h, "
+                "dequantise + float64 down GEMM" if self.mlp else
+                "quantise, dequantise + float64 GEMM")
+        return (f"{rows} activation rows per step of {self.wl.name} (full K and N): oracle {what}, "
+                f"weights pre-dequantised; {reps} steps in {el:.1f} s")
 
     def timed(self, rows: int, steps: int, warmup: int):
+        """(step TFLOP/s, elapsed s, quantiser GB/s, GEMM TFLOP/s) over `steps` steps."""
         for _ in range(warmup):
             self.run(rows)
+        tq = tg = 0.0
         t0 = time.perf_counter()
         for _ in range(steps):
-            self.run(rows)
+            a, b = self.run(rows)
+            tq += a
+            tg += b
         el = time.perf_counter() - t0
-        return self.flops(rows) * steps / el / 1e12, el
+        gemm_flops = self.flops(rows) * steps
+        return (gemm_flops / el / 1e12, el, self.quant_bytes(rows) * steps / tq / 1e9,
+                gemm_flops / tg / 1e12)
 
 
-def cpu_baseline(wl: workloads.Workload, target_s: float = 12.0, rows: int = 32):
-    s = OracleSample(wl)
+def cpu_baseline(samp: OracleSample, target_s: float = 12.0, rows: int = 32):
     t0 = time.perf_counter()
-    s.run(rows)
+    samp.run(rows)
     t1 = time.perf_counter() - t0
     steps = max(1, int(target_s / max(t1, 1e-3)))
-    tflops, el = s.timed(rows, steps, 0)
-    return {"value": round(tflops, 6), "unit": "TFLOPS", "cores": s.threads, "kind": "oracle",
-            "sample": s.describe(rows, steps, el)}
+    tflops, el, q_gbs, g_tflops = samp.timed(rows, steps, 0)
+    return {"value": round(tflops, 6), "unit": "TFLOPS", "cores": samp.threads, "kind": "oracle",
+            "sample": samp.describe(rows, steps, el), "quantize_GBps": round(q_gbs, 4),
+            "gemm_tflops": round(g_tflops, 6)}
 
 
 # ------------------------------------------------------------------ main
 WORKLOAD_BY_NAME = {"prefill": 2, "gdn_inproj": 3, "mlp": 4, "decode": 5}
 
 
+def config_shape(wl: workloads.Workload) -> dict:
+    if wl.name.startswith("mlp"):
+        return {"M": wl.M, "K": wl.K, "N_gate_up": wl.N, "N_down": workloads.MLP_DOWN_N,
+                "K_down": workloads.MLP_DOWN_K}
+    return {"M": wl.M, "N": wl.N, "K": wl.K}
+
+
+def layer_kernels(layer, pk, stream, fp4_peak):
+    """Per-kernel device times of one workload's launches, each timed alone,
+    with their roofline fractions (FP4 tensor peak for GEMMs, HBM for the
+    quantiser)."""
+    nv = layer.nv
+    q_bytes = layer.M * layer.K * 2 + layer.M * layer.K // 2 + nv.nvfp4_scale_bytes(layer.M, layer.K)
+    if isinstance(layer, MlpChain):
+        t = time_each({"quantize": layer.quantize, "gate_up": layer.gate_up, "down": layer.down}, stream)
+        gemms = {"gate_up": 2.0 * layer.M * layer.K * layer.N, "down": 2.0 * layer.M * layer.H * layer.N2}
+    else:
+        t = time_each({"quantize": layer.quantize, "gemm": layer.gemm}, stream)
+        gemms = {"gemm": layer.flops}
+    out = {"quantize_us": round(t["quantize"] * 1e3, 2),
+           "quantize_GBps": round(q_bytes / (t["quantize"] * 1e-3) / 1e9, 1)}
+    out["quantize_hbm_frac"] = round(out["quantize_GBps"] / pk["hbm"], 4)
+    for name, flops in gemms.items():
+        tf = flops / (t[name] * 1e-3) / 1e12
+        out[f"{name}_us"] = round(t[name] * 1e3, 2)
+        out[f"{name}_tflops"] = round(tf, 1)
+        out[f"{name}_frac"] = round(tf / fp4_peak, 4)
+    return out
+
+
+def reference_main(args, wl, rank):
+    """--impl reference: the oracle as it stands on this machine's host cores,
+    on the same workload, metric and unit, each step a bounded row sample."""
+    if rank != 0:
+        return
+    samp = OracleSample(wl)
+    t0 = time.perf_counter()
+    samp.run(1)
+    t1 = time.perf_counter() - t0
+    budget = 120.0 / (args.steps + args.warmup)          # whole run within a few minutes
+    rows = int(np.clip(budget / max(t1, 1e-4), 1, 256))
+    tflops, el, q_gbs, g_tflops = samp.timed(rows, args.steps, args.warmup)
+    line = {"metric": METRIC, "value": round(tflops, 6), "unit": "TFLOPS", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(el / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": wl.name, **config_shape(wl), "sample_rows_per_step": rows},
+            "cpu_baseline": {"value": round(tflops, 6), "unit": "TFLOPS", "cores": samp.threads,
+                             "kind": "oracle", "sample": samp.describe(rows, args.steps, el),
+                             "quantize_GBps": round(q_gbs, 4), "gemm_tflops": round(g_tflops, 6)},
+            "e2e": {"value": round(tflops, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=4000)
-    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--workload", default="prefill", choices=sorted(WORKLOAD_BY_NAME))
+    ap.add_argument("--workload", default="mlp", choices=sorted(WORKLOAD_BY_NAME),
+                    help="the timed step (default: the MLP pair, the largest configuration)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-small-m", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-kernel figures of the other large configurations")
     ap.add_argument("--no-overlap", action="store_true",
                     help="launch the quantiser and the small-M GEMM without launch overlap")
     args = ap.parse_args()
@@ -606,27 +716,7 @@ def main():
     M = wl.M
 
     if args.impl == "reference":
-        if rank != 0:
-            return
-        samp = OracleSample(wl)
-        t0 = time.perf_counter()
-        samp.run(1)
-        t1 = time.perf_counter() - t0
-        budget = 120.0 / (args.steps + args.warmup)          # whole run within a few minutes
-        rows = int(np.clip(budget / max(t1, 1e-4), 1, 256))
-        tflops, el = samp.timed(rows, args.steps, args.warmup)
-        line = {"metric": METRIC, "value": round(tflops, 6), "unit": "TFLOPS", "n_gpus": args.gpus,
-                "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": round(el / args.steps * 1e3, 3),
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                "data": "synthetic", "impl": "reference",
-                "config": {"workload": wl.name, "M": M, "N": wl.N, "K": wl.K,
-                           "sample_rows_per_step": rows},
-                "cpu_baseline": {"value": round(tflops, 6), "unit": "TFLOPS", "cores": samp.threads,
-                                 "kind": "oracle", "sample": samp.describe(rows, args.steps, el)},
-                "e2e": {"value": round(tflops, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0,
-                        "d2h_bytes_per_step": 0}}
-        print(json.dumps(line), flush=True)
+        reference_main(args, wl, rank)
         return
 
     import nvfp4_w4a4_quantized_quantizer_b200 as nv
@@ -647,43 +737,31 @@ def main():
     mlp = args.workload == "mlp"
     layer = MlpChain(device) if mlp else Layer(wl, M, device)
     torch.cuda.synchronize()
+    pk = peaks()
+    fp4_peak = pk["bf16"] * FP4_PER_BF16
 
-    # main timed region: barrier + sync on both sides, max over ranks
     with ClockSampler(local) as clk:
+        # main timed region: exactly K steps, barrier + sync on both sides, max over ranks
         total_ms = timed_region(pg, lambda: time_steps(layer, args.steps, args.warmup, stream),
                                 torch.cuda.synchronize)
+        # per-kernel device times (graphs of one kernel each, >= MIN_KERNEL_S per kernel)
+        kern = {wl.name: layer_kernels(layer, pk, stream, fp4_peak)}
     clocks = clk.summary()
     total_ms = max_over_ranks(total_ms, pg, device)
     ms_step = total_ms / args.steps
     value = job_value(ws, layer.flops, ms_step)
 
-    # per-kernel device times (separate pass: graphs of one kernel each)
-    reps = max(4, min(args.steps, 480) // GRAPH_STEPS)
-    pk = peaks()
-    fp4_peak = pk["bf16"] * FP4_PER_BF16
     if mlp:
-        t = time_each({"quantize": layer.quantize, "gate_up": layer.gate_up, "down": layer.down},
-                      max(2, reps // 4), stream)
-        q_ms, g_ms = t["quantize"], t["gate_up"]
-        g_flops = 2.0 * layer.M * layer.K * layer.N           # the dominant kernel: gate_up
-        d_tflops = 2.0 * layer.M * layer.H * layer.N2 / (t["down"] * 1e-3) / 1e12
-        extra = {"down_us": round(t["down"] * 1e3, 2), "down_tflops": round(d_tflops, 1),
-                 "down_frac": round(d_tflops / fp4_peak, 4)}
+        g_name, g_flops = "gate_up", 2.0 * layer.M * layer.K * layer.N     # the dominant kernel
         step_desc = ("quantize_act + gate_up (2 modules) with SiLU(gate)*up and its requantisation "
                      "in the epilogue + down GEMM (bf16 out)")
-        cfg_shape = {"M": layer.M, "K": layer.K, "N_gate_up": layer.N, "N_down": layer.N2,
-                     "K_down": layer.H}
         profile = f"gemm_tc_{wl.name}.md"
     else:
-        q_ms, g_ms = time_kernels(layer, reps, stream)
-        g_flops = layer.flops
-        extra = {}
+        g_name, g_flops = "gemm", layer.flops
         step_desc = "quantize_act + fused NVFP4 GEMM (bf16 out)"
-        cfg_shape = {"M": M, "N": wl.N, "K": wl.K}
         profile = f"gemm_tc_{wl.name}.md"
+    g_ms = kern[wl.name][f"{g_name}_us"] * 1e-3
     g_tflops = g_flops / (g_ms * 1e-3) / 1e12
-    q_bytes = layer.M * layer.K * 2 + layer.M * layer.K // 2 + nv.nvfp4_scale_bytes(layer.M, layer.K)
-    q_gbs = q_bytes / (q_ms * 1e-3) / 1e9
     traffic = ncu_traffic(profile)
 
     e_ms, h2d, d2h = e2e(layer, max(20, min(200, args.steps // 20)), 3, stream)
@@ -692,40 +770,47 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4",
         "data": "synthetic",
-        "config": {"workload": wl.name, **cfg_shape,
+        "config": {"workload": wl.name, **config_shape(wl),
                    "step": step_desc,
                    "l2": f"inputs rotated over {len(layer.xs)} activation / {len(layer.ws)} weight copies "
                          "(working set > L2)", "parallelism": f"replicas x{ws}",
                    "launch": f"steps replayed from CUDA graphs of {GRAPH_STEPS} steps; launch overlap "
                              + ("off" if args.no_overlap else "on (quantiser, small-M GEMM)")},
-        "roofline": {"bound": "tensor", "achieved": round(g_tflops, 1), "peak": round(fp4_peak, 1),
-                     "unit": "TFLOP/s", "frac": round(g_tflops / fp4_peak, 4),
+        "roofline": {"bound": "tensor", "kernel": g_name, "achieved": round(g_tflops, 1),
+                     "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(g_tflops / fp4_peak, 4),
                      "traffic": traffic,
-                     "peak_note": f"{pk['source']} bf16 burst {pk['bf16']} x {FP4_PER_BF16} nominal FP4/BF16",
-                     # the same kernel against the sustained (power-capped) figure: the timed
-                     # region is thousands of back-to-back launches with sw_power_cap active
-                     "peak_sustained": round(pk["bf16_sus"] * FP4_PER_BF16, 1),
-                     "frac_sustained": round(g_tflops / (pk["bf16_sus"] * FP4_PER_BF16), 4)},
-        "kernels": {"gemm_us": round(g_ms * 1e3, 2), "gemm_tflops": round(g_tflops, 1),
-                    "quantize_us": round(q_ms * 1e3, 2), "quantize_GBps": round(q_gbs, 1),
-                    "quantize_hbm_frac": round(q_gbs / pk["hbm"], 4), **extra},
+                     "peak_note": f"{pk['source']} bf16 burst {pk['bf16']} x {FP4_PER_BF16} nominal "
+                                  "FP4/BF16 (the kernel is timed alone, >= 0.2 s of graph replays)"},
+        "kernels": kern,
         "e2e": {"value": round(layer.flops / (e_ms * 1e-3) / 1e12, 2), "unit": "TFLOPS",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": (layer.launches_per_step if mlp else 2) * args.steps,
         "clocks": clocks,
     }
-    if rank == 0 and not args.no_small_m and ws == 1:
+    single = rank == 0 and ws == 1
+    if single and not args.no_configs:
+        # the other large configurations' kernels, each timed alone
+        for name in ("prefill", "gdn_inproj", "mlp"):
+            w2 = workloads.WORKLOADS[WORKLOAD_BY_NAME[name]]
+            if w2.name in kern:
+                continue
+            other = MlpChain(device) if name == "mlp" else Layer(w2, w2.M, device)
+            with ClockSampler(local) as clk2:
+                kern[w2.name] = layer_kernels(other, pk, stream, fp4_peak)
+            kern[w2.name]["clocks"] = clk2.summary()
+            del other
+            torch.cuda.empty_cache()
+    if single and not args.no_small_m:
         sm = small_m_sweep(device, stream)
         for v in sm.values():
             v["hbm_frac"] = round(v["weight_GBps"] / pk["hbm"], 4)
         line["small_m"] = sm
-    if rank == 0 and not args.no_small_m and ws == 1:
         kv = kv_fp8_rate(device, stream)
         kv["hbm_frac"] = round(kv["GBps"] / pk["hbm"], 4)
         line["kv_fp8"] = kv
         line["gdn_recurrence"] = gdn_rate(device, stream)
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl)
+    if single and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(OracleSample(wl))
     if rank == 0:
         print(json.dumps(line), flush=True)
     if pg:

@@ -54,6 +54,12 @@
  * Streams: `stream` is a cudaStream_t (NULL = legacy default stream).  All
  * calls are asynchronous on that stream except nvfp4_quantize_weight() and
  * nvfp4_last_device_error(), which synchronise it.
+ *
+ * Per-device state: the library caches, per device, its capability checks,
+ * kernel attributes, occupancy figures and TMA descriptors (keyed by
+ * pointer and shape).  They stay valid for the life of the device's primary
+ * context; after cudaDeviceReset the library must not be called on that
+ * device again in the same process.
  */
 #ifndef NVFP4_H_
 #define NVFP4_H_
@@ -170,13 +176,20 @@ nvfp4_status nvfp4_quantize_weight(const void* w_bf16, int64_t N, int64_t K, int
  * device current; make that first call before any stream capture.  All
  * calls share the one array per device: the accumulators are cleared on
  * `stream` at the start of every call, and calls whose work overlaps on the
- * GPU (e.g. on different streams) race on it.  Arguments, layouts and the
+ * GPU (e.g. on different streams) race on it.  The looked-up address is kept
+ * for the life of the process: after cudaDeviceReset (or any teardown of the
+ * device's primary context) it no longer names the array, so the library
+ * must not be called on that device again.  Arguments, layouts and the
  * synchronisation of `stream` are those of nvfp4_quantize_weight. */
 #define NVFP4_NOALLOC_MAX_SEGMENTS 32
 nvfp4_status nvfp4_quantize_weight_noalloc(const void* w_bf16, int64_t N, int64_t K, int64_t ldw,
                                            const int64_t* seg_offsets, int32_t nseg,
                                            float* w_gs_out, void* codes, void* scales,
                                            nvfp4_stream_t stream);
+/* The module limit of nvfp4_quantize_weight_noalloc as compiled into the
+ * library (NVFP4_NOALLOC_MAX_SEGMENTS), for callers that bind the library
+ * without this header. */
+int32_t nvfp4_noalloc_max_segments(void);
 
 /* Block-scaled FP4 x FP4 GEMM (step a3) with a single module (step a4 with
  * op NONE): y[m, n] = fp32(a_gs * w_gs) * sum_k e2m1(qa[m,k]) sa[m,k/16]

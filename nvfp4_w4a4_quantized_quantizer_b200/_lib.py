@@ -17,7 +17,6 @@ STATUS_NAMES = {0: "NVFP4_OK", -1: "NVFP4_ERR_INVALID_ARG", -2: "NVFP4_ERR_ALIGN
 OP_NONE, OP_SIGMOID, OP_GDN_DECAY = 0, 1, 2
 OUT_BF16, OUT_FP32 = 0, 1
 MAX_SEGMENTS = 32
-NOALLOC_MAX_SEGMENTS = 32
 
 # Every symbol include/nvfp4.h declares, with (restype, argtypes).
 _vp, _i64, _i32, _u64, _f32, _sz = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32,
@@ -40,6 +39,7 @@ SIGNATURES = {
     "nvfp4_quantize_weight_workspace_bytes": (_sz, [_i32]),
     "nvfp4_quantize_weight": (_st, [_vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _vp]),
     "nvfp4_quantize_weight_noalloc": (_st, [_vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp]),
+    "nvfp4_noalloc_max_segments": (_i32, []),
     "nvfp4_linear": (_st, [_vp, _vp, _f32, _vp, _vp, _f32, _i64, _i64, _i64, _vp, _i64, _st, _vp]),
     "nvfp4_fused_linear": (_st, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.POINTER(Segment), _i32,
                                  _vp, _i64, _st, _vp]),

@@ -660,7 +660,7 @@ nvfp4_status nvfp4_fused_linear_ws(const void* a_codes, const void* a_scales, co
   if ((st = code_map(w_codes, N, K / 2, nvfp4::tc::BN / (pair ? 2 : 1), dev, &tb)) != NVFP4_OK)
     return st;
   if ((st = scale_map(a_scales, M, K, 1, dev, &tsa)) != NVFP4_OK) return st;
-  if ((st = scale_map(w_scales, N, K, pair ? 1 : 2, dev, &tsb)) != NVFP4_OK) return st;
+  if ((st = scale_map(w_scales, N, K, 2, dev, &tsb)) != NVFP4_OK) return st;
   const int64_t num_n = (N + nvfp4::tc::BN - 1) / nvfp4::tc::BN;
   if (!pair) {
     constexpr int smem = nvfp4::tc::Cfg<1>::SMEM_BYTES;
@@ -713,6 +713,8 @@ nvfp4_status nvfp4_fused_linear_ws(const void* a_codes, const void* a_scales, co
   }
   return check_launch();
 }
+
+int32_t nvfp4_noalloc_max_segments(void) { return NVFP4_NOALLOC_MAX_SEGMENTS; }
 
 nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales, const void* w_codes,
                                 const void* w_scales, int64_t M, int64_t N, int64_t K,

@@ -266,15 +266,17 @@ struct Cfg {
   static constexpr int A_BYTES = BM * BKB;                 // 16 KB
   static constexpr int B_BYTES = B_ROWS * BKB;             // 32 / 16 KB
   static constexpr int SFA_BYTES = 4 * 512;                // 4 atoms (K = 64 each) x 128 rows
-  // Weight scales: a one-CTA tile needs both 128-row blocks of its 256 rows;
-  // in a pair each CTA's MMA half reads the scales of the weight rows that
-  // CTA loaded, from its own TMEM, so each CTA loads only its own block.
-  static constexpr int SFB_BYTES = (CG == 1 ? 2 : 1) * 4 * 512;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 54 / 36 KB
-  static constexpr int STAGES = CG == 1 ? 4 : 6;
-  // TMEM scale region per stage: SFA 16 columns, then SFB 8 (CG 1) or 4
-  // (CG 2) columns per MMA
-  static constexpr uint32_t SFB_PER_MMA = CG == 1 ? 8 : 4;
+  // Weight scales: both 128-row blocks of the tile's 256 weight rows, in
+  // either kernel.  In a CTA pair each CTA's half of a cta_group::2 MMA (its
+  // own 128 output rows) reads the scales of all 256 weight rows from its
+  // own TMEM: a layout experiment that left one half of them out (NaN scale
+  // codes) in either CTA turned half of that CTA's output columns into NaN.
+  static constexpr int SFB_BYTES = 2 * 4 * 512;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 54 / 38 KB
+  static constexpr int STAGES = CG == 1 ? 4 : 5;
+  // TMEM scale region per stage: SFA 16 columns (4 per MMA), then SFB 32
+  // columns (8 per MMA: 4 per 128-row block)
+  static constexpr uint32_t SFB_PER_MMA = 8;
   static constexpr uint32_t SF_STRIDE = 16 + 4 * SFB_PER_MMA;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
@@ -339,7 +341,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       mbar_arrive_remote(mapa_shared(bar, 0));
   };
   auto wait_pair = [&](uint32_t bar, uint32_t parity) {
-    return mbar_wait(bar, parity, g.wait_ns, abort_flag);
+    return mbar_wait_warp(bar, parity, g.wait_ns, abort_flag);
   };
   // A role that gives up raises the abort flag of both CTAs of the pair.
   auto raise_abort = [&](uint32_t site, uint32_t role) {
@@ -416,12 +418,17 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             mbar_arrive_expect_tx_warp(sfull_bar(stage), SFA_BYTES + SFB_BYTES);
             tma_load_3d_warp(smem_addr(st + A_BYTES + B_BYTES), &tmSA, 0, kt * 4,
                         mb * CG + static_cast<int>(rank), sfull_bar(stage), pol);
-            // CG 2: this CTA's own weight-row block (tmSB has 1-block boxes);
-            // SwiGLU: the gate block nb (even CTA) or the up block H/128 + nb
-            const int sfb_block = SWIGLU ? nb + (rank ? g.H / 128 : 0)
-                                         : nb * 2 + (CG == 2 ? static_cast<int>(rank) : 0);
-            tma_load_3d_warp(smem_addr(st + A_BYTES + B_BYTES + SFA_BYTES), &tmSB, 0, kt * 4,
-                             sfb_block, sfull_bar(stage), pol);
+            if constexpr (SWIGLU) {
+              // the gate rows' scale block, then the up rows' (1-block boxes)
+              tma_load_3d_warp(smem_addr(st + A_BYTES + B_BYTES + SFA_BYTES), &tmSB, 0, kt * 4, nb,
+                               sfull_bar(stage), pol);
+              tma_load_3d_warp(smem_addr(st + A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES / 2), &tmSB, 0,
+                               kt * 4, g.H / 128 + nb, sfull_bar(stage), pol);
+            } else {
+              // both row blocks of the tile (2-block boxes)
+              tma_load_3d_warp(smem_addr(st + A_BYTES + B_BYTES + SFA_BYTES), &tmSB, 0, kt * 4,
+                               nb * 2, sfull_bar(stage), pol);
+            }
           }
           ++issued;
           if (++stage == STAGES) {
@@ -451,7 +458,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       const WorkItem w = work_item(g, unit, units, num_tiles, num_kt, it);
       bool ok = true;
       for (int kt = w.kt0; kt < w.kt1; ++kt) {
-        if (!mbar_wait(sfull_bar(stage), phase, g.wait_ns, abort_flag)) {
+        if (!mbar_wait_warp(sfull_bar(stage), phase, g.wait_ns, abort_flag)) {
           raise_abort(SITE_MMA_FULL, warp);
           ok = false;
           break;
@@ -468,7 +475,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
           r[4 * kk + 2] = a;
           r[4 * kk + 3] = a;
 #pragma unroll
-          for (int j = 0; j < (CG == 1 ? 2 : 1); ++j) {
+          for (int j = 0; j < 2; ++j) {
             // weight rows 128 j + 32 c + lane of the stage's blocks, c = 0..3
             // -> columns SFB_PER_MMA kk + 4 j + c
             const uint4 b = ld_shared_v4(sfb_s + j * 2048 + kk * 512 + lane * 16);
@@ -480,12 +487,12 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         }
         const uint32_t col = tmem_base + lane_off + SF_COL + SF_STRIDE * stage;
         tmem_st_x32(col, r);
-        if constexpr (CG == 1) tmem_st_x16(col + 32, r + 32);
+        tmem_st_x16(col + 32, r + 32);
         tmem_wait_st();
         tc_fence_before();
         // the MMA warp waits on this barrier alone: arrive only once the
         // stage's codes have landed too
-        if (!mbar_wait(full_bar(stage), phase, g.wait_ns, abort_flag)) {
+        if (!mbar_wait_warp(full_bar(stage), phase, g.wait_ns, abort_flag)) {
           raise_abort(SITE_MMA_FULL, warp);
           ok = false;
           break;
@@ -852,7 +859,7 @@ __global__ void __launch_bounds__(sm::THREADS, 2)
       uint32_t phase = 0;
       int64_t issued = 0;
       for (int kt = 0; kt < num_kt; ++kt) {
-        if (!mbar_wait(empty_bar(stage), phase ^ 1u, g.wait_ns, abort_flag)) {
+        if (!mbar_wait_warp(empty_bar(stage), phase ^ 1u, g.wait_ns, abort_flag)) {
           if (!*abort_flag) record_error(SITE_PRODUCER_EMPTY, warp);
           *abort_flag = 1;
           break;
@@ -889,7 +896,7 @@ __global__ void __launch_bounds__(sm::THREADS, 2)
     int stage = 0;
     uint32_t phase = 0;
     for (int kt = 0; kt < num_kt; ++kt) {
-      if (!mbar_wait(full_bar(stage), phase, g.wait_ns, abort_flag)) {
+      if (!mbar_wait_warp(full_bar(stage), phase, g.wait_ns, abort_flag)) {
         if (!*abort_flag) record_error(SITE_MMA_FULL, warp);
         *abort_flag = 1;
         break;
@@ -929,8 +936,8 @@ __global__ void __launch_bounds__(sm::THREADS, 2)
       uint32_t phase = 0;
       bool ok = true;
       for (int kt = 0; kt < num_kt; ++kt) {
-        if (!mbar_wait(sf_bar(stage), phase, g.wait_ns, abort_flag) ||
-            !mbar_wait(full_bar(stage), phase, g.wait_ns, abort_flag)) {
+        if (!mbar_wait_warp(sf_bar(stage), phase, g.wait_ns, abort_flag) ||
+            !mbar_wait_warp(full_bar(stage), phase, g.wait_ns, abort_flag)) {
           if (!*abort_flag) record_error(SITE_MMA_FULL, 1);
           *abort_flag = 1;
           ok = false;
@@ -966,7 +973,7 @@ __global__ void __launch_bounds__(sm::THREADS, 2)
     // 16-byte stores of one contiguous segment instead of M strided 2-byte
     // stores per thread.
     griddep_wait();   // y may still be read or written by the kernel ahead
-    const bool ok = mbar_wait(acc_full, 0, g.wait_ns, abort_flag);
+    const bool ok = mbar_wait_warp(acc_full, 0, g.wait_ns, abort_flag);
     if (ok) {
       tc_fence_after();
       uint32_t v[NT];

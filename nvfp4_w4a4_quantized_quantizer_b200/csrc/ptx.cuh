@@ -100,6 +100,16 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
   }
 }
 
+// The same wait executed by every lane of a warp, with one decision for the
+// whole warp: true only if every lane saw the phase complete.  Loops that
+// give up on a failed wait and otherwise run warp-collective instructions
+// (elect.sync, shuffles, tcgen05 .sync.aligned forms, named barriers) use
+// this form, so no lane leaves such a loop while others stay in it.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, uint64_t limit_ns,
+                                               const volatile int* abort_flag) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, limit_ns, abort_flag));
+}
+
 // ------------------------------------------- programmatic dependent launch
 // A kernel launched with programmatic stream serialization may start before
 // the kernel ahead of it on the stream has finished.  griddep_wait() returns

@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(QUANT_THREADS) k_quantize(const __grid_constan
   bool ok = true;
   for (; cur.row < a.rows; cur.advance(step_rows, step_cols, per_row), ++i) {
     const int s = static_cast<int>(i % QUANT_SLOTS);
-    if (!mbar_wait(smem_addr(bars + s), static_cast<uint32_t>((i / QUANT_SLOTS) & 1), a.wait_ns,
+    if (!mbar_wait_warp(smem_addr(bars + s), static_cast<uint32_t>((i / QUANT_SLOTS) & 1), a.wait_ns,
                    nullptr)) {
       if (lane == 0) record_error(SITE_QUANT, static_cast<uint32_t>(warp));
       ok = false;

@@ -232,14 +232,22 @@ def fused_linear64_shared_scale(x_codes, x_scales, w_codes, w_scales, segments) 
 
 
 # ------------------------------------------------- MLP pair glue (workload 4)
-def silu_mul_bf16(gate, up) -> np.ndarray:
-    """h = bf16_RNE(fp32(silu(gate) * up)) from float64 gate/up; returns float32 values.
-
-    The MLP pair feeds SiLU(gate) * up, rounded to bf16, into the down
-    projection's activation quantiser.
-    """
-    g = np.asarray(gate, dtype=np.float64)
-    h = (g * sigmoid64(g) * np.asarray(up, dtype=np.float64)).astype(np.float32)
-    u = h.view(np.uint32).astype(np.uint64)
+def _bf16_rne(x32) -> np.ndarray:
+    """float32 values -> nearest bf16 values (ties to even), as float32."""
+    u = np.asarray(x32, dtype=np.float32).view(np.uint32).astype(np.uint64)
     u = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
     return u.astype(np.uint32).view(np.float32)
+
+
+def silu_mul_bf16(gate, up) -> np.ndarray:
+    """h = bf16_RNE(fp32(silu(g) * u)) with g = bf16(fp32(gate)), u = bf16(fp32(up)).
+
+    Reading R8: the gate_up projection is itself a W4A4 linear layer and, like
+    every layer here, emits bf16, so SiLU(gate) * up reads bf16 gate and up
+    values (each the RNE bf16 of the fp32 value); the product is evaluated in
+    float64, rounded to fp32 and then to bf16, which is the down projection's
+    activation input.  Returns float32 values.
+    """
+    g = _bf16_rne(np.asarray(gate, dtype=np.float64).astype(np.float32)).astype(np.float64)
+    u = _bf16_rne(np.asarray(up, dtype=np.float64).astype(np.float32)).astype(np.float64)
+    return _bf16_rne((g * sigmoid64(g) * u).astype(np.float32))

@@ -49,6 +49,12 @@ def test_size_helpers(lib):
     assert lib.nvfp4_quantize_weight_workspace_bytes(6) == 256
 
 
+def test_noalloc_limit_matches_header(lib):
+    text = open(os.path.join(ROOT, "include", "nvfp4.h")).read()
+    m = re.search(r"#define\s+NVFP4_NOALLOC_MAX_SEGMENTS\s+(\d+)", text)
+    assert m and lib.nvfp4_noalloc_max_segments() == int(m.group(1))
+
+
 def test_global_scale_matches_fp32_division(lib):
     import numpy as np
     for amax in (1.0, 123.456, 6.0e4, 3.1e-3):

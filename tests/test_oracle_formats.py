@@ -121,3 +121,23 @@ def test_global_scale_is_fp32_division():
         ulp = float(np.spacing(gs))
         assert abs(float(gs) - exact) <= 0.5 * ulp
     assert oracle.global_scale(2688.0) == np.float32(1.0)
+
+
+def test_global_scale_of_an_all_zero_tensor_is_one():
+    """Reading R3: an all-zero tensor (amax = 0) gets gs = 1, not 0.  Any
+    positive gs encodes zeros the same way; 0 would make the block-scale
+    divisor 6 gs zero and the block reciprocal infinite.  The scale must be a
+    usable one: positive, finite, and the zero tensor must quantise to zero
+    codes and zero scales and dequantise to exact zeros."""
+    gs = oracle.global_scale(0.0)
+    assert gs.dtype == np.float32 and gs == np.float32(1.0)
+    assert oracle.global_scale(np.float32(-0.0)) == np.float32(1.0)
+    x = np.zeros((3, 64), np.float32)
+    with np.errstate(all="raise"):
+        q, s = oracle.quantize(x, gs)
+        xh = oracle.dequantize(q, s, gs)
+    assert not q.any() and not s.any()
+    assert np.array_equal(xh, np.zeros_like(xh))
+    # the smallest positive amax already takes the division branch
+    tiny = np.float32(np.finfo(np.float32).smallest_subnormal)
+    assert oracle.global_scale(tiny) == np.float32(tiny / np.float32(2688.0))

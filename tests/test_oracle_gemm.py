@@ -179,14 +179,16 @@ def test_gates_contract_relative_error(op):
 
 # ------------------------------------------------- MLP glue (SiLU(gate) * up)
 def test_silu_mul_bf16_rounding_matches_ml_dtypes():
-    """The bf16 rounding step against an independent RNE: ml_dtypes' bfloat16
-    cast of the same float32 products (random, ties at every exponent, and
-    values whose low 16 bits are exactly 0x8000)."""
+    """The bf16 rounding steps against an independent RNE: ml_dtypes' bfloat16
+    casts of the float32 gate / up inputs and of the float32 products (random,
+    ties at every exponent, and values whose low 16 bits are exactly 0x8000)."""
     rng = np.random.default_rng(21)
     g = rng.standard_normal(20000) * 4
     u = rng.standard_normal(20000) * 3
     h = oracle.silu_mul_bf16(g, u)
-    prod32 = (g * (1.0 / (1.0 + np.exp(-g))) * u).astype(np.float32)
+    gb = g.astype(np.float32).astype(ml_dtypes.bfloat16).astype(np.float64)
+    ub = u.astype(np.float32).astype(ml_dtypes.bfloat16).astype(np.float64)
+    prod32 = (gb * (1.0 / (1.0 + np.exp(-gb))) * ub).astype(np.float32)
     want = prod32.astype(ml_dtypes.bfloat16).astype(np.float32)
     # the oracle's product is float64 rounded once to float32, as here; allow
     # the rare case where the two float64 evaluations land on different float32s
@@ -194,13 +196,33 @@ def test_silu_mul_bf16_rounding_matches_ml_dtypes():
     assert diff.mean() < 1e-3
     ulp = np.abs(want[diff]) * 2.0 ** -7
     assert np.all(np.abs(h[diff] - want[diff]) <= ulp)
-    # exact ties: float32 values halfway between two bf16 values round to even
-    base = np.array([1.0, 1.5, -3.25, 1000.0], np.float32).view(np.uint32)
-    ties = (base | 0x8000).view(np.float32)
-    # silu(50) = 50 exactly in float64 (sigmoid(50) rounds to 1), and
-    # 50 * (tie / 50) in float64 rounds back to the float32 tie
-    got = oracle.silu_mul_bf16(np.full(4, 50.0), ties.astype(np.float64) / 50.0)
-    np.testing.assert_array_equal(got, ties.astype(ml_dtypes.bfloat16).astype(np.float32))
+    # exact ties: silu(48) = 48 exactly in float64 (sigmoid(48) rounds to 1),
+    # and 48 * (1 + k/128) for odd k (u exact in bf16) has nine significant
+    # bits: a float32 value halfway between two bf16 values, rounded to even
+    k = np.array([1, 3, 5, 7, 9, 17, -1, -33], np.float64)
+    up = 1.0 + k / 128.0
+    prod = (48.0 * up).astype(np.float32)
+    assert np.all((prod.view(np.uint32) & 0xFFFF) == 0x8000)
+    got = oracle.silu_mul_bf16(np.full(len(k), 48.0), up)
+    np.testing.assert_array_equal(got, prod.astype(ml_dtypes.bfloat16).astype(np.float32))
+
+
+def test_silu_mul_bf16_reads_bf16_gate_and_up():
+    """Reading R8: gate and up are the gate_up layer's bf16 outputs, so the
+    oracle rounds them to bf16 before SiLU * up: inputs that round to the same
+    bf16 values give the same h, and h differs from the product of the
+    unrounded values where the rounding of the inputs moves it."""
+    one_plus = np.float64(1.0 + 2.0 ** -10)          # not a bf16 value: rounds to 1
+    assert oracle.silu_mul_bf16(np.array([one_plus]), np.array([1.0]))[0] == \
+        oracle.silu_mul_bf16(np.array([1.0]), np.array([1.0]))[0]
+    rng = np.random.default_rng(5)
+    g = rng.standard_normal(4096) * 3
+    u = rng.standard_normal(4096) * 2
+    gb = g.astype(np.float32).astype(ml_dtypes.bfloat16).astype(np.float64)
+    ub = u.astype(np.float32).astype(ml_dtypes.bfloat16).astype(np.float64)
+    np.testing.assert_array_equal(oracle.silu_mul_bf16(g, u), oracle.silu_mul_bf16(gb, ub))
+    unrounded = (g / (1.0 + np.exp(-g)) * u).astype(np.float32).astype(ml_dtypes.bfloat16)
+    assert np.mean(oracle.silu_mul_bf16(g, u) != unrounded.astype(np.float32)) > 0.05
 
 
 def test_silu_mul_bf16_closed_values_and_limits():

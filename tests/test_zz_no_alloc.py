@@ -62,7 +62,7 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
 
 def test_noalloc_rejects_more_modules_than_its_scratch_holds():
     lib = _lib.load()
-    n = _lib.NOALLOC_MAX_SEGMENTS + 1
+    n = lib.nvfp4_noalloc_max_segments() + 1   # the limit compiled into the library
     N = 16 * n
     w = torch.zeros((N, K), dtype=torch.bfloat16, device="cuda")
     offs_c = (ctypes.c_int64 * n)(*range(0, N, 16))
