@@ -43,6 +43,9 @@ METRIC = "NVFP4 W4A4 linear TFLOPS & % of B200 FP4 peak; small-M weight GB/s"
 FP4_PER_BF16 = 4.0          # nominal dense FP4 / BF16 tensor throughput ratio (9 / 2.25 PFLOP/s)
 ROTATE_ACT = 6              # distinct activation buffers (each step uses the next one)
 ROTATE_W = 4                # distinct weight copies
+# The CTA-pair GEMM gets the caller workspace that lets it run its last
+# partial wave of tiles (and one whole wave) as a stream-K tail.
+SPLIT_TAIL = True
 
 
 # --------------------------------------------------------------- plumbing
@@ -244,7 +247,7 @@ class Layer:
         wc, ws = self.ws[i % len(self.ws)]
         self.nv.nvfp4_fused_linear(self.codes[i % 2], self.scales[i % 2], wc, ws, self.M, self.N,
                                    self.K, self.segs, y=self.ys[i % 2], stream=stream,
-                                   workspace=self.work)
+                                   workspace=self.work if SPLIT_TAIL else None)
 
     @property
     def flops(self):
@@ -312,7 +315,8 @@ class MlpChain:
     def down(self, i, stream):
         _, _, w2c, w2s = self.ws[i % len(self.ws)]
         self.nv.nvfp4_fused_linear(self.hc, self.hsc, w2c, w2s, self.M, self.N2, self.H, self.segs2,
-                                   y=self.ys[i % 2], stream=stream, workspace=self.work)
+                                   y=self.ys[i % 2], stream=stream,
+                                   workspace=self.work if SPLIT_TAIL else None)
 
     def gemm(self, i, stream):
         """Everything after the first quantisation."""

@@ -228,31 +228,33 @@ nvfp4_status nvfp4_fused_linear(const void* a_codes, const void* a_scales,
                                 void* y, int64_t ldy, nvfp4_out_dtype out_dtype,
                                 nvfp4_stream_t stream);
 
-/* Workspace of nvfp4_fused_linear_ws: NVFP4_GEMM_WS_COUNTER_BYTES of
- * arrival counters followed by one 256 KB fp32 partial tile per K-part. */
+/* Workspace of nvfp4_fused_linear_ws: NVFP4_GEMM_WS_COUNTER_BYTES of flags
+ * followed by 256 KB fp32 partial tiles, one per CTA pair of the launch. */
 #define NVFP4_GEMM_WS_COUNTER_BYTES 4096
 #define NVFP4_GEMM_WS_MAX_UNITS 128
 
-/* Bytes of a workspace that never limits the split of
+/* Bytes of a workspace large enough for any launch of
  * nvfp4_fused_linear_ws (NVFP4_GEMM_WS_COUNTER_BYTES + 128 partial tiles,
- * about 32 MB).  Any device. */
+ * about 32 MB; a B200 runs 74 CTA pairs).  Any device. */
 size_t nvfp4_gemm_workspace_bytes(void);
 
 /* nvfp4_fused_linear with a caller-owned device workspace that lets the
- * CTA-pair kernel balance its last, partial wave of tiles: each tile of that
- * wave is computed as up to 4 K-parts by pairs that would otherwise idle;
- * each part writes an fp32 partial tile to the workspace and the last part
- * to arrive sums the parts in part order (the same order whichever arrives
- * last, so results do not depend on timing) and applies the epilogue.  The
- * sum differs from the unsplit kernel's by fp32 rounding only.
+ * CTA-pair kernel balance its last, partial wave of tiles (a stream-K
+ * tail): when the 256 x 256 tiles are not a multiple of the pairs, the last
+ * (pairs + remainder) tiles are cut into equal ranges of k-tiles, one per
+ * pair, after the pairs' whole tiles.  A tile shared by two pairs is
+ * finished by the pair that runs its first k-tiles: the other pair
+ * publishes its fp32 partial tile in the workspace, and the sum is always
+ * formed as (first k-tiles) + (last k-tiles), so results do not depend on
+ * timing.  They differ from nvfp4_fused_linear's by fp32 rounding only.
  * workspace: 16-byte aligned; its first NVFP4_GEMM_WS_COUNTER_BYTES must be
- * zero before its first use (every call leaves them zero, also after a
- * bounded wait ran out); it must not be in use by another call that may run
- * at the same time.  workspace_bytes below nvfp4_gemm_workspace_bytes()
- * limits the number of parts; NULL (or too small for two parts) runs the
- * last wave as whole tiles, exactly like nvfp4_fused_linear.  Other
- * arguments, layouts and errors as for nvfp4_fused_linear; an unaligned
- * workspace returns NVFP4_ERR_ALIGNMENT. */
+ * zero before its first use (every call that completes without an error
+ * leaves them zero; after a bounded wait ran out, clear them again); it
+ * must not be in use by another call that may run at the same time.
+ * workspace_bytes below NVFP4_GEMM_WS_COUNTER_BYTES + (pairs) x 256 KB, or
+ * a NULL workspace, runs every tile whole, exactly like
+ * nvfp4_fused_linear.  Other arguments, layouts and errors as for
+ * nvfp4_fused_linear; an unaligned workspace returns NVFP4_ERR_ALIGNMENT. */
 nvfp4_status nvfp4_fused_linear_ws(const void* a_codes, const void* a_scales,
                                    const void* w_codes, const void* w_scales,
                                    int64_t M, int64_t N, int64_t K,

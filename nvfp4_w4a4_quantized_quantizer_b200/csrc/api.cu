@@ -231,9 +231,9 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 constexpr int64_t kMaxDim = (1ll << 31) - 1;
 
-// One K-part's fp32 partial tile: 2 CTAs x 128 rows x 256 columns.
+// One stream-K partial tile (a workspace slot): 2 CTAs x 128 rows x 256
+// columns of fp32.
 constexpr size_t kPartialBytes = 2ull * nvfp4::tc::BM * nvfp4::tc::BN * 4;
-constexpr int64_t kMaxSplit = 4;
 
 nvfp4_status check_bf16_matrix(const void* x, int64_t R, int64_t K, int64_t ld) {
   if (x == nullptr) return NVFP4_ERR_INVALID_ARG;
@@ -607,6 +607,7 @@ nvfp4_status nvfp4_fused_linear_ws(const void* a_codes, const void* a_scales, co
   nvfp4::GemmArgs g;
   g.sfa = static_cast<const uint8_t*>(a_scales);
   g.sfb = static_cast<const uint8_t*>(w_scales);
+  g.wq = static_cast<const uint8_t*>(w_codes);
   g.M = static_cast<int>(M);
   g.N = static_cast<int>(N);
   g.K = static_cast<int>(K);
@@ -616,11 +617,9 @@ nvfp4_status nvfp4_fused_linear_ws(const void* a_codes, const void* a_scales, co
   g.sector_stores = ((reinterpret_cast<uintptr_t>(y) & 31u) == 0) &&
                     ((ldy * (g.out_fp32 ? 4 : 2)) % 32 == 0);
   g.wait_ns = g_wait_ns;
-  g.full_tiles = 0;
-  g.split = 1;
-  g.split_units = 0;
+  g.sk_tiles = 0;
   g.partial = nullptr;
-  g.counters = nullptr;
+  g.flags = nullptr;
   // Tile raster.  Consecutive CTAs (pairs) run tiles that share one operand
   // tile, and the rest of that operand is re-read from L2 for each of the
   // other operand's tiles.  By default they share weight tiles (M fastest),
@@ -683,26 +682,19 @@ nvfp4_status nvfp4_fused_linear_ws(const void* a_codes, const void* a_scales, co
   const int64_t tiles = ((M + 2 * nvfp4::tc::BM - 1) / (2 * nvfp4::tc::BM)) * num_n;
   const int pairs = static_cast<int>(tiles < info->pairs ? tiles : info->pairs);
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  // Last partial wave: when the tiles are not a multiple of the pairs, each
-  // tile of the last wave is split into S K-parts run by otherwise idle
-  // pairs (S = pairs / leftover tiles, at most 4, at most the k-tiles and
-  // within the workspace); the parts meet in the caller's workspace.
-  if (workspace != nullptr && tiles > pairs) {
-    const int64_t num_kt = (K + nvfp4::tc::BK - 1) / nvfp4::tc::BK;
-    const int64_t left = tiles % pairs;
-    const int64_t max_units =
+  // Stream-K tail: when the tiles are not a multiple of the pairs, the last
+  // partial wave and one whole wave before it (sk_tiles = pairs + the
+  // remainder) are cut into equal k-tile ranges, one per pair, instead of
+  // leaving most pairs idle during the last wave.  Needs one workspace slot
+  // per pair (the partial tile a pair publishes) and its flags.
+  if (workspace != nullptr && tiles > pairs && tiles % pairs != 0) {
+    const int64_t slots =
         workspace_bytes > NVFP4_GEMM_WS_COUNTER_BYTES
             ? static_cast<int64_t>((workspace_bytes - NVFP4_GEMM_WS_COUNTER_BYTES) / kPartialBytes)
             : 0;
-    int64_t S = left > 0 ? pairs / left : 0;
-    if (S > kMaxSplit) S = kMaxSplit;
-    if (S > num_kt) S = num_kt;
-    while (S >= 2 && left * S > max_units) --S;
-    if (S >= 2 && left * 2 * 4 <= NVFP4_GEMM_WS_COUNTER_BYTES) {
-      g.full_tiles = static_cast<int>(tiles - left);
-      g.split = static_cast<int>(S);
-      g.split_units = static_cast<int>(left * S);
-      g.counters = static_cast<unsigned*>(workspace);
+    if (slots >= pairs && static_cast<int64_t>(pairs) * 2 * 4 <= NVFP4_GEMM_WS_COUNTER_BYTES) {
+      g.sk_tiles = static_cast<int>(pairs + tiles % pairs);
+      g.flags = static_cast<unsigned*>(workspace);
       g.partial = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                            NVFP4_GEMM_WS_COUNTER_BYTES);
     }

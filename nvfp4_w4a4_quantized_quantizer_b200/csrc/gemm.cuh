@@ -53,6 +53,7 @@ struct SegTable {
 struct GemmArgs {
   const uint8_t* sfa;  // activation (or, swapped, token) scale atoms
   const uint8_t* sfb;  // weight scale atoms
+  const uint8_t* wq;   // weight codes [N, K/2] (the small-M kernel's L2 prefetch)
   int M, N, K;
   void* y;
   int64_t ldy;
@@ -60,18 +61,24 @@ struct GemmArgs {
   int sector_stores;   // y base 32-byte aligned and rows a multiple of 32 bytes
   int n_fastest;       // tile raster: 0 = M fastest (consecutive CTAs share a weight tile),
                        // 1 = N fastest (they share an activation tile)
-  // Last-wave K split (CTA-pair kernel): tiles [full_tiles, num_tiles) are each
-  // computed as `split` K-parts by split_units = (num_tiles - full_tiles) * split
-  // units; unit u (u < split_units) takes part u % split of tile
-  // full_tiles + u / split after its whole tiles.  split <= 1: no split.
-  // The parts meet in a caller-owned workspace: one arrival counter per
-  // (split tile, CTA of the pair), all zero between launches (the last part
-  // wraps its counter back to 0), and one fp32 partial tile per unit.
-  int full_tiles;
-  int split;
-  int split_units;
-  float* partial;      // [split_units][2 CTAs][2 halves][32 chunks][128 rows] float4
-  unsigned* counters;  // [num_tiles - full_tiles][2 CTAs]
+  // Stream-K tail (CTA-pair kernel).  With sk_tiles > 0 the last sk_tiles
+  // tiles [num_tiles - sk_tiles, num_tiles) are not run whole: their
+  // sk_tiles * num_kt k-tiles are cut into `units` contiguous ranges of
+  // (nearly) equal length, range u = [sk_len * u / units, sk_len * (u + 1) /
+  // units), one per CTA pair, after the pair's whole tiles (dp_tiles =
+  // num_tiles - sk_tiles, a multiple of the pair count, walked u, u + units,
+  // ...).  sk_tiles >= units, so a range is at least one tile long and a tile
+  // is shared by at most two pairs: the pair whose range starts inside it
+  // runs its tail k-tiles first and publishes that fp32 partial tile in
+  // slot u of the caller's workspace (then raises the slot's flag); the pair
+  // whose range ends inside it runs its head k-tiles last, waits for the
+  // flag of slot u + 1, adds the partial to its own accumulator (head +
+  // tail, the same order whatever the timing) and applies the epilogue.
+  // The consumer sets the flag back to zero, so the flags are zero between
+  // launches.  sk_tiles == 0: every tile whole.
+  int sk_tiles;
+  float* partial;      // [slot][2 CTAs][2 column halves][32 chunks][128 rows] float4
+  unsigned* flags;     // [slot][2 CTAs]
   uint64_t wait_ns;
   // SwiGLU epilogue (k_gemm_tc<2, true>): the weight is [gate; up], H rows
   // each; tile column nb covers h columns [128 nb, 128 nb + 128) -- the even
@@ -160,40 +167,80 @@ __device__ __forceinline__ int seg_advance(const SegTable& t, int seg, int n) {
 // Tiles are walked M fastest (consecutive CTAs share a weight tile and the
 // activations stay in L2) or, when GemmArgs::n_fastest is set, N fastest
 // (they share an activation tile: for activations too large for the L2).
-// One unit of work of a CTA (pair): a whole tile (part < 0) or one K-part of
-// a tile of the last partial wave.
+// One item of work of a CTA (pair): k-tiles [kt0, kt1) of one tile, run
+// whole (ITEM_WHOLE), as the tail of a stream-K tile whose partial sum is
+// published (ITEM_TAIL), or as its head, summed with that partial
+// (ITEM_HEAD).  A pair's items: its whole data-parallel tiles, then its
+// stream-K range (a tail, whole tiles, a head; each part optional).
+enum ItemKind : int { ITEM_WHOLE = 0, ITEM_TAIL = 1, ITEM_HEAD = 2 };
+
 struct WorkItem {
   int tile;
   int kt0, kt1;   // k-tiles [kt0, kt1)
-  int part;
+  int kind;
 };
 
-__device__ __forceinline__ int work_full(const GemmArgs& g, int num_tiles) {
-  return g.split > 1 ? g.full_tiles : num_tiles;
+struct WorkPlan {
+  int n_dp;        // whole data-parallel tiles: unit, unit + units, ...
+  int sk_base;     // first tile of the stream-K range (absolute index)
+  int tail_kt0;    // > 0: the range starts with the tail [tail_kt0, num_kt) of tile sk_base
+  int n_whole;     // whole tiles of the range after the tail
+  int head_kt1;    // > 0: the range ends with the head [0, head_kt1) of the next tile
+  int n_items;
+};
+
+__device__ __forceinline__ WorkPlan work_plan(const GemmArgs& g, int unit, int units,
+                                              int num_tiles, int num_kt) {
+  WorkPlan p;
+  if (g.sk_tiles <= 0) {
+    p.n_dp = unit < num_tiles ? (num_tiles - 1 - unit) / units + 1 : 0;
+    p.sk_base = 0;
+    p.tail_kt0 = p.n_whole = p.head_kt1 = 0;
+    p.n_items = p.n_dp;
+    return p;
+  }
+  const int dp_tiles = num_tiles - g.sk_tiles;            // a multiple of units
+  p.n_dp = dp_tiles / units;
+  const int64_t len = static_cast<int64_t>(g.sk_tiles) * num_kt;
+  const int s0 = static_cast<int>(len * unit / units);
+  const int s1 = static_cast<int>(len * (unit + 1) / units);
+  const int a = s0 / num_kt;                               // tile (within the range) of s0
+  p.tail_kt0 = s0 - a * num_kt;
+  const int first_whole = p.tail_kt0 ? a + 1 : a;
+  const int b = s1 / num_kt;                               // tile of the range's end
+  p.head_kt1 = s1 - b * num_kt;
+  p.n_whole = b - first_whole;
+  p.sk_base = dp_tiles + a;
+  p.n_items = p.n_dp + (p.tail_kt0 ? 1 : 0) + p.n_whole + (p.head_kt1 ? 1 : 0);
+  return p;
 }
 
-__device__ __forceinline__ int work_count(const GemmArgs& g, int unit, int units, int num_tiles) {
-  const int full = work_full(g, num_tiles);
-  int n = unit < full ? (full - 1 - unit) / units + 1 : 0;
-  if (g.split > 1 && unit < g.split_units) ++n;
-  return n;
-}
-
-__device__ __forceinline__ WorkItem work_item(const GemmArgs& g, int unit, int units,
-                                              int num_tiles, int num_kt, int i) {
-  const int full = work_full(g, num_tiles);
-  const int nfull = unit < full ? (full - 1 - unit) / units + 1 : 0;
+__device__ __forceinline__ WorkItem work_item(const WorkPlan& p, int unit, int units, int num_kt,
+                                              int i) {
   WorkItem w;
-  if (i < nfull) {
+  w.kt0 = 0;
+  w.kt1 = num_kt;
+  w.kind = ITEM_WHOLE;
+  if (i < p.n_dp) {
     w.tile = unit + i * units;
-    w.kt0 = 0;
-    w.kt1 = num_kt;
-    w.part = -1;
-  } else {
-    w.tile = full + unit / g.split;
-    w.part = unit % g.split;
-    w.kt0 = w.part * num_kt / g.split;
-    w.kt1 = (w.part + 1) * num_kt / g.split;
+    return w;
+  }
+  int j = i - p.n_dp;
+  int t = p.sk_base;
+  if (p.tail_kt0) {
+    if (j == 0) {
+      w.tile = t;
+      w.kt0 = p.tail_kt0;
+      w.kind = ITEM_TAIL;
+      return w;
+    }
+    --j;
+    ++t;
+  }
+  w.tile = t + j;
+  if (j >= p.n_whole) {
+    w.kt1 = p.head_kt1;
+    w.kind = ITEM_HEAD;
   }
   return w;
 }
@@ -322,7 +369,8 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
   const int num_n = SWIGLU ? g.H / 128 : (g.N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
   const int num_kt = (g.K + BK - 1) / BK;
-  const int n_items = work_count(g, unit, units, num_tiles);
+  const WorkPlan plan = work_plan(g, unit, units, num_tiles, num_kt);
+  const int n_items = plan.n_items;
 
   auto full_bar = [&](int s) { return smem_addr(bars + s); };
   auto empty_bar = [&](int s) { return smem_addr(bars + STAGES + s); };
@@ -392,7 +440,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       int64_t issued = 0;
       bool ok = true;
       for (int it = 0; it < n_items && ok; ++it) {
-        const WorkItem w = work_item(g, unit, units, num_tiles, num_kt, it);
+        const WorkItem w = work_item(plan, unit, units, num_kt, it);
         const int tile = w.tile;
         const int mb = g.n_fastest ? tile / num_n : tile % num_m;
         const int nb = g.n_fastest ? tile % num_n : tile / num_m;
@@ -455,7 +503,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     int stage = 0;
     uint32_t phase = 0;
     for (int it = 0; it < n_items; ++it) {
-      const WorkItem w = work_item(g, unit, units, num_tiles, num_kt, it);
+      const WorkItem w = work_item(plan, unit, units, num_kt, it);
       bool ok = true;
       for (int kt = w.kt0; kt < w.kt1; ++kt) {
         if (!mbar_wait_warp(sfull_bar(stage), phase, g.wait_ns, abort_flag)) {
@@ -525,7 +573,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       int local = 0;
       bool ok = true;
       for (int it = 0; it < n_items && ok; ++it, ++local) {
-        const WorkItem w = work_item(g, unit, units, num_tiles, num_kt, it);
+        const WorkItem w = work_item(plan, unit, units, num_kt, it);
         if (!wait_pair(tmem_empty, static_cast<uint32_t>((local & 1) ^ 1))) {
           raise_abort(SITE_MMA_TMEM_EMPTY, 1);
           break;
@@ -624,29 +672,73 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         }
       }
     };
-    // K-parts: chunk c (columns 4c..4c+3 of this thread's 128) of unit u's
-    // partial tile; for one chunk a warp's 32 rows are 512 contiguous bytes
+    // Stream-K partial tiles: chunk c (columns 4c..4c+3 of this thread's
+    // 128) of slot u; for one chunk a warp's 32 rows are 512 contiguous bytes
     auto part_chunk = [&](int u, int c) {
       return reinterpret_cast<float4*>(g.partial) +
              ((((static_cast<size_t>(u) * 2 + rank) * 2 + half) * 32 + c) * BM + row_in_tile);
     };
-    volatile int* last_flag = abort_flag + 1;
     int local = 0;
     bool dead = false;   // a wait ran out: skip the work, keep every barrier
     for (int it = 0; it < n_items; ++it, ++local) {
-      const WorkItem wi = work_item(g, unit, units, num_tiles, num_kt, it);
+      const WorkItem wi = work_item(plan, unit, units, num_kt, it);
       const int mb = g.n_fastest ? wi.tile / num_n : wi.tile % num_m;
       const int nb = g.n_fastest ? wi.tile % num_n : wi.tile / num_m;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ACC_COL + half * 128;
       bool ok = !dead;
+      // The head k-tiles of a stream-K tile (always the pair's last item):
+      // the tail partial was published by the next pair as the first item of
+      // its range.  Wait for its flag and start loading it while this pair's
+      // own k-tiles finish; once the accumulator is complete, add the
+      // partial to it in TMEM (head + tail), 16 columns at a time with two
+      // column groups of it in registers, then run the whole-tile epilogue.
+      const bool head = !SWIGLU && wi.kind == ITEM_HEAD;
+      const unsigned* flag = g.flags + (unit + 1) * 2 + rank;
+      float4 pr[2][4];
+      if (head) {
+        if (ok && !flag_wait_warp(flag, g.wait_ns, abort_flag)) {
+          raise_abort(SITE_SK_FLAG, warp);
+          dead = true;
+          ok = false;
+        }
+        if (ok) {
+#pragma unroll
+          for (int gg = 0; gg < 2; ++gg)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) pr[gg][c] = __ldcg(part_chunk(unit + 1, gg * 4 + c));
+        }
+      }
       if (ok && !wait_pair(tmem_full, static_cast<uint32_t>(local & 1))) {
         raise_abort(SITE_EPI_TMEM_FULL, warp);
         dead = true;
         ok = false;
       }
       uint32_t v[128];
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ACC_COL + half * 128;
       if (ok) {
         tc_fence_after();
+        if (head) {
+#pragma unroll
+          for (int grp = 0; grp < 8; ++grp) {
+            uint32_t t[16];
+            tmem_ld_x16(taddr + grp * 16, t);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const float4 x = pr[grp & 1][c];
+              t[4 * c + 0] = __float_as_uint(__uint_as_float(t[4 * c + 0]) + x.x);
+              t[4 * c + 1] = __float_as_uint(__uint_as_float(t[4 * c + 1]) + x.y);
+              t[4 * c + 2] = __float_as_uint(__uint_as_float(t[4 * c + 2]) + x.z);
+              t[4 * c + 3] = __float_as_uint(__uint_as_float(t[4 * c + 3]) + x.w);
+            }
+            if (grp < 6) {
+#pragma unroll
+              for (int c = 0; c < 4; ++c)
+                pr[grp & 1][c] = __ldcg(part_chunk(unit + 1, (grp + 2) * 4 + c));
+            }
+            tmem_st_x16(taddr + grp * 16, t);
+          }
+          tmem_wait_st();
+        }
         if constexpr (SWIGLU) {
           // this warp's 64 h columns: gate accumulator columns [64 half, +64)
           // into v[0..63], the matching up columns [128 + 64 half, +64) into v[64..127]
@@ -661,32 +753,35 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
           for (int c = 0; c < 4; ++c) tmem_ld_x32(taddr + c * 32, v + c * 32);
         }
         tmem_wait_ld();
-        // A K-part is always a CTA's last item: no MMA waits for its
-        // accumulator, which stays in TMEM for the sum below.
-        if (wi.part < 0) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) arrive_leader(tmem_empty);
-        }
+        // the accumulator is in registers: the MMA warp may start the next item
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) arrive_leader(tmem_empty);
       }
       if constexpr (SWIGLU) {
-        // whole tiles only (the host never splits this launch); rows past M
-        // inside the last 128-row block still write their (zero) scale
-        // bytes: the scale buffer's padding rows must hold zeros
+        // whole tiles only (the host never gives this launch a stream-K
+        // range); rows past M inside the last 128-row block still write
+        // their (zero) scale bytes: the scale buffer's padding rows must
+        // hold zeros
         const int64_t gm = static_cast<int64_t>(mb * CG + static_cast<int>(rank)) * BM + row_in_tile;
         const int64_t rows_padded = (static_cast<int64_t>(g.M) + 127) / 128 * 128;
         if (ok && gm < rows_padded) swiglu_store_row(g, gm, nb * 128 + half * 64, v);
         continue;
-      } else if (wi.part < 0) {
+      } else if (wi.kind != ITEM_TAIL) {
         if (ok)
           store_row(mb, nb, [&](int grp, uint32_t (&a)[16]) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) a[i] = v[grp * 16 + i];
           });
+        if (head) {
+          // every epilogue warp has read the partial: the flag returns to zero
+          asm volatile("bar.sync 1, 256;" ::: "memory");
+          if (ok && warp == EPI_WARP0 && lane == 0) st_relaxed_gpu_u32(const_cast<unsigned*>(flag), 0u);
+        }
         continue;
       }
-      // one K-part of a last-wave tile: publish it; the CTA that publishes
-      // the tile's last part sums all parts in part order and stores
+      // the tail k-tiles of a stream-K tile (the first item of the pair's
+      // range): publish the partial in slot `unit`, then raise its flag
       if (ok) {
 #pragma unroll
         for (int c = 0; c < 32; ++c)
@@ -695,46 +790,9 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                              __uint_as_float(v[4 * c + 2]), __uint_as_float(v[4 * c + 3])));
         __threadfence();
       }
-      // Every epilogue warp passes both barriers once per part and every part
-      // counts itself, whatever its waits returned, so that each counter
-      // wraps back to zero (atomicInc with limit split - 1) in every launch.
       asm volatile("bar.sync 1, 256;" ::: "memory");
-      if (warp == EPI_WARP0 && lane == 0) {
-        const unsigned idx = static_cast<unsigned>((wi.tile - g.full_tiles) * 2) + rank;
-        const unsigned lim = static_cast<unsigned>(g.split - 1);
-        *last_flag = atomicInc(g.counters + idx, lim) == lim;
-      }
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      if (ok && *last_flag && !*abort_flag) {
-        __threadfence();
-        // sum the parts in part order, whichever CTA is last, 16 columns at
-        // a time: this CTA's own part is re-read from TMEM (a K-part is a
-        // CTA's last item, so its accumulator was not released), the others
-        // come from the workspace
-        const int u0 = (wi.tile - g.full_tiles) * g.split;
-        const int mine = wi.part;
-        store_row(mb, nb, [&](int grp, uint32_t (&a)[16]) {
-          for (int p = 0; p < g.split; ++p) {
-            uint32_t t[16];
-            if (p == mine) {
-              tmem_ld_x16(taddr + grp * 16, t);
-              tmem_wait_ld();
-            } else {
-#pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                const float4 x = __ldcg(part_chunk(u0 + p, grp * 4 + c));
-                t[4 * c] = __float_as_uint(x.x);
-                t[4 * c + 1] = __float_as_uint(x.y);
-                t[4 * c + 2] = __float_as_uint(x.z);
-                t[4 * c + 3] = __float_as_uint(x.w);
-              }
-            }
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              a[i] = p == 0 ? t[i] : __float_as_uint(__uint_as_float(a[i]) + __uint_as_float(t[i]));
-          }
-        });
-      }
+      if (ok && !*abort_flag && warp == EPI_WARP0 && lane == 0)
+        red_release_gpu_add_u32(g.flags + unit * 2 + rank, 1u);
     }
   }
 
@@ -774,6 +832,7 @@ constexpr uint32_t ACC_COL = 0;         // NT columns
 constexpr uint32_t SF_COL = 64;         // + 32 * stage
 constexpr uint32_t SF_STRIDE = 32;
 constexpr int BAR_BYTES = 256;
+constexpr int64_t L2_PREFETCH_CHUNK = 32768;   // bytes per L2 bulk prefetch
 // Two CTAs fit on one SM (shared memory, 256 TMEM columns and <= 80
 // registers per thread each), so that with launch overlap the next call's
 // CTAs start streaming their weights beside this call's.
@@ -852,6 +911,19 @@ __global__ void __launch_bounds__(sm::THREADS, 2)
     // warp-wide loop; one elected lane issues each copy
     {
       const bool is_w = (warp == 0);
+      if (is_w && lane == 0) {
+        // Ask L2 for this CTA's whole weight block (its 128 code rows are
+        // contiguous, K/2 bytes each, and its scale atoms too) before the
+        // kernel ahead has finished: with launch overlap the weight stream
+        // of this call then keeps HBM busy while the call ahead drains, and
+        // the ring below reads most of it from L2.
+        const int rows = min(BW, g.N - wt * BW);
+        const uint8_t* wb = g.wq + static_cast<int64_t>(wt) * BW * (g.K / 2);
+        const int64_t wbytes = static_cast<int64_t>(rows) * (g.K / 2);
+        for (int64_t o = 0; o < wbytes; o += L2_PREFETCH_CHUNK)
+          bulk_prefetch_l2(wb + o, static_cast<uint32_t>(wbytes - o < L2_PREFETCH_CHUNK ? wbytes - o : L2_PREFETCH_CHUNK));
+        bulk_prefetch_l2(g.sfb + wt * kb4 * 512, static_cast<uint32_t>(kb4 * 512));
+      }
       if (!is_w) griddep_wait();   // the token operands may come from the kernel ahead
       // weights stream through once; tokens are re-read by every CTA
       const uint64_t pol = is_w ? policy_evict_first() : policy_evict_last();

@@ -30,6 +30,7 @@ enum ErrorSite : uint32_t {
   SITE_EPI_TMEM_FULL = 4,
   SITE_DRAIN = 5,
   SITE_QUANT = 6,
+  SITE_SK_FLAG = 7,
   SITE_TEST = 15,
 };
 
@@ -110,6 +111,43 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, ui
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, limit_ns, abort_flag));
 }
 
+// ------------------------------------------------ flags in global memory
+__device__ __forceinline__ uint32_t ld_acquire_gpu_u32(const unsigned* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_gpu_add_u32(unsigned* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void st_relaxed_gpu_u32(unsigned* p, uint32_t v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// The whole warp waits until the flag at `p` (written by another CTA with
+// release semantics) is non-zero, reading it with acquire semantics; false
+// when `limit_ns` elapses first or another role raised `abort`.  One
+// decision for the whole warp, like mbar_wait_warp.
+__device__ __forceinline__ bool flag_wait_warp(const unsigned* p, uint64_t limit_ns,
+                                               const volatile int* abort_flag) {
+  bool ok = ld_acquire_gpu_u32(p) != 0u;
+  if (!ok) {
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+      __nanosleep(32);
+      if (ld_acquire_gpu_u32(p) != 0u) {
+        ok = true;
+        break;
+      }
+      if (abort_flag != nullptr && *abort_flag) break;
+      if (globaltimer_ns() - t0 > limit_ns) break;
+    }
+  }
+  return __all_sync(0xffffffffu, ok);
+}
+
 // ------------------------------------------- programmatic dependent launch
 // A kernel launched with programmatic stream serialization may start before
 // the kernel ahead of it on the stream has finished.  griddep_wait() returns
@@ -170,6 +208,12 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
       "l"(src), "r"(bytes), "r"(bar), "l"(policy)
       : "memory");
+}
+
+// Ask L2 to fetch [src, src + bytes) (16-byte aligned, a multiple of 16
+// bytes); no completion is tracked.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 // Warp-wide forms of the copy issue: every lane executes them with the

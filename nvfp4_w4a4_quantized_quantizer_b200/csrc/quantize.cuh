@@ -161,8 +161,14 @@ struct UnitCursor {
 
 __global__ void __launch_bounds__(QUANT_THREADS) k_quantize(const __grid_constant__ QuantArgs a) {
   extern __shared__ __align__(128) uint8_t qsmem[];
+  // The reciprocal table in shared memory: the lanes of a warp look up
+  // different scale codes, which a constant-bank (parameter) load would
+  // serve one distinct address at a time.
+  __shared__ float s_rtab[128];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  for (int t = threadIdx.x; t < 128; t += QUANT_THREADS) s_rtab[t] = a.rtab[t];
+  __syncthreads();
   uint8_t* ring = qsmem + warp * (QUANT_SLOTS * QUANT_UNIT * 2);
   uint64_t* bars = reinterpret_cast<uint64_t*>(qsmem + QUANT_SMEM) + warp * QUANT_SLOTS;
   const int K = static_cast<int>(a.K);
@@ -239,7 +245,7 @@ __global__ void __launch_bounds__(QUANT_THREADS) k_quantize(const __grid_constan
       w[4] = hi.x; w[5] = hi.y; w[6] = hi.z; w[7] = hi.w;
       const float amax = bf16x16_absmax(w);
       const uint32_t sc = cvt_e4m3(__fdiv_rn(amax, c));
-      const float rr = a.rtab[sc];
+      const float rr = s_rtab[sc];
       uint64_t rr2;
       asm("mov.b64 %0, {%1, %1};" : "=l"(rr2) : "f"(rr));
       float f[8];

@@ -76,7 +76,8 @@ def _gpu_layer(wl, xbits, wbits, calib_bits):
                             gate.get("dt") if s.op == "gdn_decay" else None)
              for i, (s, o) in enumerate(zip(wl.segments, wl.seg_offsets))]
     M = xbits.shape[0]
-    # with the workspace, as bench.py calls it (the last wave split along K)
+    # with the workspace, as bench.py calls it (a stream-K tail when the
+    # tiles do not fill the last wave)
     work = nv.nvfp4_gemm_workspace("cuda")
     y32 = nv.nvfp4_fused_linear(ac, as_, wc, ws, M, wl.N, wl.K, specs, out_dtype=nv.OUT_FP32,
                                 workspace=work)
@@ -86,7 +87,8 @@ def _gpu_layer(wl, xbits, wbits, calib_bits):
     assert int(work[:4096].count_nonzero()) == 0
     if M == 4096:
         # the prefill GEMM's 320 tiles leave a partial last wave on 74 pairs,
-        # which the workspace call splits: its fp32 sums associate differently
+        # so the workspace call shares tiles between pairs: their fp32 sums
+        # associate differently
         plain = nv.nvfp4_fused_linear(ac, as_, wc, ws, M, wl.N, wl.K, specs, out_dtype=nv.OUT_FP32)
         assert not torch.equal(plain, y32)
         del plain

@@ -271,10 +271,12 @@ def test_overlap_keeps_stream_order_of_shared_buffers(overlap):
     assert nv.nvfp4_last_device_error()[0] == 0
 
 
-# ------------------------------------------------- last-wave K split (workspace)
+# ----------------------------------------------- stream-K tail (workspace)
 # Shapes with more 256 x 256 tiles than a B200's 74 CTA pairs and a partial
-# last wave: 180 tiles (32 left, 2 parts of 1 k-tile), 320 tiles (24 left,
-# 3 parts of 1-2 k-tiles), ragged M and N inside the split tiles.
+# last wave, so the last 74 + remainder tiles run as equal k-tile ranges per
+# pair: 180 tiles with K = 512 (106 tiles of 2 k-tiles in ranges of 2-3
+# k-tiles: heads and tails of one k-tile), 320 tiles with K = 1280 (98 tiles
+# of 5 k-tiles, ranges of 6-7), ragged M and N inside the shared tiles.
 @pytest.mark.parametrize("path,M,N,K", [
     (PAIR, 2304, 5120, 512), (PAIR, 4096, 5120, 1280), (PAIR, 2200, 5104, 512),
     (PAIR_NFAST, 2304, 5120, 512), (AUTO, 4096, 5120, 1280)])
@@ -296,10 +298,10 @@ def test_split_last_wave(path, M, N, K):
     yb = nv.nvfp4_fused_linear(A[0], A[1], W[0], W[1], M, N, K, seg, workspace=work)
     st, info = nv.nvfp4_last_device_error()
     assert st == 0, f"device error word {info:#x}"
-    # every call leaves the arrival counters at zero
+    # every call leaves the flags at zero
     assert int(work[:4096].count_nonzero()) == 0
     y32, y32b = y32.cpu().numpy(), y32b.cpu().numpy()
-    # the parts are summed in a fixed order: no run-to-run variation
+    # head + tail is summed in a fixed order: no run-to-run variation
     np.testing.assert_array_equal(y32, y32b)
     ref = oracle.linear64(oracle.dequantize(ac, as_, a_gs), oracle.dequantize(wc, ws, w_gs))
     H.check_gemm_fp32(y32, ref, f"split {M}x{N}x{K}")
@@ -307,8 +309,8 @@ def test_split_last_wave(path, M, N, K):
 
 
 def test_split_with_gates_and_small_workspace():
-    """GDN gate segments inside split tiles; a workspace too small for two
-    parts per leftover tile gives exactly the unsplit result."""
+    """GDN gate segments inside tiles shared by two pairs; a workspace too
+    small for one partial tile per pair gives exactly the plain result."""
     M, N, K = 2304, 5120, 512
     rng = np.random.default_rng(5)
     ac = rng.integers(0, 16, size=(M, K)).astype(np.uint8)
