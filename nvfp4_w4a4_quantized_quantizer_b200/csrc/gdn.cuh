@@ -32,8 +32,9 @@ namespace gdn {
 constexpr int C = 64;          // tokens per chunk
 constexpr int D = 128;         // key and value head width
 constexpr int LD = D + 1;      // padded rows of S, K, Q: a warp reading a column is bank-conflict free
+constexpr int CP = C + 1;      // padded rows of A
 constexpr int THREADS = 256;
-constexpr int SMEM_FLOATS = D * LD + 2 * C * LD + C * D + C * C + 4 * C;
+constexpr int SMEM_FLOATS = D * LD + 2 * C * LD + C * D + C * CP + 4 * C;
 constexpr int SMEM_BYTES = SMEM_FLOATS * 4;
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 }  // namespace gdn
@@ -52,6 +53,29 @@ struct GdnArgs {
   int rows;
 };
 
+// acc[a][b] = sum_d X[ra[a] * LD + d] * Y[rb[b] * LD + d] over d < D: a
+// 4 x 4 register tile of row dot products (8 shared loads per 16 FMAs).
+__device__ __forceinline__ void dot_tile4(const float* X, const int (&ra)[4], const float* Y,
+                                          const int (&rb)[4], float (&acc)[4][4]) {
+  using namespace gdn;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
+#pragma unroll 4
+  for (int d = 0; d < D; ++d) {
+    float x[4], y[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = X[ra[i] * LD + d];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) y[j] = Y[rb[j] * LD + d];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(x[i], y[j], acc[i][j]);
+  }
+}
+
 __global__ void __launch_bounds__(gdn::THREADS, 1) k_gdn_chunked(const GdnArgs a) {
   using namespace gdn;
   extern __shared__ __align__(16) float gsm[];
@@ -59,8 +83,8 @@ __global__ void __launch_bounds__(gdn::THREADS, 1) k_gdn_chunked(const GdnArgs a
   float* Kc = S + D * LD;           // [C][LD]
   float* Qc = Kc + C * LD;          // [C][LD]
   float* Vc = Qc + C * LD;          // [C][rn]: values, then the right-hand side, then U
-  float* A = Vc + C * D;            // [C][C]: A, then the masked, scaled Q K^T
-  float* G = A + C * C;             // [C] running log decay
+  float* A = Vc + C * D;            // [C][CP]: A, then the masked, scaled Q K^T
+  float* G = A + C * CP;            // [C] running log decay
   float* B = G + C;                 // [C] beta
   float* E = B + C;                 // [C] e^{G_t}
   float* W = E + C;                 // [C] e^{G_last - G_t}
@@ -110,22 +134,47 @@ __global__ void __launch_bounds__(gdn::THREADS, 1) k_gdn_chunked(const GdnArgs a
     }
     __syncthreads();
 
+    // Register tiles of 4 x 4 outputs.  Token rows and key columns map as
+    // base + 16 * k (and value rows as 4 * tile + k), so that across a warp
+    // the shared loads of the inner loops hit distinct banks or broadcast.
+    const int ni = (rn + 3) / 4;              // tiles of 4 value rows
     // A_tj = beta_t e^{G_t - G_j} (k_t . k_j), j < t
-    for (int x = tid; x < C * C; x += THREADS) {
-      const int t = x / C, j = x - t * C;
-      float acc = 0.0f;
-      if (j < t && t < cn) {
-        for (int d = 0; d < D; ++d) acc = fmaf(Kc[t * LD + d], Kc[j * LD + d], acc);
-        acc *= B[t] * expf(G[t] - G[j]);
+    {
+      const int ty = tid / 16, tx = tid % 16;
+      int rt[4], rj[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        rt[k] = ty + 16 * k;
+        rj[k] = tx + 16 * k;
       }
-      A[x] = acc;
+      float acc[4][4];
+      dot_tile4(Kc, rt, Kc, rj, acc);
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int t = rt[p], j = rj[q];
+          A[t * CP + j] = (j < t && t < cn) ? acc[p][q] * B[t] * expf(G[t] - G[j]) : 0.0f;
+        }
     }
     // right-hand side: beta_t v_t - beta_t e^{G_t} S_0 k_t (this CTA's rows)
-    for (int x = tid; x < C * rn; x += THREADS) {
-      const int t = x / rn, i = x - t * rn;
-      float sk = 0.0f;
-      for (int d = 0; d < D; ++d) sk = fmaf(S[i * LD + d], Kc[t * LD + d], sk);
-      Vc[x] = B[t] * Vc[x] - B[t] * E[t] * sk;
+    for (int tile = tid; tile < 16 * ni; tile += THREADS) {
+      const int tt = tile % 16, ti = tile / 16;
+      int rt[4], ri[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        rt[k] = tt + 16 * k;
+        ri[k] = min(4 * ti + k, rn - 1);
+      }
+      float acc[4][4];
+      dot_tile4(Kc, rt, S, ri, acc);
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int t = rt[p], i = 4 * ti + q;
+          if (i < rn) Vc[t * rn + i] = B[t] * Vc[t * rn + i] - B[t] * E[t] * acc[p][q];
+        }
     }
     __syncthreads();
     // (I + A) U = rhs by forward substitution; thread i owns column i
@@ -133,41 +182,99 @@ __global__ void __launch_bounds__(gdn::THREADS, 1) k_gdn_chunked(const GdnArgs a
       const int i = tid;
       for (int t = 1; t < cn; ++t) {
         float acc = Vc[t * rn + i];
-        for (int j = 0; j < t; ++j) acc = fmaf(-A[t * C + j], Vc[j * rn + i], acc);
+        for (int j = 0; j < t; ++j) acc = fmaf(-A[t * CP + j], Vc[j * rn + i], acc);
         Vc[t * rn + i] = acc;
       }
     }
     __syncthreads();
     // P_tj = e^{G_t - G_j} (q_t . k_j), j <= t (into A)
-    for (int x = tid; x < C * C; x += THREADS) {
-      const int t = x / C, j = x - t * C;
-      float acc = 0.0f;
-      if (j <= t && t < cn) {
-        for (int d = 0; d < D; ++d) acc = fmaf(Qc[t * LD + d], Kc[j * LD + d], acc);
-        acc *= expf(G[t] - G[j]);
+    {
+      const int ty = tid / 16, tx = tid % 16;
+      int rt[4], rj[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        rt[k] = ty + 16 * k;
+        rj[k] = tx + 16 * k;
       }
-      A[x] = acc;
+      float acc[4][4];
+      dot_tile4(Qc, rt, Kc, rj, acc);
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int t = rt[p], j = rj[q];
+          A[t * CP + j] = (j <= t && t < cn) ? acc[p][q] * expf(G[t] - G[j]) : 0.0f;
+        }
     }
     __syncthreads();
-    // o_t = e^{G_t} S_0 q_t + sum_j P_tj U_j
-    for (int x = tid; x < cn * rn; x += THREADS) {
-      const int t = x / rn, i = x - t * rn;
-      float sq = 0.0f;
-      for (int d = 0; d < D; ++d) sq = fmaf(S[i * LD + d], Qc[t * LD + d], sq);
-      float pu = 0.0f;
-      for (int j = 0; j <= t; ++j) pu = fmaf(A[t * C + j], Vc[j * rn + i], pu);
-      a.o[((c0 + t) * a.Hv + h) * D + r0 + i] = E[t] * sq + pu;
+    // o_t = e^{G_t} S_0 q_t + sum_j P_tj U_j (P_tj = 0 past t)
+    for (int tile = tid; tile < 16 * ni; tile += THREADS) {
+      const int tt = tile % 16, ti = tile / 16;
+      int rt[4], ri[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        rt[k] = tt + 16 * k;
+        ri[k] = min(4 * ti + k, rn - 1);
+      }
+      float sq[4][4];
+      dot_tile4(Qc, rt, S, ri, sq);
+      float pu[4][4];
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) pu[p][q] = 0.0f;
+      const int jmax = min(rt[3], cn - 1);     // the tile's last token row
+      for (int j = 0; j <= jmax; ++j) {
+        float pv[4], uv[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) pv[p] = A[rt[p] * CP + j];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) uv[q] = Vc[j * rn + ri[q]];
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) pu[p][q] = fmaf(pv[p], uv[q], pu[p][q]);
+      }
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int t = rt[p], i = 4 * ti + q;
+          if (t < cn && i < rn) a.o[((c0 + t) * a.Hv + h) * D + r0 + i] = E[t] * sq[p][q] + pu[p][q];
+        }
     }
     const float gc = G[cn - 1];
     if (tid < C) W[tid] = tid < cn ? expf(gc - G[tid]) : 0.0f;
     __syncthreads();   // every output of the chunk read the old state; W is ready
     // S = e^{G_C} S_0 + sum_t e^{G_C - G_t} U_t k_t^T
     const float ec = expf(gc);
-    for (int x = tid; x < rn * D; x += THREADS) {
-      const int i = x / D, j = x - i * D;
-      float acc = ec * S[i * LD + j];
-      for (int t = 0; t < cn; ++t) acc = fmaf(Vc[t * rn + i] * W[t], Kc[t * LD + j], acc);
-      S[i * LD + j] = acc;
+    for (int tile = tid; tile < 32 * ni; tile += THREADS) {
+      const int tj = tile % 32, ti = tile / 32;
+      int ri[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) ri[k] = min(4 * ti + k, rn - 1);
+      float acc[4][4];
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[p][q] = ec * S[ri[p] * LD + tj + 32 * q];
+      for (int t = 0; t < cn; ++t) {
+        const float w = W[t];
+        float uv[4], kv[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) uv[p] = Vc[t * rn + ri[p]] * w;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) kv[q] = Kc[t * LD + tj + 32 * q];
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc[p][q] = fmaf(uv[p], kv[q], acc[p][q]);
+      }
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+        if (4 * ti + p < rn)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) S[(4 * ti + p) * LD + tj + 32 * q] = acc[p][q];
     }
   }
   __syncthreads();
