@@ -43,9 +43,13 @@ METRIC = "NVFP4 W4A4 linear TFLOPS & % of B200 FP4 peak; small-M weight GB/s"
 FP4_PER_BF16 = 4.0          # nominal dense FP4 / BF16 tensor throughput ratio (9 / 2.25 PFLOP/s)
 ROTATE_ACT = 6              # distinct activation buffers (each step uses the next one)
 ROTATE_W = 4                # distinct weight copies
-# The CTA-pair GEMM gets the caller workspace that lets it run its last
-# partial wave of tiles (and one whole wave) as a stream-K tail.
-SPLIT_TAIL = True
+# The CTA-pair GEMM's stream-K tail (nvfp4_fused_linear_ws) is correct but
+# measured slower than whole tiles on every large configuration here
+# (prefill 60.0 vs 56.9 us, GDN in-projection 327 vs 323 us, interleaved
+# runs): the main loop is bound by L2 -> shared-memory delivery for the whole
+# chip, so the pairs of a partial last wave run their tiles faster, and the
+# stream-K partial tiles add traffic.  The bench launches without it.
+SPLIT_TAIL = False
 
 
 # --------------------------------------------------------------- plumbing

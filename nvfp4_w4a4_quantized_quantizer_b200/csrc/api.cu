@@ -607,7 +607,6 @@ nvfp4_status nvfp4_fused_linear_ws(const void* a_codes, const void* a_scales, co
   nvfp4::GemmArgs g;
   g.sfa = static_cast<const uint8_t*>(a_scales);
   g.sfb = static_cast<const uint8_t*>(w_scales);
-  g.wq = static_cast<const uint8_t*>(w_codes);
   g.M = static_cast<int>(M);
   g.N = static_cast<int>(N);
   g.K = static_cast<int>(K);

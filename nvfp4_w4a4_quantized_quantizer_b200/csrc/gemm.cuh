@@ -53,7 +53,6 @@ struct SegTable {
 struct GemmArgs {
   const uint8_t* sfa;  // activation (or, swapped, token) scale atoms
   const uint8_t* sfb;  // weight scale atoms
-  const uint8_t* wq;   // weight codes [N, K/2] (the small-M kernel's L2 prefetch)
   int M, N, K;
   void* y;
   int64_t ldy;
@@ -65,16 +64,20 @@ struct GemmArgs {
   // tiles [num_tiles - sk_tiles, num_tiles) are not run whole: their
   // sk_tiles * num_kt k-tiles are cut into `units` contiguous ranges of
   // (nearly) equal length, range u = [sk_len * u / units, sk_len * (u + 1) /
-  // units), one per CTA pair, after the pair's whole tiles (dp_tiles =
-  // num_tiles - sk_tiles, a multiple of the pair count, walked u, u + units,
-  // ...).  sk_tiles >= units, so a range is at least one tile long and a tile
-  // is shared by at most two pairs: the pair whose range starts inside it
-  // runs its tail k-tiles first and publishes that fp32 partial tile in
-  // slot u of the caller's workspace (then raises the slot's flag); the pair
-  // whose range ends inside it runs its head k-tiles last, waits for the
-  // flag of slot u + 1, adds the partial to its own accumulator (head +
-  // tail, the same order whatever the timing) and applies the epilogue.
-  // The consumer sets the flag back to zero, so the flags are zero between
+  // units), one per CTA pair, beside the pair's whole data-parallel tiles
+  // (dp_tiles = num_tiles - sk_tiles, a multiple of the pair count, walked
+  // u, u + units, ...).  sk_tiles >= units, so a range is at least one tile
+  // long and a tile is shared by at most two pairs.  The pair whose range
+  // starts inside a tile runs those (tail) k-tiles as its very first item
+  // and publishes the fp32 partial tile in slot u of the caller's
+  // workspace, then raises the slot's flag; the pair whose range ends
+  // inside it runs its (head) k-tiles as its very last item, waits for the
+  // flag of slot u + 1 (raised long before), adds the partial to its own
+  // accumulator (head + tail, the same order whatever the timing) and
+  // applies the epilogue.  A short item right after another one would wait
+  // for the epilogue of the one before to drain the single accumulator;
+  // first and last, the short items overlap whole tiles instead.  The
+  // consumer sets the flag back to zero, so the flags are zero between
   // launches.  sk_tiles == 0: every tile whole.
   int sk_tiles;
   float* partial;      // [slot][2 CTAs][2 column halves][32 chunks][128 rows] float4
@@ -170,8 +173,9 @@ __device__ __forceinline__ int seg_advance(const SegTable& t, int seg, int n) {
 // One item of work of a CTA (pair): k-tiles [kt0, kt1) of one tile, run
 // whole (ITEM_WHOLE), as the tail of a stream-K tile whose partial sum is
 // published (ITEM_TAIL), or as its head, summed with that partial
-// (ITEM_HEAD).  A pair's items: its whole data-parallel tiles, then its
-// stream-K range (a tail, whole tiles, a head; each part optional).
+// (ITEM_HEAD).  A pair's items in order: the tail of its stream-K range (if
+// the range starts inside a tile), its whole data-parallel tiles, the whole
+// tiles of its range, the head of its range (if it ends inside a tile).
 enum ItemKind : int { ITEM_WHOLE = 0, ITEM_TAIL = 1, ITEM_HEAD = 2 };
 
 struct WorkItem {
@@ -221,23 +225,21 @@ __device__ __forceinline__ WorkItem work_item(const WorkPlan& p, int unit, int u
   w.kt0 = 0;
   w.kt1 = num_kt;
   w.kind = ITEM_WHOLE;
-  if (i < p.n_dp) {
-    w.tile = unit + i * units;
-    return w;
-  }
-  int j = i - p.n_dp;
-  int t = p.sk_base;
   if (p.tail_kt0) {
-    if (j == 0) {
-      w.tile = t;
+    if (i == 0) {
+      w.tile = p.sk_base;
       w.kt0 = p.tail_kt0;
       w.kind = ITEM_TAIL;
       return w;
     }
-    --j;
-    ++t;
+    --i;
   }
-  w.tile = t + j;
+  if (i < p.n_dp) {
+    w.tile = unit + i * units;
+    return w;
+  }
+  const int j = i - p.n_dp;
+  w.tile = p.sk_base + (p.tail_kt0 ? 1 : 0) + j;
   if (j >= p.n_whole) {
     w.kt1 = p.head_kt1;
     w.kind = ITEM_HEAD;
@@ -687,9 +689,9 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ACC_COL + half * 128;
       bool ok = !dead;
       // The head k-tiles of a stream-K tile (always the pair's last item):
-      // the tail partial was published by the next pair as the first item of
-      // its range.  Wait for its flag and start loading it while this pair's
-      // own k-tiles finish; once the accumulator is complete, add the
+      // the tail partial was published by the next pair as its first item.
+      // Wait for its flag and start loading it while this pair's own
+      // k-tiles finish; once the accumulator is complete, add the
       // partial to it in TMEM (head + tail), 16 columns at a time with two
       // column groups of it in registers, then run the whole-tile epilogue.
       const bool head = !SWIGLU && wi.kind == ITEM_HEAD;
@@ -780,8 +782,8 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         }
         continue;
       }
-      // the tail k-tiles of a stream-K tile (the first item of the pair's
-      // range): publish the partial in slot `unit`, then raise its flag
+      // the tail k-tiles of a stream-K tile (the pair's first item): publish
+      // the partial in slot `unit`, then raise its flag
       if (ok) {
 #pragma unroll
         for (int c = 0; c < 32; ++c)
@@ -832,7 +834,6 @@ constexpr uint32_t ACC_COL = 0;         // NT columns
 constexpr uint32_t SF_COL = 64;         // + 32 * stage
 constexpr uint32_t SF_STRIDE = 32;
 constexpr int BAR_BYTES = 256;
-constexpr int64_t L2_PREFETCH_CHUNK = 32768;   // bytes per L2 bulk prefetch
 // Two CTAs fit on one SM (shared memory, 256 TMEM columns and <= 80
 // registers per thread each), so that with launch overlap the next call's
 // CTAs start streaming their weights beside this call's.
@@ -911,19 +912,6 @@ __global__ void __launch_bounds__(sm::THREADS, 2)
     // warp-wide loop; one elected lane issues each copy
     {
       const bool is_w = (warp == 0);
-      if (is_w && lane == 0) {
-        // Ask L2 for this CTA's whole weight block (its 128 code rows are
-        // contiguous, K/2 bytes each, and its scale atoms too) before the
-        // kernel ahead has finished: with launch overlap the weight stream
-        // of this call then keeps HBM busy while the call ahead drains, and
-        // the ring below reads most of it from L2.
-        const int rows = min(BW, g.N - wt * BW);
-        const uint8_t* wb = g.wq + static_cast<int64_t>(wt) * BW * (g.K / 2);
-        const int64_t wbytes = static_cast<int64_t>(rows) * (g.K / 2);
-        for (int64_t o = 0; o < wbytes; o += L2_PREFETCH_CHUNK)
-          bulk_prefetch_l2(wb + o, static_cast<uint32_t>(wbytes - o < L2_PREFETCH_CHUNK ? wbytes - o : L2_PREFETCH_CHUNK));
-        bulk_prefetch_l2(g.sfb + wt * kb4 * 512, static_cast<uint32_t>(kb4 * 512));
-      }
       if (!is_w) griddep_wait();   // the token operands may come from the kernel ahead
       // weights stream through once; tokens are re-read by every CTA
       const uint64_t pol = is_w ? policy_evict_first() : policy_evict_last();

@@ -102,13 +102,21 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
 }
 
 // The same wait executed by every lane of a warp, with one decision for the
-// whole warp: true only if every lane saw the phase complete.  Loops that
-// give up on a failed wait and otherwise run warp-collective instructions
-// (elect.sync, shuffles, tcgen05 .sync.aligned forms, named barriers) use
-// this form, so no lane leaves such a loop while others stay in it.
+// whole warp.  Loops that give up on a failed wait and otherwise run
+// warp-collective instructions (elect.sync, shuffles, tcgen05 .sync.aligned
+// forms, named barriers) use this form, so no lane leaves such a loop while
+// others stay in it.  A completed phase stays complete until this warp has
+// consumed it, so lanes that find it complete at once return true without
+// a vote (the common case costs nothing extra); the lanes that had to wait
+// vote among themselves on the result.  A lane that returned at once saw
+// the phase complete, so the waiting lanes see it too and vote true: every
+// lane returns the same value.
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, uint64_t limit_ns,
                                                const volatile int* abort_flag) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, limit_ns, abort_flag));
+  if (mbar_test(bar, parity)) return true;
+  const unsigned waiting = __activemask();   // the lanes that found the phase incomplete
+  const bool ok = mbar_wait(bar, parity, limit_ns, abort_flag);
+  return __all_sync(waiting, ok);
 }
 
 // ------------------------------------------------ flags in global memory
@@ -208,12 +216,6 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
       "l"(src), "r"(bytes), "r"(bar), "l"(policy)
       : "memory");
-}
-
-// Ask L2 to fetch [src, src + bytes) (16-byte aligned, a multiple of 16
-// bytes); no completion is tracked.
-__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 // Warp-wide forms of the copy issue: every lane executes them with the

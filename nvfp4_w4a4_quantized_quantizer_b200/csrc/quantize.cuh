@@ -115,23 +115,24 @@ constexpr int QUANT_SLOTS = 4;
 constexpr int QUANT_SMEM = QUANT_WARPS * QUANT_SLOTS * QUANT_UNIT * 2;   // 64 KB
 constexpr int QUANT_BAR_BYTES = QUANT_WARPS * QUANT_SLOTS * 8;
 
-// |x| max of sixteen bf16 values (eight packed words), exact: the magnitude
-// bits of non-negative bf16 values order like unsigned integers, so one
-// 16-bit-lane unsigned max per word pair does it.
-__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+// |x| max of sixteen bf16 values (eight packed words), exact.  max with
+// .xorsign.abs compares magnitudes (bf16 comparisons are exact, subnormals
+// kept) and returns the larger magnitude with a sign we discard; the word
+// order does not matter.  The result is the bf16 magnitude as fp32 bits.
+__device__ __forceinline__ uint32_t max_abs_bf16x2(uint32_t a, uint32_t b) {
   uint32_t d;
-  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
 }
 
 __device__ __forceinline__ float bf16x16_absmax(const uint32_t (&w)[8]) {
-  const uint32_t m01 = max_u16x2(w[0] & 0x7FFF7FFFu, w[1] & 0x7FFF7FFFu);
-  const uint32_t m23 = max_u16x2(w[2] & 0x7FFF7FFFu, w[3] & 0x7FFF7FFFu);
-  const uint32_t m45 = max_u16x2(w[4] & 0x7FFF7FFFu, w[5] & 0x7FFF7FFFu);
-  const uint32_t m67 = max_u16x2(w[6] & 0x7FFF7FFFu, w[7] & 0x7FFF7FFFu);
-  const uint32_t m = max_u16x2(max_u16x2(m01, m23), max_u16x2(m45, m67));
-  const uint32_t hi = m >> 16, lo = m & 0xFFFFu;
-  return __uint_as_float((hi > lo ? hi : lo) << 16);
+  const uint32_t m01 = max_abs_bf16x2(w[0], w[1]);
+  const uint32_t m23 = max_abs_bf16x2(w[2], w[3]);
+  const uint32_t m45 = max_abs_bf16x2(w[4], w[5]);
+  const uint32_t m67 = max_abs_bf16x2(w[6], w[7]);
+  const uint32_t m = max_abs_bf16x2(max_abs_bf16x2(m01, m23), max_abs_bf16x2(m45, m67));
+  const uint32_t both = max_abs_bf16x2(m, __byte_perm(m, 0u, 0x1032));   // both halves = the max
+  return __uint_as_float((both & 0x7FFFu) << 16);
 }
 
 // The two bf16 values of a packed word times r, as two fp32 products each
@@ -240,9 +241,11 @@ __global__ void __launch_bounds__(QUANT_THREADS) k_quantize(const __grid_constan
       const uint32_t h = static_cast<uint32_t>((lane >> 2) & 1) * 16u;
       const uint4 v0 = ld_shared_v4(slot + e * 2 + h);
       const uint4 v1 = ld_shared_v4(slot + e * 2 + (h ^ 16u));
-      const uint4 lo = h ? v1 : v0, hi = h ? v0 : v1;
-      w[0] = lo.x; w[1] = lo.y; w[2] = lo.z; w[3] = lo.w;
-      w[4] = hi.x; w[5] = hi.y; w[6] = hi.z; w[7] = hi.w;
+      // w holds the block's two halves in load order (swapped for h != 0):
+      // the amax does not depend on the order, the code words are put back
+      // in element order before the store
+      w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+      w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
       const float amax = bf16x16_absmax(w);
       const uint32_t sc = cvt_e4m3(__fdiv_rn(amax, c));
       const float rr = s_rtab[sc];
@@ -262,7 +265,7 @@ __global__ void __launch_bounds__(QUANT_THREADS) k_quantize(const __grid_constan
       const uint32_t s2 = __shfl_down_sync(0xffffffffu, sc, 2);
       const uint32_t s3 = __shfl_down_sync(0xffffffffu, sc, 3);
       if (live) {
-        *reinterpret_cast<uint2*>(code_row + e / 2) = make_uint2(qv[0], qv[1]);
+        *reinterpret_cast<uint2*>(code_row + e / 2) = h ? make_uint2(qv[1], qv[0]) : make_uint2(qv[0], qv[1]);
         if ((lane & 3) == 0) {
           // blocks e/16 .. e/16 + 3 of the unit: atom (e / 64) after the unit's first
           const uint32_t word = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);

@@ -76,8 +76,8 @@ def _gpu_layer(wl, xbits, wbits, calib_bits):
                             gate.get("dt") if s.op == "gdn_decay" else None)
              for i, (s, o) in enumerate(zip(wl.segments, wl.seg_offsets))]
     M = xbits.shape[0]
-    # with the workspace, as bench.py calls it (a stream-K tail when the
-    # tiles do not fill the last wave)
+    # with the workspace (a stream-K tail when the tiles do not fill the
+    # last wave), so that path is checked at full size too
     work = nv.nvfp4_gemm_workspace("cuda")
     y32 = nv.nvfp4_fused_linear(ac, as_, wc, ws, M, wl.N, wl.K, specs, out_dtype=nv.OUT_FP32,
                                 workspace=work)
