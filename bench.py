@@ -702,6 +702,55 @@ def reference_main(args, wl, rank):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------ ncu cases
+# One kernel of one configuration, launched a few times on its own with one
+# set of device-resident operands (a few hundred MB at most), for profiler
+# captures (`ncu -k ... python bench.py --kernel-case NAME`).  Setup launches
+# (weight quantisation, calibration) come first; the listed kernel's launches
+# follow.
+KERNEL_CASES = {
+    "quantize_prefill": "k_quantize on the 4096 x 5120 prefill activations",
+    "gemm_prefill": "k_gemm_tc<2> on the 4096 x 5120 x 5120 prefill projection",
+    "gemm_gdn": "k_gemm_tc<2> on the 8192 x 5120 x 16480 GDN in-projection (6 modules, gates)",
+    "gate_up_mlp": "k_gemm_tc<2, true> (gate_up + SiLU*up + requantisation), 16384 x 5120 x 2 x 17408",
+    "down_mlp": "k_gemm_tc<2> on the 16384 x 17408 x 5120 MLP down projection",
+    "decode_m1": "k_gemm_small<16> on the GDN in-projection weights, 1 token",
+    "decode_m64": "k_gemm_small<64> on the GDN in-projection weights, 64 tokens",
+}
+
+
+def kernel_case(name: str, launches: int, device):
+    import nvfp4_w4a4_quantized_quantizer_b200 as nv
+    st = torch.cuda.current_stream()
+    if name in ("gate_up_mlp", "down_mlp"):
+        ch = MlpChain(device, rotate_act=1, rotate_w=1)
+        ch.quantize(0, st)
+        if name == "down_mlp":
+            ch.gate_up(0, st)
+            fn = ch.down
+        else:
+            fn = ch.gate_up
+    else:
+        wl = workloads.WORKLOADS[{"quantize_prefill": 2, "gemm_prefill": 2, "gemm_gdn": 3,
+                                  "decode_m1": 5, "decode_m64": 5}[name]]
+        M = {"decode_m1": 1, "decode_m64": 64}.get(name, wl.M)
+        layer = Layer(wl, M, device, rotate_act=1, rotate_w=1)
+        layer.quantize(0, st)
+        fn = layer.quantize if name == "quantize_prefill" else layer.gemm
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(st)
+    for i in range(launches):
+        fn(i, st)
+    b.record(st)
+    b.synchronize()
+    st_err, info = nv.nvfp4_last_device_error()
+    print(json.dumps({"kernel_case": name, "what": KERNEL_CASES[name], "launches": launches,
+                      "ms_per_launch": round(a.elapsed_time(b) / launches, 4), "status": st_err}),
+          flush=True)
+    return 0 if st_err == 0 else 1
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -714,6 +763,9 @@ def main():
     ap.add_argument("--no-small-m", action="store_true")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the per-kernel figures of the other large configurations")
+    ap.add_argument("--kernel-case", choices=sorted(KERNEL_CASES),
+                    help="launch one kernel of one configuration a few times (profiler captures)")
+    ap.add_argument("--launches", type=int, default=3)
     ap.add_argument("--no-overlap", action="store_true",
                     help="launch the quantiser and the small-M GEMM without launch overlap")
     args = ap.parse_args()
@@ -726,6 +778,12 @@ def main():
     if args.impl == "reference":
         reference_main(args, wl, rank)
         return
+    if args.kernel_case:
+        import nvfp4_w4a4_quantized_quantizer_b200 as nv
+        nv.load()
+        nv.nvfp4_set_launch_overlap(False)
+        torch.cuda.set_device(local)
+        sys.exit(kernel_case(args.kernel_case, args.launches, torch.device("cuda", local)))
 
     import nvfp4_w4a4_quantized_quantizer_b200 as nv
     nv.load()

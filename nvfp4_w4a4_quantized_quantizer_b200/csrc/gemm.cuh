@@ -436,7 +436,16 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     // ---------------------------------------------------- TMA producers
     // warp-wide loop; one elected lane issues each copy
     {
-      const uint64_t pol = policy_evict_last();
+      // L2 policy per operand.  With the N-fastest raster (activations too
+      // large for L2, e.g. the MLP down projection's 143 MB of codes) each
+      // activation tile is read by consecutive pairs at about the same time
+      // and then not again: it is marked evict-first, and the weights, re-read
+      // for every activation tile, evict-last (down projection 621 vs 639 us).
+      // With the M-fastest raster both stay evict-last: marking the weight
+      // tiles evict-first made the GDN in-projection 3% slower.
+      const uint64_t keep = policy_evict_last();
+      const uint64_t pol_a = g.n_fastest ? policy_evict_first() : keep;
+      const uint64_t pol_b = keep;
       int stage = 0;
       uint32_t phase = 0;
       int64_t issued = 0;
@@ -459,25 +468,25 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
           uint8_t* st = smem + stage * STAGE_BYTES;
           if (warp == 0) {
             mbar_arrive_expect_tx_warp(full_bar(stage), A_BYTES);
-            tma_load_2d_warp(smem_addr(st), &tmA, kt * BKB, arow, full_bar(stage), pol);
+            tma_load_2d_warp(smem_addr(st), &tmA, kt * BKB, arow, full_bar(stage), pol_a);
           } else if (warp == 2) {
             mbar_arrive_expect_tx_warp(full_bar(stage), B_BYTES);
-            tma_load_2d_warp(smem_addr(st + A_BYTES), &tmB, kt * BKB, brow, full_bar(stage), pol);
+            tma_load_2d_warp(smem_addr(st + A_BYTES), &tmB, kt * BKB, brow, full_bar(stage), pol_b);
           } else {
             // both boxes always transfer their full size (out-of-range atoms read as 0)
             mbar_arrive_expect_tx_warp(sfull_bar(stage), SFA_BYTES + SFB_BYTES);
             tma_load_3d_warp(smem_addr(st + A_BYTES + B_BYTES), &tmSA, 0, kt * 4,
-                        mb * CG + static_cast<int>(rank), sfull_bar(stage), pol);
+                        mb * CG + static_cast<int>(rank), sfull_bar(stage), pol_a);
             if constexpr (SWIGLU) {
               // the gate rows' scale block, then the up rows' (1-block boxes)
               tma_load_3d_warp(smem_addr(st + A_BYTES + B_BYTES + SFA_BYTES), &tmSB, 0, kt * 4, nb,
-                               sfull_bar(stage), pol);
+                               sfull_bar(stage), pol_b);
               tma_load_3d_warp(smem_addr(st + A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES / 2), &tmSB, 0,
-                               kt * 4, g.H / 128 + nb, sfull_bar(stage), pol);
+                               kt * 4, g.H / 128 + nb, sfull_bar(stage), pol_b);
             } else {
               // both row blocks of the tile (2-block boxes)
               tma_load_3d_warp(smem_addr(st + A_BYTES + B_BYTES + SFA_BYTES), &tmSB, 0, kt * 4,
-                               nb * 2, sfull_bar(stage), pol);
+                               nb * 2, sfull_bar(stage), pol_b);
             }
           }
           ++issued;
@@ -625,6 +634,9 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     // 16 grp .. 16 grp + 15 of this thread's 128.
     // Rows past M skip only the stores: fetch may issue warp-collective
     // TMEM loads, so every lane of the warp runs it.
+    // With the N-fastest raster the output is marked evict-first too, so it
+    // does not push the kept weights out of L2.
+    const uint64_t out_pol = g.n_fastest ? policy_evict_first() : policy_evict_normal();
     auto store_row = [&](int mb, int nb, auto&& fetch) {
       const int64_t gm = static_cast<int64_t>(mb * CG + static_cast<int>(rank)) * BM + row_in_tile;
       const bool row_live = gm < g.M;
@@ -665,7 +677,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             }
             __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.y) + gm * g.ldy + n;
             if (g.sector_stores) {
-              st_global_v8(dst, w);   // the row's 16 columns = one full 32-byte sector
+              st_global_v8_hint(dst, w, out_pol);   // the row's 16 columns = one full 32-byte sector
             } else {
               reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
               reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
@@ -829,25 +841,31 @@ constexpr int SFW_WARP0 = 4;
 constexpr int EPI_WARP0 = 8;
 constexpr int EPI_WARPS = 4;
 constexpr int THREADS = 32 * (EPI_WARP0 + EPI_WARPS);
-constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t ACC_COL = 0;         // NT columns
 constexpr uint32_t SF_COL = 64;         // + 32 * stage
 constexpr uint32_t SF_STRIDE = 32;
 constexpr int BAR_BYTES = 256;
-// Two CTAs fit on one SM (shared memory, 256 TMEM columns and <= 80
-// registers per thread each), so that with launch overlap the next call's
-// CTAs start streaming their weights beside this call's.
 constexpr int SMEM_PER_SM = 233472;     // 228 KB
 constexpr int SMEM_RESERVED = 1024;     // per CTA
+// Up to 16 tokens two CTAs fit on one SM (shared memory, 256 TMEM columns
+// and <= 80 registers per thread each), so that with launch overlap the
+// next call's CTAs start streaming their weights beside this call's.  With
+// 32 or 64 tokens a stage carries 4 or 8 KB of tokens beside 16 KB of
+// weights, and a CTA alone on its SM with 8 or 7 stages streams faster than
+// two with 4 or 3 each (13.4 vs 14.5 us and 16.9 vs 19.6 us per call with
+// overlap on; interleaved runs).
 template <int NT>
 struct Cfg {
   static constexpr int X_BYTES = NT * BKB;   // NT rows x 128 bytes
   static constexpr int STAGE_BYTES = W_BYTES + X_BYTES + SFW_BYTES + SFX_BYTES;
-  static constexpr int STAGES = NT <= 16 ? 5 : (NT <= 32 ? 4 : 3);   // 22 / 24 / 28 KB stages
+  static constexpr int STAGES = NT <= 16 ? 5 : (NT <= 32 ? 8 : 7);   // 22 / 24 / 28 KB stages
+  static constexpr bool TWO_PER_SM = NT <= 16;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+  static constexpr uint32_t TMEM_COLS = SF_COL + STAGES * SF_STRIDE <= 256 ? 256u : 512u;
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
   static_assert(SF_COL + STAGES * SF_STRIDE <= TMEM_COLS, "TMEM budget");
-  static_assert(2 * (SMEM_BYTES + SMEM_RESERVED) <= SMEM_PER_SM, "two CTAs per SM");
+  static_assert(!TWO_PER_SM || 2 * (SMEM_BYTES + SMEM_RESERVED) <= SMEM_PER_SM, "two CTAs per SM");
+  static_assert(TWO_PER_SM || SMEM_BYTES + SMEM_RESERVED <= SMEM_PER_SM, "shared memory");
   static_assert(NT * BW * 4 <= STAGES * STAGE_BYTES, "the epilogue's transpose fits the ring");
 };
 }  // namespace sm
@@ -895,7 +913,7 @@ __global__ void __launch_bounds__(sm::THREADS, 2)
     prefetch_tensormap(&tmX);
   }
   if (warp == 1) {
-    tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
+    tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -1032,7 +1050,19 @@ __global__ void __launch_bounds__(sm::THREADS, 2)
     // every MMA has completed) so that each token's 128 columns leave as
     // 16-byte stores of one contiguous segment instead of M strided 2-byte
     // stores per thread.
+    // This column's module, alpha and gate parameters, looked up while the
+    // weights stream (each lookup is a dependent constant-bank or global
+    // load; after the accumulator is ready they would delay the stores).
+    // Columns past N (the last tile's padding) are never stored; they take
+    // no gate, so no gate parameter past the module's heads is read.
+    const bool live = n < g.N;
+    const int s = seg_advance(seg, 0, live ? n : g.N - 1);
+    const float alpha = seg.alpha[s];
+    const int op = live ? seg.op[s] : 0;     // columns past N take no gate
+    const int h = n - seg.n_off[s];
     griddep_wait();   // y may still be read or written by the kernel ahead
+    const float ea = op == 2 ? __expf(__ldg(seg.a_log[s] + h)) : 0.0f;
+    const float dtb = op == 2 ? __ldg(seg.dt_bias[s] + h) : 0.0f;
     const bool ok = mbar_wait_warp(acc_full, 0, g.wait_ns, abort_flag);
     if (ok) {
       tc_fence_after();
@@ -1044,15 +1074,6 @@ __global__ void __launch_bounds__(sm::THREADS, 2)
         tmem_ld_x16(taddr + 16 * c, rr);
       }
       tmem_wait_ld();
-      // columns past N (the last tile's padding) are never stored; they take
-      // no gate, so no gate parameter past the module's heads is read
-      const bool live = n < g.N;
-      const int s = seg_advance(seg, 0, live ? n : g.N - 1);
-      const float alpha = seg.alpha[s];
-      const int op = live ? seg.op[s] : 0;     // columns past N take no gate
-      const int h = n - seg.n_off[s];
-      const float ea = op == 2 ? __expf(__ldg(seg.a_log[s] + h)) : 0.0f;
-      const float dtb = op == 2 ? __ldg(seg.dt_bias[s] + h) : 0.0f;
       float* t32 = reinterpret_cast<float*>(smem);
       __nv_bfloat16* t16 = reinterpret_cast<__nv_bfloat16*>(smem);
       auto emit = [&](int j, float o) {
@@ -1114,7 +1135,7 @@ __global__ void __launch_bounds__(sm::THREADS, 2)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+  if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
 }
 
 }  // namespace nvfp4
