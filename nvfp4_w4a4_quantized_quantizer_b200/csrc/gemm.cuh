@@ -25,7 +25,7 @@
 //   k_gemm_small  M <= 64 (decode shapes): operands swapped so the weight
 //                 rows fill the 128-row MMA side and the tokens are the MMA N
 //                 dimension (16/32/64); one CTA per 128 weight rows streams
-//                 the whole K range through a 6-stage ring.
+//                 the whole K range through a ring of 7-9 stages.
 // Every wait is bounded (mbar_wait); a wait that runs out records the
 // device error word, raises the abort flag (of both CTAs of a pair) and the
 // kernel returns after draining its own copies and MMAs and freeing TMEM.
@@ -860,25 +860,24 @@ constexpr uint32_t SF_STRIDE = 32;
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_PER_SM = 233472;     // 228 KB
 constexpr int SMEM_RESERVED = 1024;     // per CTA
-// Up to 16 tokens two CTAs fit on one SM (shared memory, 256 TMEM columns
-// and <= 80 registers per thread each), so that with launch overlap the
-// next call's CTAs start streaming their weights beside this call's.  With
-// 32 or 64 tokens a stage carries 4 or 8 KB of tokens beside 16 KB of
-// weights, and a CTA alone on its SM with 8 or 7 stages streams faster than
-// two with 4 or 3 each (13.4 vs 14.5 us and 16.9 vs 19.6 us per call with
-// overlap on; interleaved runs).
+// One CTA per SM with the deepest ring that fits: 9 / 8 / 7 stages of 22 /
+// 24 / 28 KB for 16 / 32 / 64 tokens.  Each CTA streams one 128-row weight
+// block, and its rate is bounded by the bytes it has in flight, so depth
+// beats a second CTA per SM: at 16 tokens two CTAs of 5 stages (the next
+// call's CTAs streaming beside this call's under launch overlap) took 10.8
+// us per call on 16480 x 5120 weights, one of 9 stages 10.2 us, and a
+// 10th stage or an L2 run-ahead prefetch of 5-10 k-tiles beyond the ring
+// gained nothing or lost (interleaved runs).
 template <int NT>
 struct Cfg {
   static constexpr int X_BYTES = NT * BKB;   // NT rows x 128 bytes
   static constexpr int STAGE_BYTES = W_BYTES + X_BYTES + SFW_BYTES + SFX_BYTES;
-  static constexpr int STAGES = NT <= 16 ? 5 : (NT <= 32 ? 8 : 7);   // 22 / 24 / 28 KB stages
-  static constexpr bool TWO_PER_SM = NT <= 16;
+  static constexpr int STAGES = NT <= 16 ? 9 : (NT <= 32 ? 8 : 7);
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = SF_COL + STAGES * SF_STRIDE <= 256 ? 256u : 512u;
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
   static_assert(SF_COL + STAGES * SF_STRIDE <= TMEM_COLS, "TMEM budget");
-  static_assert(!TWO_PER_SM || 2 * (SMEM_BYTES + SMEM_RESERVED) <= SMEM_PER_SM, "two CTAs per SM");
-  static_assert(TWO_PER_SM || SMEM_BYTES + SMEM_RESERVED <= SMEM_PER_SM, "shared memory");
+  static_assert(SMEM_BYTES + SMEM_RESERVED <= SMEM_PER_SM, "shared memory");
   static_assert(NT * BW * 4 <= STAGES * STAGE_BYTES, "the epilogue's transpose fits the ring");
 };
 }  // namespace sm
@@ -886,7 +885,7 @@ struct Cfg {
 // tmW: weight codes [N, K/2]; tmX: token codes [M, K/2].  D (TMEM) is
 // [128 weight rows] x [NT tokens]; y[token, n] is written transposed back.
 template <int NT>
-__global__ void __launch_bounds__(sm::THREADS, 2)
+__global__ void __launch_bounds__(sm::THREADS, 1)
     k_gemm_small(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                  const GemmArgs g, const __grid_constant__ SegTable seg) {
   using namespace sm;
