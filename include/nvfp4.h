@@ -345,18 +345,20 @@ nvfp4_status nvfp4_last_device_error(nvfp4_stream_t stream, uint64_t* info);
 nvfp4_status nvfp4_set_gemm_path(int32_t path);
 
 /* Launch overlap (process-wide, off by default; on = 1, off = 0): the
- * activation quantiser and the small-M GEMM (M <= 64) are launched with
+ * activation quantiser and every GEMM (nvfp4_linear, nvfp4_fused_linear,
+ * nvfp4_fused_linear_ws, nvfp4_gate_up_silu_quantize) are launched with
  * programmatic stream serialization, so that each may start while the
- * kernel ahead of it on the stream is still running and the next call's
- * weight stream overlaps this call's tail (the decode loop of consecutive
- * layers).  The quantiser waits for the kernel ahead before it reads x or
- * writes codes and scales.  The GEMM waits for it before it reads the
- * activation codes and scales and before it writes y, but streams the
- * weight codes and scales from its start: with overlap on, the kernel
- * launched just ahead of a small-M GEMM on the same stream must not write
- * that GEMM's weight codes or scales (weights quantised offline, or any
- * other kernel in between, satisfy this).  Results are identical with
- * overlap on or off. */
+ * kernel ahead of it on the stream is still running: its setup and the
+ * first stages of its weight stream overlap that kernel's tail (the decode
+ * loop of consecutive layers; the last partial wave of a large GEMM).  The
+ * quantiser waits for the kernel ahead before it reads x or writes codes
+ * and scales.  A GEMM waits for it before it reads the activation codes or
+ * any scales and before it writes y (h) or its workspace, but streams the
+ * weight codes from its start (the small-M GEMM also the weight scales):
+ * with overlap on, the kernel launched just ahead of a GEMM on the same
+ * stream must not write that GEMM's weight codes or scales (weights
+ * quantised offline, or any other kernel in between, satisfy this).
+ * Results are identical with overlap on or off. */
 nvfp4_status nvfp4_set_launch_overlap(int32_t on);
 
 /* Time limit of every bounded in-kernel wait, in nanoseconds (default 2e9;

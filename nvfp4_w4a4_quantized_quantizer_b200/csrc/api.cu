@@ -367,10 +367,11 @@ nvfp4_status noalloc_scratch(float** out) {
 }
 
 // Launch configuration of a CTA-pair kernel (clusters of two CTAs, its
-// dynamic shared memory, `st`); once per device and kernel, also the
-// shared-memory attribute and the number of pairs that fit at once (clusters
-// are placed within one GPC, so an SM count that is odd inside a GPC leaves
-// an SM out).  attr must outlive cfg.
+// dynamic shared memory, `st`, and with launch overlap on programmatic
+// stream serialization); once per device and kernel, also the shared-memory
+// attribute and the number of pairs that fit at once (clusters are placed
+// within one GPC, so an SM count that is odd inside a GPC leaves an SM
+// out).  attr (two entries) must outlive cfg.
 template <typename Kernel>
 nvfp4_status pair_config(Kernel kernel, DeviceInfo* info, bool* configured, int* max_pairs,
                          cudaStream_t st, cudaLaunchConfig_t* cfg, cudaLaunchAttribute* attr) {
@@ -399,6 +400,11 @@ nvfp4_status pair_config(Kernel kernel, DeviceInfo* info, bool* configured, int*
     }
     *max_pairs = clusters;
     *configured = true;
+  }
+  if (g_overlap) {
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg->numAttrs = 2;
   }
   return NVFP4_OK;
 }
@@ -670,11 +676,11 @@ nvfp4_status nvfp4_fused_linear_ws(const void* a_codes, const void* a_scales, co
     }
     const int64_t tiles = ((M + nvfp4::tc::BM - 1) / nvfp4::tc::BM) * num_n;
     const int grid = static_cast<int>(tiles < info->sms ? tiles : info->sms);
-    nvfp4::k_gemm_tc<1><<<grid, nvfp4::tc::THREADS, smem, cs>>>(ta, tb, tsa, tsb, g, table);
-    return check_launch();
+    return launch_maybe_overlapped(nvfp4::k_gemm_tc<1>, dim3(grid), dim3(nvfp4::tc::THREADS), smem,
+                                   cs, ta, tb, tsa, tsb, g, table);
   }
   cudaLaunchConfig_t cfg;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   if ((st = pair_config(nvfp4::k_gemm_tc<2>, info, &info->attr_tc2, &info->pairs, cs, &cfg,
                         attr)) != NVFP4_OK)
     return st;
@@ -762,7 +768,7 @@ nvfp4_status nvfp4_gate_up_silu_quantize(const void* a_codes, const void* a_scal
   if ((st = scale_map(w_scales, 2 * H, K, 1, dev, &tsb)) != NVFP4_OK) return st;
 
   cudaLaunchConfig_t cfg;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   if ((st = pair_config(nvfp4::k_gemm_tc<2, true>, info, &info->attr_tc2_swiglu,
                         &info->swiglu_pairs, cs, &cfg, attr)) != NVFP4_OK)
     return st;

@@ -442,12 +442,19 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     cluster_sync();   // the other CTA's barriers are initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // With launch overlap the next kernel may now be scheduled as SMs free up.
+  // Only the weight codes stream before the kernel ahead has finished: the
+  // activation and scale producers and the epilogue wait for it
+  // (griddep_wait) before they read its outputs or write y, h or the
+  // stream-K workspace.
+  griddep_launch_dependents();
 
   // Each warpgroup resizes its registers at the top of its own branch.
   if (warp < SFW_WARP0) regs_dealloc<REGS_SMALL>();
   if (warp == 0 || warp == 2 || warp == 3) {
     // ---------------------------------------------------- TMA producers
     // warp-wide loop; one elected lane issues each copy
+    if (warp != 2) griddep_wait();   // activation codes and both operands' scales
     {
       // L2 policy per operand.  With the N-fastest raster (activations too
       // large for L2, e.g. the MLP down projection's 143 MB of codes) each
@@ -639,6 +646,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
   } else if (warp >= EPI_WARP0) {
     // ---------------------------------------------------------- epilogue
     regs_alloc<REGS_EPI>();
+    griddep_wait();   // y (or h) and the workspace may still be in use by the kernel ahead
     const int q = warp & 3;                       // TMEM lane quarter this warp may access
     const int half = (warp - EPI_WARP0) >> 2;     // columns [128*half, 128*half + 128)
     const int row_in_tile = q * 32 + lane;

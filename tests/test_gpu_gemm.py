@@ -271,6 +271,79 @@ def test_overlap_keeps_stream_order_of_shared_buffers(overlap):
     assert nv.nvfp4_last_device_error()[0] == 0
 
 
+@pytest.mark.parametrize("path,M", [(AUTO, 300), (LARGE, 200), (PAIR, 300), (PAIR_NFAST, 520)])
+def test_overlap_keeps_stream_order_large_gemm(path, M, overlap):
+    """The same chain of layers through one code buffer and one output
+    buffer on the large-M kernels (one CTA per tile, CTA pairs, both
+    rasters), each launched just behind the quantiser that writes its
+    activation codes: bit-identical to the launches without overlap."""
+    N, K = 2064, 1024
+    nv.nvfp4_set_gemm_path(path)
+    layers = [_decode_layer(M, N, K, seed=300 + 11 * i) for i in range(3)]
+    nv.nvfp4_set_launch_overlap(False)
+    expect = []
+    for xb, _, a_gs, wc, ws, w_gs in layers:
+        ac, as_ = nv.nvfp4_quantize_act(H.bf16_dev(xb), a_gs)
+        expect.append(nv.nvfp4_linear(ac, as_, a_gs, wc, ws, w_gs, M, N, K, out_dtype=nv.OUT_FP32).cpu())
+    nv.nvfp4_set_launch_overlap(True)
+    xs = [H.bf16_dev(l[0]) for l in layers]
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+    scales = torch.empty(nv.nvfp4_scale_bytes(M, K), dtype=torch.uint8, device="cuda")
+    outs = [torch.empty((M, N), dtype=torch.float32, device="cuda") for _ in layers]
+    y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    for rep in range(3):
+        for i, (_, _, a_gs, wc, ws, w_gs) in enumerate(layers):
+            nv.nvfp4_quantize_act(xs[i], a_gs, codes=codes, scales=scales)
+            nv.nvfp4_linear(codes, scales, a_gs, wc, ws, w_gs, M, N, K, y=outs[i],
+                            out_dtype=nv.OUT_FP32)
+        for i in range(len(layers)):
+            assert torch.equal(outs[i].cpu(), expect[i]), (rep, i)
+        for i, (_, _, a_gs, wc, ws, w_gs) in enumerate(layers):
+            nv.nvfp4_quantize_act(xs[i], a_gs, codes=codes, scales=scales)
+            nv.nvfp4_linear(codes, scales, a_gs, wc, ws, w_gs, M, N, K, y=y, out_dtype=nv.OUT_FP32)
+        assert torch.equal(y.cpu(), expect[-1]), rep
+    assert nv.nvfp4_last_device_error()[0] == 0
+
+
+def test_overlap_mlp_chain(overlap):
+    """quantise x -> gate_up + SiLU * up + requantisation of h -> down, the
+    down GEMM with its stream-K workspace, repeated through the same h and y
+    buffers with launch overlap: equal to the chain without overlap."""
+    # down: 9 x 10 tiles of 256 x 256 on 74 pairs, so the workspace's
+    # stream-K tail runs (flags and partial tiles behind griddep_wait)
+    M, Hd, K, N2 = 2304, 640, 512, 2560
+    xb = workloads.random_bf16((M, K), seed=71, std=1.0)
+    wgu = workloads.random_bf16((2 * Hd, K), seed=72, std=1 / np.sqrt(K))
+    wd = workloads.random_bf16((N2, Hd), seed=73, std=1 / np.sqrt(Hd))
+    a_gs = float(oracle.global_scale(np.abs(H.f32(xb)).max()))
+    wc, ws, (g_gs, u_gs) = nv.nvfp4_quantize_weight(H.bf16_dev(wgu), seg_offsets=[0, Hd])
+    dc, dsc, (d_gs,) = nv.nvfp4_quantize_weight(H.bf16_dev(wd))
+    h_gs = 0.01
+    work = nv.nvfp4_gemm_workspace(torch.device("cuda"))
+    x = H.bf16_dev(xb)
+
+    def chain(hc, hs, y):
+        ac, as_ = nv.nvfp4_quantize_act(x, a_gs)
+        nv.nvfp4_gate_up_silu_quantize(ac, as_, wc, ws, M, Hd, K, a_gs, g_gs, u_gs, h_gs,
+                                       h_codes=hc, h_scales=hs)
+        segs = [nv.SegmentSpec(0, d_gs, h_gs)]
+        nv.nvfp4_fused_linear(hc, hs, dc, dsc, M, N2, Hd, segs, y=y, out_dtype=nv.OUT_FP32,
+                              workspace=work)
+
+    hc = torch.empty((M, Hd // 2), dtype=torch.uint8, device="cuda")
+    hs = torch.empty(nv.nvfp4_scale_bytes(M, Hd), dtype=torch.uint8, device="cuda")
+    y = torch.empty((M, N2), dtype=torch.float32, device="cuda")
+    nv.nvfp4_set_launch_overlap(False)
+    chain(hc, hs, y)
+    ref_h, ref_s, ref_y = hc.cpu(), hs.cpu(), y.cpu()
+    nv.nvfp4_set_launch_overlap(True)
+    for rep in range(4):
+        chain(hc, hs, y)
+    assert torch.equal(hc.cpu(), ref_h) and torch.equal(hs.cpu(), ref_s)
+    assert torch.equal(y.cpu(), ref_y)
+    assert nv.nvfp4_last_device_error()[0] == 0
+
+
 # ----------------------------------------------- stream-K tail (workspace)
 # Shapes with more 256 x 256 tiles than a B200's 74 CTA pairs and a partial
 # last wave, so the last 74 + remainder tiles run as equal k-tile ranges per
