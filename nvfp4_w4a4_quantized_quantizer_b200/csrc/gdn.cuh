@@ -21,8 +21,8 @@
 //
 // k_gdn_chunked: one CTA per (value head, block of value rows); the fp32
 // state rows and one chunk's keys, queries and value columns stay in shared
-// memory (at most 182 KB); fp32 CUDA-core arithmetic.  A first correct form:
-// the products are dense and would belong on the tensor cores.
+// memory (at most 186 KB); fp32 CUDA-core arithmetic.  The products are
+// dense and would belong on the tensor cores.
 #pragma once
 
 #include <cstdint>
@@ -31,7 +31,11 @@ namespace nvfp4 {
 namespace gdn {
 constexpr int C = 64;          // tokens per chunk
 constexpr int D = 128;         // key and value head width
-constexpr int LD = D + 1;      // padded rows of S, K, Q: a warp reading a column is bank-conflict free
+// Rows of S, K and Q are padded to 132 floats: 16-byte aligned for float4
+// loads along d, and 33 16-byte bank groups apart, so eight lanes reading
+// eight consecutive rows at one d (a quarter warp's 128-bit access) hit
+// eight different groups.
+constexpr int LD = D + 4;
 constexpr int CP = C + 1;      // padded rows of A
 constexpr int THREADS = 256;
 constexpr int SMEM_FLOATS = D * LD + 2 * C * LD + C * D + C * CP + 4 * C;
@@ -53,8 +57,9 @@ struct GdnArgs {
   int rows;
 };
 
-// acc[a][b] = sum_d X[ra[a] * LD + d] * Y[rb[b] * LD + d] over d < D: a
-// 4 x 4 register tile of row dot products (8 shared loads per 16 FMAs).
+// acc[a][b] = sum_d X[ra[a] * LD + d] * Y[rb[b] * LD + d] over d < D, d in
+// order: a 4 x 4 register tile of row dot products, four d at a time from
+// 128-bit shared loads (8 loads per 64 FMAs).
 __device__ __forceinline__ void dot_tile4(const float* X, const int (&ra)[4], const float* Y,
                                           const int (&rb)[4], float (&acc)[4][4]) {
   using namespace gdn;
@@ -62,17 +67,22 @@ __device__ __forceinline__ void dot_tile4(const float* X, const int (&ra)[4], co
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
-#pragma unroll 4
-  for (int d = 0; d < D; ++d) {
-    float x[4], y[4];
+#pragma unroll 2
+  for (int d = 0; d < D; d += 4) {
+    float4 x[4], y[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) x[i] = X[ra[i] * LD + d];
+    for (int i = 0; i < 4; ++i) x[i] = *reinterpret_cast<const float4*>(X + ra[i] * LD + d);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) y[j] = Y[rb[j] * LD + d];
+    for (int j = 0; j < 4; ++j) y[j] = *reinterpret_cast<const float4*>(Y + rb[j] * LD + d);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(x[i], y[j], acc[i][j]);
+      for (int j = 0; j < 4; ++j) {
+        acc[i][j] = fmaf(x[i].x, y[j].x, acc[i][j]);
+        acc[i][j] = fmaf(x[i].y, y[j].y, acc[i][j]);
+        acc[i][j] = fmaf(x[i].z, y[j].z, acc[i][j]);
+        acc[i][j] = fmaf(x[i].w, y[j].w, acc[i][j]);
+      }
   }
 }
 
@@ -101,12 +111,13 @@ __global__ void __launch_bounds__(gdn::THREADS, 1) k_gdn_chunked(const GdnArgs a
   for (int64_t c0 = 0; c0 < a.T; c0 += C) {
     const int cn = static_cast<int>(a.T - c0 < C ? a.T - c0 : C);
     __syncthreads();   // the previous chunk is done with Kc, Qc, Vc, A and S
-    for (int x = tid; x < C * D; x += THREADS) {
-      const int t = x / D, d = x - t * D;
+    for (int x = tid; x < C * D / 4; x += THREADS) {
+      const int t = x / (D / 4), d = 4 * (x - t * (D / 4));
       const bool live = t < cn;
-      const int64_t tok = c0 + t;
-      Kc[t * LD + d] = live ? a.k[(tok * Hk + hk) * D + d] : 0.0f;
-      Qc[t * LD + d] = live ? a.q[(tok * Hk + hk) * D + d] : 0.0f;
+      const int64_t at = (static_cast<int64_t>(c0 + t) * Hk + hk) * D + d;
+      const float4 zero = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      *reinterpret_cast<float4*>(Kc + t * LD + d) = live ? *reinterpret_cast<const float4*>(a.k + at) : zero;
+      *reinterpret_cast<float4*>(Qc + t * LD + d) = live ? *reinterpret_cast<const float4*>(a.q + at) : zero;
     }
     for (int x = tid; x < C * rn; x += THREADS) {
       const int t = x / rn, i = x - t * rn;
