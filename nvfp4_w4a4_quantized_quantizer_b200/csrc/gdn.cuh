@@ -21,8 +21,9 @@
 //
 // k_gdn_chunked: one CTA per (value head, block of value rows); the fp32
 // state rows and one chunk's keys, queries and value columns stay in shared
-// memory (at most 186 KB); fp32 CUDA-core arithmetic.  The products are
-// dense and would belong on the tensor cores.
+// memory (at most 187 KB); fp32 CUDA-core arithmetic with register tiles fed
+// by 128-bit shared loads.  The products are dense and would belong on the
+// tensor cores.
 #pragma once
 
 #include <cstdint>
@@ -36,7 +37,7 @@ constexpr int D = 128;         // key and value head width
 // eight consecutive rows at one d (a quarter warp's 128-bit access) hit
 // eight different groups.
 constexpr int LD = D + 4;
-constexpr int CP = C + 1;      // padded rows of A
+constexpr int CP = C + 4;      // padded rows of A: 16-byte aligned, 17 bank groups apart
 constexpr int THREADS = 256;
 constexpr int SMEM_FLOATS = D * LD + 2 * C * LD + C * D + C * CP + 4 * C;
 constexpr int SMEM_BYTES = SMEM_FLOATS * 4;
@@ -92,7 +93,7 @@ __global__ void __launch_bounds__(gdn::THREADS, 1) k_gdn_chunked(const GdnArgs a
   float* S = gsm;                   // [rn value rows][LD key]
   float* Kc = S + D * LD;           // [C][LD]
   float* Qc = Kc + C * LD;          // [C][LD]
-  float* Vc = Qc + C * LD;          // [C][rn]: values, then the right-hand side, then U
+  float* Vc = Qc + C * LD;          // [C][RP]: values, then the right-hand side, then U
   float* A = Vc + C * D;            // [C][CP]: A, then the masked, scaled Q K^T
   float* G = A + C * CP;            // [C] running log decay
   float* B = G + C;                 // [C] beta
@@ -101,12 +102,14 @@ __global__ void __launch_bounds__(gdn::THREADS, 1) k_gdn_chunked(const GdnArgs a
   const int h = blockIdx.x / a.parts;          // value head
   const int r0 = (blockIdx.x % a.parts) * a.rows;
   const int rn = min(D, r0 + a.rows) - r0;      // this CTA's value rows [r0, r0 + rn)
+  const int RP = (rn + 3) & ~3;                  // row pitch of Vc: float4 rows, columns past rn zero
   const int hk = h / a.group;
   const int Hk = a.Hv / a.group;
   const int tid = threadIdx.x;
   float* state = a.state + (static_cast<int64_t>(h) * D + r0) * D;
 
   for (int x = tid; x < rn * D; x += THREADS) S[(x / D) * LD + x % D] = state[x];
+  for (int x = tid; x < C * RP; x += THREADS) Vc[x] = 0.0f;
 
   for (int64_t c0 = 0; c0 < a.T; c0 += C) {
     const int cn = static_cast<int>(a.T - c0 < C ? a.T - c0 : C);
@@ -121,7 +124,7 @@ __global__ void __launch_bounds__(gdn::THREADS, 1) k_gdn_chunked(const GdnArgs a
     }
     for (int x = tid; x < C * rn; x += THREADS) {
       const int t = x / rn, i = x - t * rn;
-      Vc[x] = t < cn ? a.v[((c0 + t) * a.Hv + h) * D + r0 + i] : 0.0f;
+      Vc[t * RP + i] = t < cn ? a.v[((c0 + t) * a.Hv + h) * D + r0 + i] : 0.0f;
     }
     if (tid < 32) {
       // running sum of g over the chunk: 64 values, two per lane
@@ -184,20 +187,41 @@ __global__ void __launch_bounds__(gdn::THREADS, 1) k_gdn_chunked(const GdnArgs a
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int t = rt[p], i = 4 * ti + q;
-          if (i < rn) Vc[t * rn + i] = B[t] * Vc[t * rn + i] - B[t] * E[t] * acc[p][q];
+          if (i < rn) Vc[t * RP + i] = B[t] * Vc[t * RP + i] - B[t] * E[t] * acc[p][q];
         }
     }
     __syncthreads();
-    // (I + A) U = rhs by forward substitution; thread i owns column i
-    if (tid < rn) {
-      const int i = tid;
-      for (int t = 1; t < cn; ++t) {
-        float acc = Vc[t * rn + i];
-        for (int j = 0; j < t; ++j) acc = fmaf(-A[t * CP + j], Vc[j * rn + i], acc);
-        Vc[t * rn + i] = acc;
+    // (I + A) U = rhs by forward substitution in 16-row blocks: the terms
+    // of the rows solved in earlier blocks are one product computed by all
+    // threads, then the block's own rows are solved column by column
+    // (thread i, column i).  Rows past cn have zero right-hand sides and
+    // zero rows of A.
+    for (int t0 = 0; t0 < cn; t0 += 16) {
+      if (t0 > 0) {
+        for (int x = tid; x < 16 * rn; x += THREADS) {
+          const int t = t0 + x / rn, i = x - (x / rn) * rn;
+          const float* At = A + t * CP;
+          float s0 = 0.0f, s1 = 0.0f;
+          for (int j = 0; j < t0; j += 2) {
+            s0 = fmaf(At[j], Vc[j * RP + i], s0);
+            s1 = fmaf(At[j + 1], Vc[(j + 1) * RP + i], s1);
+          }
+          Vc[t * RP + i] -= s0 + s1;
+        }
+        __syncthreads();
       }
+      if (tid < rn) {
+        const int i = tid;
+        const int t1 = min(t0 + 16, cn);
+        for (int t = t0 + 1; t < t1; ++t) {
+          const float* At = A + t * CP;
+          float s = 0.0f;
+          for (int j = t0; j < t; ++j) s = fmaf(At[j], Vc[j * RP + i], s);
+          Vc[t * RP + i] -= s;
+        }
+      }
+      __syncthreads();
     }
-    __syncthreads();
     // P_tj = e^{G_t - G_j} (q_t . k_j), j <= t (into A)
     {
       const int ty = tid / 16, tx = tid % 16;
@@ -234,17 +258,27 @@ __global__ void __launch_bounds__(gdn::THREADS, 1) k_gdn_chunked(const GdnArgs a
       for (int p = 0; p < 4; ++p)
 #pragma unroll
         for (int q = 0; q < 4; ++q) pu[p][q] = 0.0f;
+      // four j at a time: P's entries past a row's own token are zero, and
+      // the rows of A and U hold 64 columns and 64 rows
       const int jmax = min(rt[3], cn - 1);     // the tile's last token row
-      for (int j = 0; j <= jmax; ++j) {
-        float pv[4], uv[4];
+      const int vi = min(4 * ti, RP - 4);      // this tile's four value columns of U
+      for (int j = 0; j <= jmax; j += 4) {
+        float4 pv[4], uv[4];
 #pragma unroll
-        for (int p = 0; p < 4; ++p) pv[p] = A[rt[p] * CP + j];
+        for (int p = 0; p < 4; ++p) pv[p] = *reinterpret_cast<const float4*>(A + rt[p] * CP + j);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) uv[q] = Vc[j * rn + ri[q]];
+        for (int jj = 0; jj < 4; ++jj) uv[jj] = *reinterpret_cast<const float4*>(Vc + (j + jj) * RP + vi);
 #pragma unroll
-        for (int p = 0; p < 4; ++p)
+        for (int p = 0; p < 4; ++p) {
+          const float pj[4] = {pv[p].x, pv[p].y, pv[p].z, pv[p].w};
 #pragma unroll
-          for (int q = 0; q < 4; ++q) pu[p][q] = fmaf(pv[p], uv[q], pu[p][q]);
+          for (int jj = 0; jj < 4; ++jj) {
+            pu[p][0] = fmaf(pj[jj], uv[jj].x, pu[p][0]);
+            pu[p][1] = fmaf(pj[jj], uv[jj].y, pu[p][1]);
+            pu[p][2] = fmaf(pj[jj], uv[jj].z, pu[p][2]);
+            pu[p][3] = fmaf(pj[jj], uv[jj].w, pu[p][3]);
+          }
+        }
       }
 #pragma unroll
       for (int p = 0; p < 4; ++p)
@@ -257,35 +291,40 @@ __global__ void __launch_bounds__(gdn::THREADS, 1) k_gdn_chunked(const GdnArgs a
     const float gc = G[cn - 1];
     if (tid < C) W[tid] = tid < cn ? expf(gc - G[tid]) : 0.0f;
     __syncthreads();   // every output of the chunk read the old state; W is ready
-    // S = e^{G_C} S_0 + sum_t e^{G_C - G_t} U_t k_t^T
+    // S = e^{G_C} S_0 + sum_t e^{G_C - G_t} U_t k_t^T: a thread updates 4
+    // value rows x 8 consecutive key columns (float4 loads of U, K and S)
     const float ec = expf(gc);
-    for (int tile = tid; tile < 32 * ni; tile += THREADS) {
-      const int tj = tile % 32, ti = tile / 32;
-      int ri[4];
+    for (int tile = tid; tile < 16 * ni; tile += THREADS) {
+      const int tj = tile % 16, ti = tile / 16;
+      const int c0k = 8 * tj;
+      float acc[4][8];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) ri[k] = min(4 * ti + k, rn - 1);
-      float acc[4][4];
-#pragma unroll
-      for (int p = 0; p < 4; ++p)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[p][q] = ec * S[ri[p] * LD + tj + 32 * q];
+      for (int p = 0; p < 4; ++p) {
+        const float4 lo = *reinterpret_cast<const float4*>(S + (4 * ti + p) * LD + c0k);
+        const float4 hi = *reinterpret_cast<const float4*>(S + (4 * ti + p) * LD + c0k + 4);
+        acc[p][0] = ec * lo.x; acc[p][1] = ec * lo.y; acc[p][2] = ec * lo.z; acc[p][3] = ec * lo.w;
+        acc[p][4] = ec * hi.x; acc[p][5] = ec * hi.y; acc[p][6] = ec * hi.z; acc[p][7] = ec * hi.w;
+      }
       for (int t = 0; t < cn; ++t) {
         const float w = W[t];
-        float uv[4], kv[4];
-#pragma unroll
-        for (int p = 0; p < 4; ++p) uv[p] = Vc[t * rn + ri[p]] * w;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) kv[q] = Kc[t * LD + tj + 32 * q];
+        const float4 u = *reinterpret_cast<const float4*>(Vc + t * RP + 4 * ti);
+        const float4 k0 = *reinterpret_cast<const float4*>(Kc + t * LD + c0k);
+        const float4 k1 = *reinterpret_cast<const float4*>(Kc + t * LD + c0k + 4);
+        const float uv[4] = {u.x * w, u.y * w, u.z * w, u.w * w};
+        const float kv[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
 #pragma unroll
         for (int p = 0; p < 4; ++p)
 #pragma unroll
-          for (int q = 0; q < 4; ++q) acc[p][q] = fmaf(uv[p], kv[q], acc[p][q]);
+          for (int q = 0; q < 8; ++q) acc[p][q] = fmaf(uv[p], kv[q], acc[p][q]);
       }
 #pragma unroll
       for (int p = 0; p < 4; ++p)
-        if (4 * ti + p < rn)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) S[(4 * ti + p) * LD + tj + 32 * q] = acc[p][q];
+        if (4 * ti + p < rn) {
+          *reinterpret_cast<float4*>(S + (4 * ti + p) * LD + c0k) =
+              make_float4(acc[p][0], acc[p][1], acc[p][2], acc[p][3]);
+          *reinterpret_cast<float4*>(S + (4 * ti + p) * LD + c0k + 4) =
+              make_float4(acc[p][4], acc[p][5], acc[p][6], acc[p][7]);
+        }
     }
   }
   __syncthreads();
