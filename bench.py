@@ -156,7 +156,7 @@ def source_digest():
     """Digest of the kernel sources' code (comments do not count): a profile's
     counters apply while this matches the digest recorded with them."""
     h = hashlib.sha256()
-    for f in ("ptx.cuh", "gemm.cuh", "quantize.cuh", "api.cu"):
+    for f in ("ptx.cuh", "gemm.cuh", "quantize.cuh", "gdn.cuh", "api.cu"):
         text = open(os.path.join(ROOT, "nvfp4_w4a4_quantized_quantizer_b200", "csrc", f)).read()
         h.update(_code_only(text).encode())
     return h.hexdigest()[:16]
@@ -499,12 +499,15 @@ def kv_fp8_rate(device, stream):
 FP32_ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
-def gdn_rate(device, stream):
-    """The gated delta rule over 8192 tokens of the GDN in-projection's heads
-    (48 value heads over 16 key heads, width 128), graph replay.  FLOPs
-    counted as the definition's 6 D^2 per token and value head."""
+GDN_T, GDN_HV, GDN_GROUP, GDN_D = 8192, 48, 3, 128
+
+
+def gdn_problem(device):
+    """Inputs of the gated delta rule over 8192 tokens of the GDN
+    in-projection's heads (48 value heads over 16 key heads, width 128) and
+    a launch function fn(i, stream)."""
     import nvfp4_w4a4_quantized_quantizer_b200 as nv
-    T, Hv, group, D = 8192, 48, 3, 128
+    T, Hv, group, D = GDN_T, GDN_HV, GDN_GROUP, GDN_D
     rng = np.random.default_rng(4)
     f = lambda a: torch.from_numpy(a.astype(np.float32)).to(device)  # noqa: E731
     k = rng.standard_normal((T, Hv // group, D))
@@ -519,7 +522,14 @@ def gdn_rate(device, stream):
     def run(i, st):
         nv.nvfp4_gdn_recurrence(ins["q"], ins["k"], ins["v"], ins["g"], ins["beta"], group=group,
                                 state=state, o=o, stream=st)
+    return run
 
+
+def gdn_rate(device, stream):
+    """The gated delta rule (gdn_problem), graph replay.  FLOPs counted as
+    the definition's 6 D^2 per token and value head."""
+    T, Hv, D = GDN_T, GDN_HV, GDN_D
+    run = gdn_problem(device)
     t = time_each({"gdn": run}, stream)["gdn"]
     tflops = 6.0 * D * D * T * Hv / (t * 1e-3) / 1e12
     return {"tokens": T, "value_heads": Hv, "us": round(t * 1e3, 1),
@@ -716,13 +726,16 @@ KERNEL_CASES = {
     "down_mlp": "k_gemm_tc<2> on the 16384 x 17408 x 5120 MLP down projection",
     "decode_m1": "k_gemm_small<16> on the GDN in-projection weights, 1 token",
     "decode_m64": "k_gemm_small<64> on the GDN in-projection weights, 64 tokens",
+    "gdn_recurrence": "k_gdn_chunked, the gated delta rule over 8192 tokens x 48 value heads",
 }
 
 
 def kernel_case(name: str, launches: int, device):
     import nvfp4_w4a4_quantized_quantizer_b200 as nv
     st = torch.cuda.current_stream()
-    if name in ("gate_up_mlp", "down_mlp"):
+    if name == "gdn_recurrence":
+        fn = gdn_problem(device)
+    elif name in ("gate_up_mlp", "down_mlp"):
         ch = MlpChain(device, rotate_act=1, rotate_w=1)
         ch.quantize(0, st)
         if name == "down_mlp":
@@ -767,7 +780,7 @@ def main():
                     help="launch one kernel of one configuration a few times (profiler captures)")
     ap.add_argument("--launches", type=int, default=3)
     ap.add_argument("--no-overlap", action="store_true",
-                    help="launch the quantiser and the small-M GEMM without launch overlap")
+                    help="launch the quantiser and the GEMMs without launch overlap")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -841,7 +854,7 @@ def main():
                    "l2": f"inputs rotated over {len(layer.xs)} activation / {len(layer.ws)} weight copies "
                          "(working set > L2)", "parallelism": f"replicas x{ws}",
                    "launch": f"steps replayed from CUDA graphs of {GRAPH_STEPS} steps; launch overlap "
-                             + ("off" if args.no_overlap else "on (quantiser, small-M GEMM)")},
+                             + ("off" if args.no_overlap else "on (quantiser and GEMMs)")},
         "roofline": {"bound": "tensor", "kernel": g_name, "achieved": round(g_tflops, 1),
                      "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(g_tflops / fp4_peak, 4),
                      "traffic": traffic,
