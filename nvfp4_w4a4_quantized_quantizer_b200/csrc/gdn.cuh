@@ -21,7 +21,7 @@
 //
 // k_gdn_chunked: one CTA per (value head, block of value rows); the fp32
 // state rows and one chunk's keys, queries and value columns stay in shared
-// memory (at most 187 KB); fp32 CUDA-core arithmetic with register tiles fed
+// memory (at most 191 KB); fp32 CUDA-core arithmetic with register tiles fed
 // by 128-bit shared loads.  The products are dense and would belong on the
 // tensor cores.
 #pragma once
@@ -39,7 +39,7 @@ constexpr int D = 128;         // key and value head width
 constexpr int LD = D + 4;
 constexpr int CP = C + 4;      // padded rows of A: 16-byte aligned, 17 bank groups apart
 constexpr int THREADS = 256;
-constexpr int SMEM_FLOATS = D * LD + 2 * C * LD + C * D + C * CP + 4 * C;
+constexpr int SMEM_FLOATS = D * LD + 2 * C * LD + C * D + C * CP + 4 * C + C * 16;
 constexpr int SMEM_BYTES = SMEM_FLOATS * 4;
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 }  // namespace gdn
@@ -99,6 +99,7 @@ __global__ void __launch_bounds__(gdn::THREADS, 1) k_gdn_chunked(const GdnArgs a
   float* B = G + C;                 // [C] beta
   float* E = B + C;                 // [C] e^{G_t}
   float* W = E + C;                 // [C] e^{G_last - G_t}
+  float* Ti = W + C;                // [C / 16][16][16] inverses of the 16 x 16 diagonal blocks of I + A
   const int h = blockIdx.x / a.parts;          // value head
   const int r0 = (blockIdx.x % a.parts) * a.rows;
   const int rn = min(D, r0 + a.rows) - r0;      // this CTA's value rows [r0, r0 + rn)
@@ -191,12 +192,31 @@ __global__ void __launch_bounds__(gdn::THREADS, 1) k_gdn_chunked(const GdnArgs a
         }
     }
     __syncthreads();
-    // (I + A) U = rhs by forward substitution in 16-row blocks: the terms
-    // of the rows solved in earlier blocks are one product computed by all
-    // threads, then the block's own rows are solved column by column
-    // (thread i, column i).  Rows past cn have zero right-hand sides and
-    // zero rows of A.
+    // (I + A) U = rhs in 16-row blocks.  The diagonal blocks of I + A are
+    // unit lower triangular and depend on A alone: their inverses are
+    // formed once per chunk (one column per thread, 64 threads).  Then for
+    // each block: the terms of the rows solved in earlier blocks (one
+    // product over all threads), and the block's rows as its inverse times
+    // that residual.  Rows past cn have zero right-hand sides and zero rows
+    // of A.
+    if (tid < C) {
+      const int b = tid >> 4, c = tid & 15;
+      const float* Ab = A + (16 * b) * CP + 16 * b;      // the diagonal block
+      float x[16];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        float v = r == c ? 1.0f : 0.0f;
+#pragma unroll
+        for (int j = 0; j < r; ++j)
+          if (j >= c) v = fmaf(-Ab[r * CP + j], x[j], v);
+        x[r] = r < c ? 0.0f : v;
+      }
+#pragma unroll
+      for (int r = 0; r < 16; ++r) Ti[(b * 16 + r) * 16 + c] = x[r];
+    }
+    __syncthreads();
     for (int t0 = 0; t0 < cn; t0 += 16) {
+      constexpr int PER = (16 * D + THREADS - 1) / THREADS;   // outputs per thread, at most
       if (t0 > 0) {
         for (int x = tid; x < 16 * rn; x += THREADS) {
           const int t = t0 + x / rn, i = x - (x / rn) * rn;
@@ -210,15 +230,24 @@ __global__ void __launch_bounds__(gdn::THREADS, 1) k_gdn_chunked(const GdnArgs a
         }
         __syncthreads();
       }
-      if (tid < rn) {
-        const int i = tid;
-        const int t1 = min(t0 + 16, cn);
-        for (int t = t0 + 1; t < t1; ++t) {
-          const float* At = A + t * CP;
-          float s = 0.0f;
-          for (int j = t0; j < t; ++j) s = fmaf(At[j], Vc[j * RP + i], s);
-          Vc[t * RP + i] -= s;
+      const float* Tb = Ti + (t0 / 16) * 256;
+      float u[PER];
+#pragma unroll
+      for (int k = 0; k < PER; ++k) {
+        const int x = tid + k * THREADS;
+        u[k] = 0.0f;
+        if (x < 16 * rn) {
+          const int r = x / rn, i = x - r * rn;
+          float acc = 0.0f;
+          for (int c = 0; c <= r; ++c) acc = fmaf(Tb[r * 16 + c], Vc[(t0 + c) * RP + i], acc);
+          u[k] = acc;
         }
+      }
+      __syncthreads();   // the block's residual rows are read
+#pragma unroll
+      for (int k = 0; k < PER; ++k) {
+        const int x = tid + k * THREADS;
+        if (x < 16 * rn) Vc[(t0 + x / rn) * RP + x % rn] = u[k];
       }
       __syncthreads();
     }
