@@ -7,10 +7,16 @@ stated in include/nvfp4.h.
 """
 from __future__ import annotations
 
+import os
+
 import numpy as np
 import torch
 
 import workloads
+
+# NVFP4_TEST_LAUNCH_OVERLAP=1 runs the whole suite with launch overlap on;
+# tests that switch it restore this default.
+LAUNCH_OVERLAP_DEFAULT = os.environ.get("NVFP4_TEST_LAUNCH_OVERLAP") == "1"
 
 
 # ------------------------------------------------------------------ layouts

@@ -13,6 +13,16 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "slow: full-size workloads (minutes)")
 
 
+@pytest.fixture(scope="session", autouse=True)
+def _launch_overlap_default():
+    """With NVFP4_TEST_LAUNCH_OVERLAP=1 every GPU test runs with launch overlap on."""
+    from tests import _helpers as H
+    if H.LAUNCH_OVERLAP_DEFAULT:
+        import nvfp4_w4a4_quantized_quantizer_b200 as nv
+        nv.nvfp4_set_launch_overlap(True)
+    yield
+
+
 def pytest_collection_modifyitems(config, items):
     try:
         import torch

@@ -180,6 +180,8 @@ def test_misc_validation(lib):
     assert lib.nvfp4_set_launch_overlap(2) == INVALID
     assert lib.nvfp4_set_launch_overlap(1) == 0
     assert lib.nvfp4_set_launch_overlap(0) == 0
+    # back to the suite's default (NVFP4_TEST_LAUNCH_OVERLAP)
+    lib.nvfp4_set_launch_overlap(1 if os.environ.get("NVFP4_TEST_LAUNCH_OVERLAP") == "1" else 0)
     assert lib.nvfp4_silu_mul(P, 4, 12, 24, P, 12, NUL) == SHAPE       # H % 8
     assert lib.nvfp4_amax(P, 4, 64, 64, NUL, NUL) == INVALID
     assert lib.nvfp4_test_e2m1(NUL, P, 4, NUL) == INVALID

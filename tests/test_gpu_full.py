@@ -155,7 +155,7 @@ def test_decode_sweep_full(M):
     try:
         _check_layer(workloads.WORKLOADS[5], M, M, 256, seed=50 + M)
     finally:
-        nv.nvfp4_set_launch_overlap(False)
+        nv.nvfp4_set_launch_overlap(H.LAUNCH_OVERLAP_DEFAULT)
 
 
 def test_mlp_pair_full():

@@ -208,7 +208,7 @@ def test_bf16_row_stride_both_store_widths(ldy, path):
 def overlap():
     nv.nvfp4_set_launch_overlap(True)
     yield
-    nv.nvfp4_set_launch_overlap(False)
+    nv.nvfp4_set_launch_overlap(H.LAUNCH_OVERLAP_DEFAULT)
 
 
 def _decode_layer(M, N, K, seed):
